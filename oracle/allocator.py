@@ -1,0 +1,116 @@
+"""Reference block manager for the paged KV cache (test infrastructure only).
+
+Written from the pages' description of the host side of PagedAttention:
+
+- "PagedAttention" glossary entry (ultralytics.com), section "Como funciona la
+  paginacion": a request receives a new block only when its previous one is
+  full, from any free location, and its block table records the order.  The
+  worked example pops blocks from the front of a free list ([41, 7, 19, 2, 33])
+  and stores token `pos` at (block_table[pos // block_size], pos % block_size).
+- same page, "Compartir bloques entre secuencias": sequences may point at the
+  same physical blocks, counted by a per-block reference count; a sequence that
+  must write into a block others still use first copies it (copy-on-write).
+- iplexlaw.co.kr blog, sections on logical vs physical order and "two answers
+  to one request": the prompt is allocated first, then the last block is filled,
+  and a new block is added only when needed; full shared blocks stay shared,
+  only the block that must split is copied; blocks with no references are freed.
+- same glossary page, "Tecnicas relacionadas" (continuous batching): a finished
+  sequence's blocks return to the free pool at once.
+
+Readings where the pages are silent: the free list is first-in first-out (pop
+from the front, freed blocks appended to the back in table order); a
+copy-on-write copies the whole block and moves the writer to the copy, leaving
+the last holder (reference count 1) to write in place; running out of free
+blocks raises MemoryError and leaves the state unchanged.
+"""
+from collections import deque
+
+
+class RefBlockManager:
+    def __init__(self, num_blocks, block_size, free_order=None):
+        if free_order is None:
+            free_order = range(num_blocks)
+        free_order = [int(b) for b in free_order]
+        # A free list may name only some blocks (the rest are owned elsewhere,
+        # as in the worked example's five free blocks of a 64-block pool).
+        assert len(set(free_order)) == len(free_order), "a block may be free only once"
+        assert all(0 <= b < num_blocks for b in free_order), "block id out of range"
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+        self.free = deque(free_order)
+        self.ref = [0] * num_blocks
+        self.tables = {}
+        self.lens = {}
+        self._next = 0
+
+    # -- allocation ---------------------------------------------------------
+    def _pop(self):
+        if not self.free:
+            raise MemoryError("no free block")
+        b = self.free.popleft()
+        assert self.ref[b] == 0
+        self.ref[b] = 1
+        return b
+
+    def alloc_seq(self, num_tokens):
+        """New sequence holding `num_tokens` prompt tokens: ceil(n / bs) blocks."""
+        need = -(-num_tokens // self.block_size)
+        if need > len(self.free):
+            raise MemoryError("not enough free blocks")
+        seq = self._next
+        self._next += 1
+        self.tables[seq] = [self._pop() for _ in range(need)]
+        self.lens[seq] = num_tokens
+        return seq
+
+    def fork(self, parent):
+        """New sequence sharing every block of `parent` (reference counts + 1)."""
+        seq = self._next
+        self._next += 1
+        self.tables[seq] = list(self.tables[parent])
+        self.lens[seq] = self.lens[parent]
+        for b in self.tables[seq]:
+            self.ref[b] += 1
+        return seq
+
+    def append_token(self, seq):
+        """Reserve the slot of the sequence's next token.
+
+        Returns (slot, cow) where cow is None or the (src, dst) block pair that
+        must be copied before the token is written.
+        """
+        n = self.lens[seq]
+        table = self.tables[seq]
+        cow = None
+        if n % self.block_size == 0:
+            # last block full (or no block yet): a fresh block, nothing to copy
+            table.append(self._pop())
+        else:
+            last = table[-1]
+            if self.ref[last] > 1:
+                new = self._pop()
+                self.ref[last] -= 1
+                table[-1] = new
+                cow = (last, new)
+        slot = table[n // self.block_size] * self.block_size + n % self.block_size
+        self.lens[seq] = n + 1
+        return slot, cow
+
+    def free_seq(self, seq):
+        """Drop a finished sequence; blocks whose count reaches 0 return to the pool."""
+        for b in self.tables.pop(seq):
+            self.ref[b] -= 1
+            if self.ref[b] == 0:
+                self.free.append(b)
+        del self.lens[seq]
+
+    # -- queries ------------------------------------------------------------
+    def slot(self, seq, pos):
+        t = self.tables[seq]
+        return t[pos // self.block_size] * self.block_size + pos % self.block_size
+
+    def slots(self, seq, start, count):
+        return [self.slot(seq, p) for p in range(start, start + count)]
+
+    def num_free(self):
+        return len(self.free)

@@ -1,0 +1,134 @@
+"""Planted mistakes: each mutant is a copy of the oracle with one plausible bug
+(a dropped term, a wrong sign or index, a transposed operand), built on the CPU
+in a temporary directory.  The pin suite must reject every one of them.
+
+The mutants never touch the committed oracle; they are compiled from edited
+copies of its source and loaded in place of it for the duration of one check.
+"""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+import tests.test_allocator_ref as A
+import tests.test_oracle_pins as P
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
+
+MUTANTS = {
+    "gqa_head_mapping": ("int g = h / group;", "int g = h % num_kv_heads;"),
+    "dropped_scale": ("scores[t - t0] = scale * dot;", "scores[t - t0] = dot;"),
+    "slot_offset": ("(size_t)(t % block_size)) * num_kv_heads + g)",
+                    "(size_t)((t + 1) % block_size)) * num_kv_heads + g)"),
+    "table_index": ("int32_t blk = table[t / block_size];\n    if (blk < 0 || blk >= num_blocks) return 0;",
+                    "int32_t blk = table[t % block_size];\n    if (blk < 0 || blk >= num_blocks) return 0;"),
+    "keys_from_value_pool": ("dot += qv[d] * (load_elem(k_pool,", "dot += qv[d] * (load_elem(v_pool,"),
+    "exp_sign": ("w = exp(scores[t - t0] - m);", "w = exp(m - scores[t - t0]);"),
+    "merge_drops_l": ("w = pl[p] * exp(pm[p] - M);", "w = exp(pm[p] - M);"),
+    "v_scale_for_k": ("* k_scale)", "* v_scale)"),
+    "e4m3_bias": ("ldexp(1.0 + (double)m / 8.0, e - 7)", "ldexp(1.0 + (double)m / 8.0, e - 8)"),
+    "e4m3_subnormal": ("ldexp((double)m / 8.0, -6)", "ldexp((double)m / 8.0, -7)"),
+    "e4m3_ties_odd": ("(a == mid && (c & 1))", "(a == mid && !(c & 1))"),
+    "e4m3_no_saturation": ("if (a >= 448.0) return (uint8_t)(sign | 0x7E);",
+                           "if (a >= 464.0) return (uint8_t)(sign | 0x7F);"),
+    "write_v_with_k_scale": ("load_src_float(v, src_dtype, (size_t)i * row + e), v_scale)",
+                             "load_src_float(v, src_dtype, (size_t)i * row + e), k_scale)"),
+    "write_slot_row": ("(char*)k_pool + (size_t)slot * row * es", "(char*)k_pool + (size_t)(slot + 1) * row * es"),
+    "copy_only_k": ("memcpy((char*)v_pool + (size_t)d * block_bytes", "if (0) memcpy((char*)v_pool + (size_t)d * block_bytes"),
+    "gather_wrong_slot": ("((size_t)blk * block_size + (size_t)(t % block_size)) * row_bytes, row_bytes);",
+                          "((size_t)blk * block_size + (size_t)(t / block_size)) * row_bytes, row_bytes);"),
+}
+
+def _pins(golden):
+    """Every pin, as callables that raise when the oracle is wrong."""
+    fns = [
+        lambda: P.test_worked_example(golden),
+        P.test_len_one_returns_v0_exactly, P.test_zero_query_gives_mean_of_v,
+        P.test_equal_keys_give_mean_of_v, P.test_constant_values_give_that_row,
+        P.test_two_tokens_logistic, P.test_empty_context_is_zero,
+        lambda: [P.test_paged_equals_contiguous(*a) for a in [(2, 2, 64), (8, 2, 64), (16, 2, 128)]],
+        P.test_bf16_paged_equals_contiguous, P.test_fp8_paged_equals_dequantised_contiguous,
+        P.test_gqa_equals_mha_with_repeated_kv_heads, P.test_placement_permutation_is_bitwise_invariant,
+        lambda: [P.test_partitioned_merge_equals_single_pass(p) for p in (16, 48, 112)],
+        P.test_stale_slots_are_not_read, P.test_invalid_block_ids_are_skipped_and_counted,
+        P.test_shared_prefix_reads_identical_kv_until_cow,
+        P.test_e4m3_decode_all_codes_match_library, P.test_e4m3_format_landmarks,
+        P.test_e4m3_encode_matches_brute_force_sweep,
+        P.test_kv_write_bf16_is_raw_copy_and_touches_nothing_else,
+        P.test_kv_write_fp8_matches_library_cast, P.test_copy_blocks_semantics,
+    ]
+    return fns
+
+
+def _build_mutant(tmp, name, old, new):
+    src = open(SRC).read()
+    assert src.count(old) >= 1, "mutation anchor not found: %s" % name
+    path_c = os.path.join(tmp, name + ".c")
+    path_so = os.path.join(tmp, name + ".so")
+    open(path_c, "w").write(src.replace(old, new))
+    subprocess.run(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+                    path_c, "-o", path_so, "-lm"], check=True)
+    return path_so
+
+
+def _load_like_oracle(path):
+    saved = oracle._lib
+    oracle._lib = None
+    real_build = oracle._build.build
+    oracle._build.build = lambda force=False: path
+    try:
+        L = oracle.lib()
+    finally:
+        oracle._build.build = real_build
+        oracle._lib = saved
+    return L
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_reject_planted_mistake(name, golden_dir, tmp_path):
+    old, new = MUTANTS[name]
+    path = _build_mutant(str(tmp_path), name, old, new)
+    mutant = _load_like_oracle(path)
+    saved = oracle._lib
+    oracle._lib = mutant
+    caught = []
+    try:
+        for fn in _pins(golden_dir):
+            try:
+                fn()
+            except Exception as e:  # noqa: BLE001 - any failure counts as a catch
+                caught.append(repr(e)[:80])
+                break
+    finally:
+        oracle._lib = saved
+    assert caught, "no pin caught the planted mistake %s" % name
+
+
+def test_pins_reject_allocator_copying_for_last_holder(monkeypatch):
+    """Planted mistake in the reference block manager: copy-on-write even when
+    the writer is the block's last holder."""
+    from oracle import allocator
+
+    def bad_append(self, seq):
+        n = self.lens[seq]
+        table = self.tables[seq]
+        cow = None
+        if n % self.block_size == 0:
+            table.append(self._pop())
+        else:
+            last = table[-1]
+            if self.ref[last] >= 1:      # the planted mistake
+                new = self._pop()
+                self.ref[last] -= 1
+                if self.ref[last] == 0:
+                    self.free.append(last)
+                table[-1] = new
+                cow = (last, new)
+        slot = table[n // self.block_size] * self.block_size + n % self.block_size
+        self.lens[seq] = n + 1
+        return slot, cow
+
+    monkeypatch.setattr(allocator.RefBlockManager, "append_token", bad_append)
+    with pytest.raises(AssertionError):
+        A.test_parallel_sampling_cow_trace()
