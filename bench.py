@@ -1,0 +1,524 @@
+"""Benchmark of the paged KV-cache decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gqa70b]
+                    [--impl ours|reference] [--partition P]
+
+A step is one pass of the hot path over one batch: the KV write of every
+sequence's new token (plus the copy-on-write block copies for the shared-prefix
+workload), then paged decode attention over every context.  The default
+workload is the Llama-3.1-70B-shaped GQA batch (256 sequences x 4,096 tokens,
+64 query / 8 KV heads, head_dim 128, bf16).  The KV pools (5 GiB) exceed the
+126 MB L2, so every step streams the cache from HBM.
+
+Metric: effective KV bytes read per second (sum over sequences of
+len * kv_heads * head_dim * 2 (K, V) * element size, divided by the step time);
+also sequence-tokens per second and microseconds per step.
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own batch of the
+same shape (independent sequences, no collective on the data path); the time is
+the max over ranks and the value the sum over ranks (weak scaling).
+
+--impl reference times the CPU oracle (the plain fp64 reference) on a bounded
+sample of the same workload, on this host's cores.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "paged decode attention: effective KV HBM GB/s (% of B200 peak); seq-tokens/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+DESCR = {
+    "gqa70b": "Llama-3.1-70B-shaped GQA decode: 64 q / 8 kv heads, head_dim 128, bf16, 256 seqs x 4096 tokens, "
+              "block 16, one new token per sequence",
+    "mha13b": "LLaMA-13B-shaped MHA decode: 40 heads, head_dim 128, bf16, 64 seqs, lengths U[128, 2048], block 16",
+    "shared_prefix": "shared-prefix parallel sampling: 64 prompts x n=3, 1000-token prefix + U{0..512}, GQA 32/8, "
+                     "head_dim 128, bf16, copy-on-write + write + decode per step",
+    "fp8_long": "FP8 E4M3 cache, GQA 32/8, head_dim 128, 128 seqs, lengths log-U[256, 32768], write + split decode",
+}
+
+
+# ------------------------------------------------------------------ distributed helpers
+
+def dist_env():
+    """(rank, world, local_rank) from the torchrun environment (1 process by default)."""
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Max of a float over all ranks (the job's time is its slowest rank's)."""
+    if world <= 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_workload(w: W.Workload, rank: int) -> W.Workload:
+    """Weak scaling: each rank gets an independent batch of the same shape (its own seed)."""
+    return W.scaled(w, seed=w.seed + 1000 * rank) if rank else w
+
+
+# ------------------------------------------------------------------ measurement helpers
+
+def measured_peak_hbm():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:  # noqa: BLE001 - absent or unreadable: the pool's earlier figure
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("decode_tc.cu", "pkv_common.cuh", "decode_plan.cu"):
+        with open(os.path.join(ROOT, "paged_kv_cache_404_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload):
+    """DRAM bytes per decode launch from a committed ncu capture, if it was taken
+    on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(workload)
+    except Exception:  # noqa: BLE001
+        return None
+    if not rec or rec.get("source_hash") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi SM clock / throttle-reason samples during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.Q,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:  # noqa: BLE001 - no nvidia-smi: no clock record
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ workload set-up (product side)
+
+class Step:
+    """Device-resident inputs of one decode step and the calls that run it."""
+
+    def __init__(self, w: W.Workload, device, partition=0):
+        import paged_kv_cache_404_b200 as pkv
+        self.pkv = pkv
+        self.w = w
+        self.device = device
+        self.partition = partition
+        if w.lens == "shared":
+            self._setup_shared()
+        else:
+            self._setup_flat()
+        self.max_len = int(self.lens.max())
+        self.g_slots = torch.from_numpy(self.slots).to(device)
+        self.g_tables = torch.from_numpy(self.tables).to(device)
+        self.g_lens = torch.from_numpy(self.lens).to(device)
+        self.g_pairs = torch.from_numpy(self.pairs).to(device) if len(self.pairs) else None
+        self.ws = pkv.decode_workspace(self.S, w.num_heads, w.head_dim, self.max_len, partition, device=device)
+        self.out = torch.empty_like(self.q)
+        self.err = torch.zeros(1, dtype=torch.int32, device=device)
+        elem = 1 if w.cache_dtype == "fp8" else 2
+        self.kv_bytes = int(self.lens.astype(np.int64).sum()) * w.num_kv_heads * w.head_dim * 2 * elem
+        self.seq_tokens = int(self.lens.astype(np.int64).sum())
+        # write + plan + decode (+ merge when a split is possible) (+ copy-on-write copy)
+        merge = (partition or 256) < self.max_len
+        self.launches = 3 + int(merge) + int(self.g_pairs is not None)
+
+    def _setup_flat(self):
+        pkv, w, dev = self.pkv, self.w, self.device
+        lens = W.context_lens(w)
+        self.S = len(lens)
+        need = int(sum(-(-int(L) // 16) for L in lens))
+        NB = W.pool_blocks(w, need)
+        bm = pkv.BlockManager(NB, 16, free_order=W.free_order(w, NB))
+        ids = [bm.alloc_seq(int(L) - 1) for L in lens]
+        slots, pairs = bm.append_tokens(ids)
+        self.slots, self.pairs = slots, pairs
+        self.tables, self.lens = bm.tables(ids, max(-(-int(L) // 16) for L in lens), pad=-1)
+        self.k_pool, self.v_pool, self.k_scale, self.v_scale = W.random_pools(w, NB, dev)
+        self.q = W.queries(w, self.S, dev)
+        self.k_new, self.v_new = W.new_tokens(w, self.S, dev)
+        self.NB = NB
+
+    def _setup_shared(self):
+        """Prompts written once and forked; continuations replayed token by token
+        (copy-on-write on first divergence); the step is the next token of all."""
+        pkv, w, dev = self.pkv, self.w, self.device
+        cont = W.continuation_lens(w)
+        S = self.S = w.num_prompts * w.samples
+        est = w.num_prompts * (-(-w.prefix_len // 16)) + int(sum(-(-(int(c) + 17) // 16) for c in cont)) + S
+        NB = int(math.ceil(est * w.pool_factor))
+        bm = pkv.BlockManager(NB, 16, free_order=W.free_order(w, NB))
+        kp, vp = W.stale_fill(w, NB, dev)
+        pk, pv = W.logical_kv(w, w.num_prompts * w.prefix_len, dev, stream=50)
+        ck, cv = W.logical_kv(w, int(cont.sum()) + 1, dev, stream=60)
+        ids = []
+        for p in range(w.num_prompts):
+            parent = bm.alloc_seq(w.prefix_len)
+            sl = slice(p * w.prefix_len, (p + 1) * w.prefix_len)
+            pkv.paged_kv_write(pk[sl], pv[sl], torch.from_numpy(bm.slots(parent, 0, w.prefix_len)).to(dev), kp, vp)
+            ids += [parent] + [bm.fork(parent) for _ in range(w.samples - 1)]
+        cur = 0
+        for t in range(int(cont.max())):
+            act = [ids[i] for i in range(S) if cont[i] > t]
+            slots, pairs = bm.append_tokens(act)
+            if len(pairs):
+                pkv.copy_blocks(kp, vp, torch.from_numpy(pairs).to(dev))
+            pkv.paged_kv_write(ck[cur:cur + len(act)], cv[cur:cur + len(act)], torch.from_numpy(slots).to(dev), kp, vp)
+            cur += len(act)
+        self.slots, self.pairs = bm.append_tokens(ids)
+        self.tables, self.lens = bm.tables(ids, max(-(-int(bm.seq_len(s)) // 16) for s in ids), pad=-1)
+        self.k_pool, self.v_pool, self.k_scale, self.v_scale = kp, vp, 1.0, 1.0
+        self.q = W.queries(w, S, dev)
+        self.k_new, self.v_new = W.new_tokens(w, S, dev)
+        self.NB = NB
+        torch.cuda.synchronize()
+
+    def copy_and_write(self):
+        if self.g_pairs is not None:
+            self.pkv.copy_blocks(self.k_pool, self.v_pool, self.g_pairs, err_count=self.err)
+        self.pkv.paged_kv_write(self.k_new, self.v_new, self.g_slots, self.k_pool, self.v_pool, self.k_scale,
+                                self.v_scale, err_count=self.err)
+
+    def decode(self):
+        self.pkv.paged_attention_decode(self.out, self.q, self.k_pool, self.v_pool, self.g_tables, self.g_lens,
+                                        self.w.scale, self.max_len, self.ws, self.k_scale, self.v_scale,
+                                        partition_tokens=self.partition, err_count=self.err)
+
+    def run(self):
+        self.copy_and_write()
+        self.decode()
+
+
+def time_steps(step: Step, steps: int, warmup: int, world: int, device):
+    """K timed steps between a barrier + synchronize on both sides; the step and
+    the decode call inside it are timed with CUDA events on the launching stream."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        step.run()
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for a, b, c in ev:
+        a.record(stream)
+        step.copy_and_write()
+        b.record(stream)
+        step.decode()
+        c.record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    total_ms = start.elapsed_time(end)
+    decode_ms = [b.elapsed_time(c) for _, b, c in ev]
+    write_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    return total_ms, decode_ms, write_ms
+
+
+def time_e2e(step: Step, steps: int, warmup: int, world: int):
+    """The same step through the public API from pinned HOST buffers: every step
+    copies its inputs (q, new K/V, slots, tables, lengths, copy pairs) host->device
+    and reads the output back device->host, all inside the timed region."""
+    stream = torch.cuda.current_stream()
+    host = {
+        "q": step.q.cpu().pin_memory(), "k_new": step.k_new.cpu().pin_memory(),
+        "v_new": step.v_new.cpu().pin_memory(), "g_slots": step.g_slots.cpu().pin_memory(),
+        "g_tables": step.g_tables.cpu().pin_memory(), "g_lens": step.g_lens.cpu().pin_memory(),
+    }
+    if step.g_pairs is not None:
+        host["g_pairs"] = step.g_pairs.cpu().pin_memory()
+    out_host = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def one():
+        for name, t in host.items():
+            getattr(step, name).copy_(t, non_blocking=True)
+        step.run()
+        out_host.copy_(step.out, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b), h2d, d2h
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+
+def oracle_sample_step(w: W.Workload, num_seqs: int, seed_offset=0):
+    """Oracle inputs for `num_seqs` sequences of the workload (host, CPU
+    generator): pool, tables, lengths, q and the step's new tokens."""
+    import oracle
+    lens = W.context_lens(w)
+    if w.lens == "shared":
+        lens = (w.prefix_len + W.continuation_lens(w) + 1).astype(np.int32)
+    lens = lens[seed_offset:seed_offset + num_seqs]
+    wn = W.scaled(w, num_seqs=len(lens))
+    need = int(sum(-(-int(L) // 16) for L in lens))
+    NB = need + 1
+    ref = oracle.RefBlockManager(NB, 16, free_order=W.free_order(wn, NB))
+    ids = [ref.alloc_seq(int(L) - 1) for L in lens]
+    slots = [ref.append_token(s)[0] for s in ids]
+    maxb = max(-(-int(L) // 16) for L in lens)
+    tabs = np.full((len(lens), maxb), -1, np.int32)
+    for i, s in enumerate(ids):
+        tabs[i, :len(ref.tables[s])] = ref.tables[s]
+    kp, vp, ks, vs = W.random_pools(wn, NB, "cpu")
+    q = W.queries(wn, len(lens), "cpu")
+    kn, vn = W.new_tokens(wn, len(lens), "cpu")
+    bits = lambda t: t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
+    return dict(oracle=oracle, lens=lens, tabs=tabs, slots=np.array(slots, np.int64), kp=bits(kp).copy(),
+                vp=bits(vp).copy(), ks=ks, vs=vs, q=bits(q), kn=bits(kn), vn=bits(vn), w=wn)
+
+
+def oracle_run(d, threads=0):
+    oracle = d["oracle"]
+    w = d["w"]
+    cdt = {"f32": oracle.F32, "bf16": oracle.BF16, "fp8": oracle.FP8_E4M3}[w.cache_dtype]
+    sdt = oracle.F32 if w.cache_dtype == "f32" else oracle.BF16
+    qdt = oracle.F32 if w.q_dtype == "f32" else oracle.BF16
+    oracle.kv_write(d["kn"], d["vn"], sdt, d["slots"], d["kp"], d["vp"], cdt, 16, d["ks"], d["vs"])
+    oracle.paged_attention_decode(d["q"], qdt, d["kp"], d["vp"], cdt, d["tabs"], d["lens"], w.scale, d["ks"],
+                                  d["vs"], num_threads=threads)
+
+
+def cpu_baseline(w: W.Workload, target_s=12.0):
+    """The oracle as it stands (fp64, OpenMP over (sequence, head), all cores) on
+    a bounded sample of the workload; returns the same metric (KV GB/s)."""
+    import oracle
+    elem = 1 if w.cache_dtype == "fp8" else 2
+    per_tok = w.num_kv_heads * w.head_dim * 2 * elem
+    n = 1
+    d = oracle_sample_step(w, n)
+    t0 = time.perf_counter()
+    oracle_run(d)
+    dt = time.perf_counter() - t0
+    n = int(max(1, min(w.num_seqs, math.floor(target_s / max(dt, 1e-3)))))
+    d = oracle_sample_step(w, n)
+    t0 = time.perf_counter()
+    oracle_run(d)
+    dt = time.perf_counter() - t0
+    toks = int(d["lens"].astype(np.int64).sum())
+    return {"value": round(toks * per_tok / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.max_threads(),
+            "kind": "oracle",
+            "sample": "%d of %d sequences (%d tokens), one write + decode step, fp64, %.2f s" % (
+                n, w.num_seqs, toks, dt),
+            "seq_tokens_per_s": round(toks / dt, 1)}
+
+
+def run_reference(args, w, rank, world):
+    """--impl reference: the CPU oracle, timed on this host, on bounded samples."""
+    if rank != 0:
+        return
+    import oracle
+    elem = 1 if w.cache_dtype == "fp8" else 2
+    per_tok = w.num_kv_heads * w.head_dim * 2 * elem
+    # size one step's sample to about 3 s of CPU work
+    probe = oracle_sample_step(w, 1)
+    t0 = time.perf_counter()
+    oracle_run(probe)
+    dt = time.perf_counter() - t0
+    n = int(max(1, min(w.num_seqs, math.floor(3.0 / max(dt, 1e-3)))))
+    d = oracle_sample_step(w, n)
+    for _ in range(args.warmup):
+        oracle_run(d)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_run(d)
+    total = time.perf_counter() - t0
+    toks = int(d["lens"].astype(np.int64).sum())
+    value = toks * per_tok * args.steps / total / 1e9
+    sample = "%d of %d sequences (%d tokens) per step, fp64 oracle, write + decode" % (n, w.num_seqs, toks)
+    line = {
+        "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "impl": "reference",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload + ": " + DESCR[args.workload], "global_batch": n,
+                   "seq_len": int(d["lens"].max()), "parallelism": "cpu (OpenMP)"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": oracle.max_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "seq_tokens_per_s": round(toks * args.steps / total, 1),
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ main
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="gqa70b", choices=sorted(DESCR))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--partition", type=int, default=0, help="partition tokens (0 = automatic)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)
+
+    rank, world, local = dist_env()
+    w0 = W.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w0, rank, world)
+        return
+
+    from paged_kv_cache_404_b200 import build as pkv_build
+    if rank == 0:
+        pkv_build.build()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+        dist.barrier()
+        pkv_build.build()
+
+    w = rank_workload(w0, rank)
+    step = Step(w, device, partition=args.partition)
+    torch.cuda.synchronize()
+
+    with ClockSampler(local) as clk:
+        total_ms, decode_ms, write_ms = time_steps(step, args.steps, args.warmup, world, device)
+    err = int(step.err.item())
+    max_ms = reduce_max(total_ms, world, device)
+    ms_per_step = max_ms / args.steps
+    bytes_all = step.kv_bytes * world
+    value = bytes_all * args.steps / (max_ms / 1e3) / 1e9
+
+    e2e = None
+    if not args.no_e2e:
+        e_ms, h2d, d2h = time_e2e(step, max(5, args.steps // 2), 3, world)
+        e_ms = reduce_max(e_ms, world, device)
+        e_steps = max(5, args.steps // 2)
+        e2e = {"value": round(bytes_all * e_steps / (e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": round(e_ms / e_steps, 4)}
+
+    peak, peak_kind = measured_peak_hbm()
+    dec_ms = statistics.mean(decode_ms)
+    achieved = step.kv_bytes / (dec_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": ncu_traffic(args.workload),
+                "kernel": "paged_attention_decode call (plan + decode + merge launches)",
+                "peak_source": peak_kind, "frac_of_nominal_8tbps": round(achieved / NOMINAL_HBM_GBS, 4)}
+
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = cpu_baseline(w0)
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp8-e4m3 cache, bf16 q/out, fp32 accumulate" if w.cache_dtype == "fp8" else w.cache_dtype,
+            "data": "synthetic (seeded N(0,1) K/V/q, seeded block placement)",
+            "config": {"workload": args.workload + ": " + DESCR[args.workload], "global_batch": step.S * world,
+                       "seq_len": step.max_len, "parallelism": "replicas: sequences sharded by rank, no collective",
+                       "l2": "inputs larger than L2 (pools %.1f GiB per GPU vs 126 MB L2)" % (
+                           2 * step.k_pool.numel() * step.k_pool.element_size() / 2**30),
+                       "partition_tokens": args.partition or "auto"},
+            "seq_tokens_per_s": round(step.seq_tokens * world * args.steps / (max_ms / 1e3), 1),
+            "us_per_step_per_layer": round(1e3 * ms_per_step, 2),
+            "us_decode": round(1e3 * dec_ms, 2), "us_write": round(1e3 * statistics.mean(write_ms), 2),
+            "pct_of_8tbps": round(100 * value / world / NOMINAL_HBM_GBS, 2),
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": step.launches * args.steps, "device_errors": err,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

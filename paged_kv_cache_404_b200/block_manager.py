@@ -1,0 +1,108 @@
+"""Python face of the native host block manager (pkv_bm_* in pagedkv.h).
+
+The manager itself is C++ (csrc/block_manager.cpp); this class only marshals
+numpy arrays.  It runs on the CPU and needs no GPU.
+"""
+import ctypes as C
+
+import numpy as np
+
+from . import _lib as L
+
+
+class BlockManager:
+    def __init__(self, num_blocks, block_size=16, free_order=None):
+        self._lib = L.lib()
+        h = C.c_void_p()
+        if free_order is None:
+            st = self._lib.pkv_bm_create(num_blocks, block_size, None, 0, C.byref(h))
+        else:
+            fo = np.ascontiguousarray(free_order, dtype=np.int32)
+            st = self._lib.pkv_bm_create(num_blocks, block_size, fo.ctypes.data, fo.size, C.byref(h))
+        L.check("pkv_bm_create", st)
+        self._h = h
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+
+    def close(self):
+        if self._h:
+            self._lib.pkv_bm_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:  # noqa: BLE001 - interpreter shutdown
+            pass
+
+    def alloc_seq(self, num_tokens):
+        out = C.c_int32()
+        L.check("pkv_bm_alloc_seq", self._lib.pkv_bm_alloc_seq(self._h, int(num_tokens), C.byref(out)))
+        return out.value
+
+    def fork(self, parent):
+        out = C.c_int32()
+        L.check("pkv_bm_fork", self._lib.pkv_bm_fork(self._h, int(parent), C.byref(out)))
+        return out.value
+
+    def append_tokens(self, seqs):
+        """One new slot per sequence, in order. Returns (slots int64 [n], cow pairs int64 [k, 2])."""
+        seqs = np.ascontiguousarray(seqs, dtype=np.int32)
+        n = seqs.size
+        slots = np.empty(n, dtype=np.int64)
+        pairs = np.empty((max(n, 1), 2), dtype=np.int64)
+        npairs, ndone = C.c_int(), C.c_int()
+        st = self._lib.pkv_bm_append_tokens(self._h, seqs.ctypes.data, n, slots.ctypes.data, pairs.ctypes.data,
+                                            C.byref(npairs), C.byref(ndone))
+        if st != L.PKV_OK:
+            raise L.PagedKVError("pkv_bm_append_tokens", st)
+        return slots, pairs[:npairs.value].copy()
+
+    def append_token(self, seq):
+        slots, pairs = self.append_tokens([seq])
+        return int(slots[0]), (tuple(int(x) for x in pairs[0]) if len(pairs) else None)
+
+    def free_seq(self, seq):
+        L.check("pkv_bm_free_seq", self._lib.pkv_bm_free_seq(self._h, int(seq)))
+
+    def num_free(self):
+        return self._lib.pkv_bm_num_free(self._h)
+
+    def seq_len(self, seq):
+        out = C.c_int32()
+        L.check("pkv_bm_seq_len", self._lib.pkv_bm_seq_len(self._h, int(seq), C.byref(out)))
+        return out.value
+
+    def refcount(self, block):
+        out = C.c_int32()
+        L.check("pkv_bm_refcount", self._lib.pkv_bm_refcount(self._h, int(block), C.byref(out)))
+        return out.value
+
+    def block_table(self, seq):
+        n = C.c_int()
+        self._lib.pkv_bm_block_table(self._h, int(seq), None, 0, C.byref(n))
+        out = np.empty(max(n.value, 1), dtype=np.int32)
+        L.check("pkv_bm_block_table",
+                self._lib.pkv_bm_block_table(self._h, int(seq), out.ctypes.data, out.size, C.byref(n)))
+        return out[:n.value].copy()
+
+    def slots(self, seq, start, count):
+        out = np.empty(max(count, 1), dtype=np.int64)
+        L.check("pkv_bm_slots", self._lib.pkv_bm_slots(self._h, int(seq), int(start), int(count), out.ctypes.data))
+        return out[:count].copy()
+
+    def tables(self, seqs, max_blocks, pad=-1):
+        """Padded block tables int32 [n, max_blocks] and lengths int32 [n]."""
+        seqs = np.ascontiguousarray(seqs, dtype=np.int32)
+        tab = np.empty((seqs.size, max_blocks), dtype=np.int32)
+        lens = np.empty(seqs.size, dtype=np.int32)
+        L.check("pkv_bm_tables", self._lib.pkv_bm_tables(self._h, seqs.ctypes.data, seqs.size, tab.ctypes.data,
+                                                         int(max_blocks), int(pad), lens.ctypes.data))
+        return tab, lens
+
+    def free_list(self):
+        n = C.c_int()
+        self._lib.pkv_bm_free_list(self._h, None, 0, C.byref(n))
+        out = np.empty(max(n.value, 1), dtype=np.int32)
+        L.check("pkv_bm_free_list", self._lib.pkv_bm_free_list(self._h, out.ctypes.data, out.size, C.byref(n)))
+        return out[:n.value].copy()

@@ -1,0 +1,223 @@
+// block_manager.cpp -- host-side block manager of the paged KV cache.
+//
+// Decides where every token of every sequence goes:
+//  - lazy allocation: a sequence receives a new block only when its last block
+//    is full, from the front of the free list ("PagedAttention" glossary entry,
+//    "Como funciona la paginacion" and its worked example, which pops blocks
+//    [41, 7, 19] from the free list [41, 7, 19, 2, 33]); a prompt is allocated
+//    first and its last block is then filled (iplexlaw.co.kr, logical vs
+//    physical order);
+//  - sharing: fork() makes a sequence that points at the same physical blocks,
+//    counted per block (glossary entry, "Compartir bloques entre secuencias");
+//  - copy-on-write: a sequence about to write into a partly filled block that
+//    others still reference gets a fresh block and a (src, dst) copy request;
+//    full shared blocks stay shared; the last holder writes in place
+//    (iplexlaw.co.kr, "two answers to one request");
+//  - release: a finished sequence drops its references and blocks whose count
+//    reaches zero return to the back of the free list at once (glossary entry,
+//    continuous batching).
+// Plain C++ with host memory only; exported through the C ABI in pagedkv.h.
+#include <cstdint>
+#include <cstring>
+#include <deque>
+#include <new>
+#include <vector>
+
+#include "pagedkv.h"
+
+struct pkv_block_manager {
+    int num_blocks = 0;
+    int block_size = 0;
+    std::deque<int32_t> free_list;
+    std::vector<int32_t> refs;                  // per physical block
+    std::vector<std::vector<int32_t>> tables;   // per sequence id
+    std::vector<int32_t> lens;                  // tokens per sequence
+    std::vector<uint8_t> alive;
+
+    bool valid_seq(int32_t s) const { return s >= 0 && (size_t)s < tables.size() && alive[s]; }
+
+    int32_t take_block() {
+        const int32_t b = free_list.front();
+        free_list.pop_front();
+        refs[b] = 1;
+        return b;
+    }
+
+    int32_t new_seq(std::vector<int32_t>&& table, int32_t len) {
+        tables.push_back(std::move(table));
+        lens.push_back(len);
+        alive.push_back(1);
+        return (int32_t)(tables.size() - 1);
+    }
+};
+
+extern "C" {
+
+int pkv_bm_create(int num_blocks, int block_size, const int32_t* free_order, int free_count,
+                  pkv_block_manager** out) {
+    if (out == nullptr || num_blocks <= 0 || block_size <= 0) return PKV_EINVAL;
+    pkv_block_manager* bm = new (std::nothrow) pkv_block_manager();
+    if (bm == nullptr) return PKV_ENOMEM;
+    bm->num_blocks = num_blocks;
+    bm->block_size = block_size;
+    bm->refs.assign(num_blocks, 0);
+    if (free_order == nullptr) {
+        for (int b = 0; b < num_blocks; ++b) bm->free_list.push_back(b);
+    } else {
+        std::vector<uint8_t> seen(num_blocks, 0);
+        for (int i = 0; i < free_count; ++i) {
+            const int32_t b = free_order[i];
+            if (b < 0 || b >= num_blocks || seen[b]) {
+                delete bm;
+                return PKV_EINVAL;
+            }
+            seen[b] = 1;
+            bm->free_list.push_back(b);
+        }
+    }
+    *out = bm;
+    return PKV_OK;
+}
+
+void pkv_bm_destroy(pkv_block_manager* bm) { delete bm; }
+
+int pkv_bm_alloc_seq(pkv_block_manager* bm, int num_tokens, int32_t* seq_out) {
+    if (bm == nullptr || seq_out == nullptr || num_tokens < 0) return PKV_EINVAL;
+    const size_t need = ((size_t)num_tokens + bm->block_size - 1) / bm->block_size;
+    if (need > bm->free_list.size()) return PKV_ENOMEM;
+    std::vector<int32_t> table;
+    table.reserve(need);
+    for (size_t i = 0; i < need; ++i) table.push_back(bm->take_block());
+    *seq_out = bm->new_seq(std::move(table), num_tokens);
+    return PKV_OK;
+}
+
+int pkv_bm_fork(pkv_block_manager* bm, int32_t parent, int32_t* child_out) {
+    if (bm == nullptr || child_out == nullptr) return PKV_EINVAL;
+    if (!bm->valid_seq(parent)) return PKV_ENOENT;
+    std::vector<int32_t> table = bm->tables[parent];
+    for (int32_t b : table) ++bm->refs[b];
+    *child_out = bm->new_seq(std::move(table), bm->lens[parent]);
+    return PKV_OK;
+}
+
+int pkv_bm_append_tokens(pkv_block_manager* bm, const int32_t* seqs, int n, int64_t* slots_out,
+                         int64_t* cow_pairs_out, int* num_pairs_out, int* num_done_out) {
+    if (bm == nullptr || n < 0 || (n > 0 && (seqs == nullptr || slots_out == nullptr || cow_pairs_out == nullptr)))
+        return PKV_EINVAL;
+    int pairs = 0;
+    int done = 0;
+    int status = PKV_OK;
+    for (; done < n; ++done) {
+        const int32_t s = seqs[done];
+        if (!bm->valid_seq(s)) {
+            status = PKV_ENOENT;
+            break;
+        }
+        std::vector<int32_t>& table = bm->tables[s];
+        const int32_t len = bm->lens[s];
+        const int32_t off = len % bm->block_size;
+        if (off == 0) {
+            // last block full (or none yet): next free block, nothing to copy
+            if (bm->free_list.empty()) {
+                status = PKV_ENOMEM;
+                break;
+            }
+            table.push_back(bm->take_block());
+        } else if (bm->refs[table.back()] > 1) {
+            // partly filled block still shared: copy it, write into the copy
+            if (bm->free_list.empty()) {
+                status = PKV_ENOMEM;
+                break;
+            }
+            const int32_t src = table.back();
+            const int32_t dst = bm->take_block();
+            --bm->refs[src];
+            table.back() = dst;
+            cow_pairs_out[2 * pairs] = src;
+            cow_pairs_out[2 * pairs + 1] = dst;
+            ++pairs;
+        }
+        slots_out[done] = (int64_t)table[len / bm->block_size] * bm->block_size + off;
+        bm->lens[s] = len + 1;
+    }
+    if (num_pairs_out) *num_pairs_out = pairs;
+    if (num_done_out) *num_done_out = done;
+    return status;
+}
+
+int pkv_bm_free_seq(pkv_block_manager* bm, int32_t seq) {
+    if (bm == nullptr) return PKV_EINVAL;
+    if (!bm->valid_seq(seq)) return PKV_ENOENT;
+    for (int32_t b : bm->tables[seq]) {
+        if (--bm->refs[b] == 0) bm->free_list.push_back(b);
+    }
+    bm->tables[seq].clear();
+    bm->tables[seq].shrink_to_fit();
+    bm->lens[seq] = 0;
+    bm->alive[seq] = 0;
+    return PKV_OK;
+}
+
+int pkv_bm_num_free(const pkv_block_manager* bm) { return bm ? (int)bm->free_list.size() : -1; }
+
+int pkv_bm_seq_len(const pkv_block_manager* bm, int32_t seq, int32_t* len_out) {
+    if (bm == nullptr || len_out == nullptr) return PKV_EINVAL;
+    if (!bm->valid_seq(seq)) return PKV_ENOENT;
+    *len_out = bm->lens[seq];
+    return PKV_OK;
+}
+
+int pkv_bm_refcount(const pkv_block_manager* bm, int32_t block, int32_t* rc_out) {
+    if (bm == nullptr || rc_out == nullptr || block < 0 || block >= bm->num_blocks) return PKV_EINVAL;
+    *rc_out = bm->refs[block];
+    return PKV_OK;
+}
+
+int pkv_bm_block_table(const pkv_block_manager* bm, int32_t seq, int32_t* out, int cap, int* n_out) {
+    if (bm == nullptr || n_out == nullptr || cap < 0 || (cap > 0 && out == nullptr)) return PKV_EINVAL;
+    if (!bm->valid_seq(seq)) return PKV_ENOENT;
+    const std::vector<int32_t>& t = bm->tables[seq];
+    *n_out = (int)t.size();
+    if ((int)t.size() > cap) return PKV_EINVAL;
+    if (!t.empty()) std::memcpy(out, t.data(), t.size() * sizeof(int32_t));
+    return PKV_OK;
+}
+
+int pkv_bm_slots(const pkv_block_manager* bm, int32_t seq, int start, int count, int64_t* out) {
+    if (bm == nullptr || start < 0 || count < 0 || (count > 0 && out == nullptr)) return PKV_EINVAL;
+    if (!bm->valid_seq(seq)) return PKV_ENOENT;
+    const std::vector<int32_t>& t = bm->tables[seq];
+    if ((size_t)start + count > t.size() * (size_t)bm->block_size) return PKV_EINVAL;
+    for (int i = 0; i < count; ++i) {
+        const int pos = start + i;
+        out[i] = (int64_t)t[pos / bm->block_size] * bm->block_size + pos % bm->block_size;
+    }
+    return PKV_OK;
+}
+
+int pkv_bm_tables(const pkv_block_manager* bm, const int32_t* seqs, int n, int32_t* tables, int max_blocks,
+                  int32_t pad, int32_t* lens) {
+    if (bm == nullptr || n < 0 || max_blocks <= 0 || (n > 0 && (seqs == nullptr || tables == nullptr)))
+        return PKV_EINVAL;
+    for (int i = 0; i < n; ++i) {
+        if (!bm->valid_seq(seqs[i])) return PKV_ENOENT;
+        const std::vector<int32_t>& t = bm->tables[seqs[i]];
+        if ((int)t.size() > max_blocks) return PKV_EINVAL;
+        int32_t* row = tables + (size_t)i * max_blocks;
+        for (int j = 0; j < max_blocks; ++j) row[j] = j < (int)t.size() ? t[j] : pad;
+        if (lens) lens[i] = bm->lens[seqs[i]];
+    }
+    return PKV_OK;
+}
+
+int pkv_bm_free_list(const pkv_block_manager* bm, int32_t* out, int cap, int* n_out) {
+    if (bm == nullptr || n_out == nullptr || cap < 0 || (cap > 0 && out == nullptr)) return PKV_EINVAL;
+    *n_out = (int)bm->free_list.size();
+    if ((int)bm->free_list.size() > cap) return PKV_EINVAL;
+    int i = 0;
+    for (int32_t b : bm->free_list) out[i++] = b;
+    return PKV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,435 @@
+// decode_tc.cu -- paged decode attention, BF16 / FP8 caches, tensor cores.
+//
+// What it computes (PagedAttention): for one new query token per sequence,
+// out[s][h] = softmax(scale * q[s][h] . K[t]) over t < len_s, applied to V[t],
+// where token t of sequence s is read through its block table at row
+// (table[s][t / 16], t % 16) of the pool (glossary entry "PagedAttention",
+// "Como funciona la paginacion" and its worked example).  The attention is
+// tiled FlashAttention-style -- one 16-token block at a time with a running
+// max and sum, so no score matrix is written to memory (same page, "Tecnicas
+// relacionadas") -- and query heads that share a key/value head (grouped-query
+// attention, same section) are served by a single read of each K/V tile.
+//
+// Work decomposition.  A unit is (sequence, partition, kv head).  The kernel
+// is persistent: one CTA per SM, each warp an independent worker that takes
+// units from an atomic counter in the plan's longest-first order.  Each warp
+// owns a ring of STAGES shared-memory stages; a stage holds the K tile and the
+// V tile of one block for its kv head (16 rows of head_dim elements each),
+// fetched by TMA (3-D tensor map over [slots][kv heads][head_dim], 128-byte
+// swizzle, box = 16 slots x 1 head x 128 bytes) and completing on per-stage
+// mbarriers.  Lane 0 issues the loads STAGES blocks ahead of the block the
+// warp is computing.
+//
+// Per block, in "swap-AB" form so the 16 tokens are the M=16 side of
+// mma.m16n8k16 and the (up to 8) query heads of the group are N=8:
+//   S^T[16 tok x 8 heads]  = K_tile[16 x D] * Q^T[D x 8]      (D/16 MMAs)
+//   online softmax over the tokens of each head column (base-2 exponent)
+//   O^T[D x 8 heads]      += V_tile^T[D x 16] * P^T[16 x 8]   (D/16 MMAs)
+// P^T's B fragment is the transpose of S^T's accumulator fragment, produced
+// with movmatrix.  BF16 tiles feed ldmatrix(.trans); FP8 tiles are converted to
+// f16 in registers (exact) and use f16 MMAs, with the per-tensor scales folded
+// into the score scale and the output.
+#include "pkv_common.cuh"
+
+namespace pkv {
+
+template <bool FP8, int D>
+struct TileCfg {
+    static constexpr int kElem = FP8 ? 1 : 2;
+    static constexpr int kRowBytes = D * kElem;            // bytes of one token row of one head
+    static constexpr int kSub = kRowBytes / 128;            // 128-byte swizzle atoms per row
+    static constexpr int kBoxElems = 128 / kElem;           // TMA box inner extent (elements)
+    static constexpr int kTileBytes = kBlockSize * kRowBytes;
+    static constexpr int kStageBytes = 2 * kTileBytes;      // K tile + V tile
+    static_assert(kRowBytes % 128 == 0, "rows must be whole 128-byte swizzle atoms");
+};
+
+// Address of 16-byte chunk `chunk` (0..kSub*8-1) of row `row` in a swizzled tile.
+template <bool FP8, int D>
+__device__ __forceinline__ uint32_t tile_addr(uint32_t tile, int row, int chunk) {
+    const int sub = chunk >> 3, c = chunk & 7;
+    return tile + sub * (kBlockSize * 128) + row * 128 + ((c ^ (row & 7)) << 4);
+}
+
+template <bool FP8, int D, int NT, int WARPS, int STAGES>
+__global__ void __launch_bounds__(WARPS * 32, 1)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                     const DecodeParams p) {
+    using C = TileCfg<FP8, D>;
+    constexpr int KS = D / 16;  // k-steps of the score MMA == m-tiles of the output MMA
+    static_assert(STAGES >= 2 && STAGES < 64, "ring depth");
+
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t bars[WARPS][2 * STAGES];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    const uint32_t ring = base + warp * STAGES * C::kStageBytes;
+    const uint32_t bar0 = smem_u32(&bars[warp][0]);  // K barrier of stage st at bar0 + 8*st, V at + 8*(STAGES+st)
+
+    if (lane == 0) {
+        if (warp == 0) {
+            prefetch_tensormap(&tmK);
+            prefetch_tensormap(&tmV);
+        }
+        for (int st = 0; st < 2 * STAGES; ++st) mbar_init(bar0 + 8 * st, 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
+
+    const int num_units = p.hdr->num_units;
+    const int P = p.hdr->partition;
+    const int G = p.group;
+    uint32_t seqno = 0;  // blocks this warp has consumed so far (stage = seqno % STAGES)
+
+    for (;;) {
+        int u = 0;
+        if (lane == 0) u = atomicAdd(&p.hdr->counter, 1);
+        u = __shfl_sync(0xffffffffu, u, 0);
+        if (u >= num_units) break;
+        const int2 item = p.items[u / p.num_kv_heads];
+        const int kvh = u - (u / p.num_kv_heads) * p.num_kv_heads;
+        const int s = item.x, part = item.y;
+        const int L = clamped_len(p, s, false);
+        const int t0 = part * P;
+        const int t1 = min(L, t0 + P);
+        const int nblk = (t1 - t0 + kBlockSize - 1) / kBlockSize;
+        const int blk0 = t0 / kBlockSize;
+        const int32_t* tab = p.block_tables + (size_t)s * p.max_blocks_per_seq + blk0;
+
+        // Block ids, 32 at a time: lane i holds block (32*chunk + i); the next
+        // chunk is loaded one chunk ahead of use.
+        auto load_ids = [&](int chunk) -> int {
+            const int j = chunk * 32 + lane;
+            return j < nblk ? __ldg(tab + j) : -1;
+        };
+        int ids_cur = load_ids(0);
+        int ids_nxt = load_ids(1);
+        int chunk_cur = 0;
+        unsigned long long okmask = 0;  // bit (j & 63): block j's id was in range
+
+        // Q^T fragments (B operand): n = query head of the group, k = head_dim.
+        uint32_t qf[NT][KS][2];
+        const int hq0 = kvh * G;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int hh = nt * 8 + g;
+            const bool hv = hh < G;
+            const __nv_bfloat16* qrow =
+                static_cast<const __nv_bfloat16*>(p.q) + ((size_t)s * p.num_heads + hq0 + (hv ? hh : 0)) * D;
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                if constexpr (!FP8) {
+                    const int d0 = ks * 16 + 2 * t;
+                    qf[nt][ks][0] = hv ? *reinterpret_cast<const uint32_t*>(qrow + d0) : 0u;
+                    qf[nt][ks][1] = hv ? *reinterpret_cast<const uint32_t*>(qrow + d0 + 8) : 0u;
+                } else {
+                    // k positions {2t, 2t+1, 2t+8, 2t+9} of step ks hold head_dim 16ks+4t+{0,1,2,3}
+                    const int d0 = ks * 16 + 4 * t;
+                    uint2 w = hv ? *reinterpret_cast<const uint2*>(qrow + d0) : make_uint2(0u, 0u);
+                    qf[nt][ks][0] = pack_f16x2(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u));
+                    qf[nt][ks][1] = pack_f16x2(__uint_as_float(w.y << 16), __uint_as_float(w.y & 0xFFFF0000u));
+                }
+            }
+        }
+
+        // Issue the TMA loads of block j of this unit into its stage (all lanes
+        // call it: the block id is broadcast with a shuffle).
+        auto issue = [&](int j) {
+            const int ch = j >> 5;
+            if (ch != chunk_cur) {
+                ids_cur = ids_nxt;
+                ids_nxt = load_ids(ch + 1);
+                chunk_cur = ch;
+            }
+            const int id = __shfl_sync(0xffffffffu, ids_cur, j & 31);
+            const bool ok = id >= 0 && id < p.num_blocks;
+            if (ok) okmask |= 1ull << (j & 63);
+            else okmask &= ~(1ull << (j & 63));
+            if (lane == 0) {
+                if (!ok && kvh == 0) count_error(p.err);
+                const uint32_t st = (seqno + j) % STAGES;
+                const uint32_t bk = bar0 + 8 * st, bv = bar0 + 8 * (STAGES + st);
+                const uint32_t dk = ring + st * C::kStageBytes, dv = dk + C::kTileBytes;
+                const int row = (ok ? id : 0) * kBlockSize;
+                mbar_arrive_expect_tx(bk, C::kTileBytes);
+#pragma unroll
+                for (int sub = 0; sub < C::kSub; ++sub)
+                    tma_load_3d(dk + sub * (kBlockSize * 128), &tmK, sub * C::kBoxElems, kvh, row, bk);
+                mbar_arrive_expect_tx(bv, C::kTileBytes);
+#pragma unroll
+                for (int sub = 0; sub < C::kSub; ++sub)
+                    tma_load_3d(dv + sub * (kBlockSize * 128), &tmV, sub * C::kBoxElems, kvh, row, bv);
+            }
+        };
+
+        const int npro = nblk < STAGES ? nblk : STAGES;
+        for (int j = 0; j < npro; ++j) issue(j);
+        int issued = npro;
+
+        float m[NT][2], l[NT][2], oacc[NT][KS][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            m[nt][0] = m[nt][1] = -INFINITY;
+            l[nt][0] = l[nt][1] = 0.f;
+#pragma unroll
+            for (int i = 0; i < KS; ++i) oacc[nt][i][0] = oacc[nt][i][1] = oacc[nt][i][2] = oacc[nt][i][3] = 0.f;
+        }
+
+        bool dead = false;
+        int j = 0;
+        for (; j < nblk; ++j) {
+            const uint32_t st = (seqno + j) % STAGES;
+            const uint32_t par = ((seqno + j) / STAGES) & 1u;
+            const uint32_t kt = ring + st * C::kStageBytes, vt = kt + C::kTileBytes;
+            const bool blk_ok = (okmask >> (j & 63)) & 1ull;
+            const int nvalid = min(kBlockSize, t1 - (t0 + j * kBlockSize));
+
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar0 + 8 * st, par))) {
+                dead = true;
+                break;
+            }
+            float sc[NT][4];
+            if (blk_ok) {
+                // ---- S^T = K Q^T
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+                if constexpr (!FP8) {
+#pragma unroll
+                    for (int ks = 0; ks < KS; ++ks) {
+                        const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
+                        const int chunk = 2 * ks + (lane >> 4);
+                        uint32_t a0, a1, a2, a3;
+                        ldmatrix_x4(tile_addr<FP8, D>(kt, row, chunk), a0, a1, a2, a3);
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) mma_bf16(sc[nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
+                    }
+                } else {
+#pragma unroll
+                    for (int kp = 0; kp < KS / 2; ++kp) {
+                        const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
+                        const int chunk = 2 * kp + (lane >> 4);
+                        uint32_t r0, r1, r2, r3;
+                        ldmatrix_x4(tile_addr<FP8, D>(kt, row, chunk), r0, r1, r2, r3);
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            mma_f16(sc[nt], e4m3x2_to_f16x2(r0), e4m3x2_to_f16x2(r1), e4m3x2_to_f16x2(r0 >> 16),
+                                    e4m3x2_to_f16x2(r1 >> 16), qf[nt][2 * kp][0], qf[nt][2 * kp][1]);
+                            mma_f16(sc[nt], e4m3x2_to_f16x2(r2), e4m3x2_to_f16x2(r3), e4m3x2_to_f16x2(r2 >> 16),
+                                    e4m3x2_to_f16x2(r3 >> 16), qf[nt][2 * kp + 1][0], qf[nt][2 * kp + 1][1]);
+                        }
+                    }
+                }
+            }
+
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar0 + 8 * (STAGES + st), par))) {
+                dead = true;
+                break;
+            }
+            if (blk_ok) {
+                // ---- online softmax over this block's tokens (rows g and g+8)
+                const bool vlo = g < nvalid, vhi = g + 8 < nvalid;
+                uint32_t pb0[NT], pb1[NT];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const float x0 = vlo ? sc[nt][0] * p.score_scale : -INFINITY;
+                    const float x1 = vlo ? sc[nt][1] * p.score_scale : -INFINITY;
+                    const float x2 = vhi ? sc[nt][2] * p.score_scale : -INFINITY;
+                    const float x3 = vhi ? sc[nt][3] * p.score_scale : -INFINITY;
+                    float b0 = fmaxf(x0, x2), b1 = fmaxf(x1, x3);
+#pragma unroll
+                    for (int o = 4; o < 32; o <<= 1) {
+                        b0 = fmaxf(b0, __shfl_xor_sync(0xffffffffu, b0, o));
+                        b1 = fmaxf(b1, __shfl_xor_sync(0xffffffffu, b1, o));
+                    }
+                    const float mn0 = fmaxf(m[nt][0], b0), mn1 = fmaxf(m[nt][1], b1);
+                    const float mu0 = mn0 == -INFINITY ? 0.f : mn0, mu1 = mn1 == -INFINITY ? 0.f : mn1;
+                    const float al0 = fast_exp2(m[nt][0] - mu0), al1 = fast_exp2(m[nt][1] - mu1);
+                    const float p0 = fast_exp2(x0 - mu0), p2 = fast_exp2(x2 - mu0);
+                    const float p1 = fast_exp2(x1 - mu1), p3 = fast_exp2(x3 - mu1);
+                    l[nt][0] = l[nt][0] * al0 + (p0 + p2);
+                    l[nt][1] = l[nt][1] * al1 + (p1 + p3);
+                    m[nt][0] = mn0;
+                    m[nt][1] = mn1;
+#pragma unroll
+                    for (int i = 0; i < KS; ++i) {
+                        oacc[nt][i][0] *= al0;
+                        oacc[nt][i][1] *= al1;
+                        oacc[nt][i][2] *= al0;
+                        oacc[nt][i][3] *= al1;
+                    }
+                    // accumulator fragment rows = tokens, cols = heads; transpose into
+                    // the B fragment of P^T (rows = tokens as k, cols = heads as n)
+                    if constexpr (!FP8) {
+                        pb0[nt] = movmatrix_trans(pack_bf16x2(p0, p1));
+                        pb1[nt] = movmatrix_trans(pack_bf16x2(p2, p3));
+                    } else {
+                        pb0[nt] = movmatrix_trans(pack_f16x2(p0, p1));
+                        pb1[nt] = movmatrix_trans(pack_f16x2(p2, p3));
+                    }
+                }
+
+                // Rows past the context hold stale data (possibly NaN): zero them so
+                // that a zero probability cannot meet a NaN in the MMA.
+                if (nvalid < kBlockSize) {
+                    const int per_row = C::kSub * 8;
+                    const int nz = (kBlockSize - nvalid) * per_row;
+                    for (int i = lane; i < nz; i += 32) {
+                        const int r = nvalid + i / per_row, c = i - (i / per_row) * per_row;
+                        const uint32_t a = vt + (c >> 3) * (kBlockSize * 128) + r * 128 + (c & 7) * 16;
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0) : "memory");
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+
+                // ---- O^T += V^T P^T
+                if constexpr (!FP8) {
+#pragma unroll
+                    for (int i = 0; i < KS; ++i) {
+                        const int row = (lane & 7) + (lane >> 4) * 8;
+                        const int chunk = 2 * i + ((lane >> 3) & 1);
+                        uint32_t a0, a1, a2, a3;
+                        ldmatrix_x4_trans(tile_addr<FP8, D>(vt, row, chunk), a0, a1, a2, a3);
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) mma_bf16(oacc[nt][i], a0, a1, a2, a3, pb0[nt], pb1[nt]);
+                    }
+                } else {
+#pragma unroll
+                    for (int q4 = 0; q4 < D / 32; ++q4) {
+                        // bytes 32*q4 + 4g .. +3 of token rows 2t, 2t+1, 2t+8, 2t+9
+                        const int chunk = 2 * q4 + (g >> 2);
+                        const int within = (g & 3) * 4;
+                        const uint32_t w0 = lds32(tile_addr<FP8, D>(vt, 2 * t, chunk) + within);
+                        const uint32_t w1 = lds32(tile_addr<FP8, D>(vt, 2 * t + 1, chunk) + within);
+                        const uint32_t w2 = lds32(tile_addr<FP8, D>(vt, 2 * t + 8, chunk) + within);
+                        const uint32_t w3 = lds32(tile_addr<FP8, D>(vt, 2 * t + 9, chunk) + within);
+                        // pair up the two tokens of each k-pair: (tok a, tok b) per head_dim column
+                        const uint32_t x01lo = __byte_perm(w0, w1, 0x5140), x01hi = __byte_perm(w0, w1, 0x7362);
+                        const uint32_t x23lo = __byte_perm(w2, w3, 0x5140), x23hi = __byte_perm(w2, w3, 0x7362);
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            // m-tile 2*q4: rows g -> column 32q4+4g, g+8 -> 32q4+4g+1
+                            mma_f16(oacc[nt][2 * q4], e4m3x2_to_f16x2(x01lo), e4m3x2_to_f16x2(x01lo >> 16),
+                                    e4m3x2_to_f16x2(x23lo), e4m3x2_to_f16x2(x23lo >> 16), pb0[nt], pb1[nt]);
+                            // m-tile 2*q4+1: rows g -> column 32q4+4g+2, g+8 -> 32q4+4g+3
+                            mma_f16(oacc[nt][2 * q4 + 1], e4m3x2_to_f16x2(x01hi), e4m3x2_to_f16x2(x01hi >> 16),
+                                    e4m3x2_to_f16x2(x23hi), e4m3x2_to_f16x2(x23hi >> 16), pb0[nt], pb1[nt]);
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            if (issued < nblk) {
+                issue(issued);
+                ++issued;
+            }
+        }
+
+        if (dead) {
+            // A load never completed: wait (bounded) for the other loads still in
+            // flight into this warp's ring, report, and stop this warp.
+            for (int k = j; k < issued; ++k) {
+                const uint32_t st = (seqno + k) % STAGES;
+                const uint32_t par = ((seqno + k) / STAGES) & 1u;
+                mbar_wait_bounded(bar0 + 8 * st, par, 1LL << 28);
+                mbar_wait_bounded(bar0 + 8 * (STAGES + st), par, 1LL << 28);
+            }
+            if (lane == 0) {
+                atomicExch(&p.hdr->timeout, 1);
+                count_error(p.err);
+            }
+            return;
+        }
+        seqno += nblk;
+
+        // ---- epilogue: full l per head column, then out or the partition's (m, l, o)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+#pragma unroll
+                for (int o = 4; o < 32; o <<= 1) l[nt][c] += __shfl_xor_sync(0xffffffffu, l[nt][c], o);
+            }
+        const bool split = p.nparts[s] > 1;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const int hh = nt * 8 + 2 * t + c;
+                if (hh >= G) continue;
+                const int hq = hq0 + hh;
+                const float inv = l[nt][c] > 0.f ? p.out_scale / l[nt][c] : 0.f;
+                if (!split) {
+                    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + ((size_t)s * p.num_heads + hq) * D;
+                    if constexpr (!FP8) {
+#pragma unroll
+                        for (int i = 0; i < KS; ++i) {
+                            o[16 * i + g] = __float2bfloat16(oacc[nt][i][c] * inv);
+                            o[16 * i + 8 + g] = __float2bfloat16(oacc[nt][i][c + 2] * inv);
+                        }
+                    } else {
+#pragma unroll
+                        for (int q4 = 0; q4 < D / 32; ++q4) {
+                            const uint32_t lo = pack_bf16x2(oacc[nt][2 * q4][c] * inv, oacc[nt][2 * q4][c + 2] * inv);
+                            const uint32_t hi =
+                                pack_bf16x2(oacc[nt][2 * q4 + 1][c] * inv, oacc[nt][2 * q4 + 1][c + 2] * inv);
+                            *reinterpret_cast<uint2*>(o + 32 * q4 + 4 * g) = make_uint2(lo, hi);
+                        }
+                    }
+                } else {
+                    const size_t slot = ((size_t)s * p.num_heads + hq) * p.max_parts + part;
+                    float* o = p.part_o + slot * D;
+                    if constexpr (!FP8) {
+#pragma unroll
+                        for (int i = 0; i < KS; ++i) {
+                            o[16 * i + g] = oacc[nt][i][c] * inv;
+                            o[16 * i + 8 + g] = oacc[nt][i][c + 2] * inv;
+                        }
+                    } else {
+#pragma unroll
+                        for (int q4 = 0; q4 < D / 32; ++q4)
+                            *reinterpret_cast<float4*>(o + 32 * q4 + 4 * g) =
+                                make_float4(oacc[nt][2 * q4][c] * inv, oacc[nt][2 * q4][c + 2] * inv,
+                                            oacc[nt][2 * q4 + 1][c] * inv, oacc[nt][2 * q4 + 1][c + 2] * inv);
+                    }
+                    if (g == 0) p.part_ml[slot] = make_float2(m[nt][c], l[nt][c]);
+                }
+            }
+    }
+}
+
+template <bool FP8, int D, int NT, int WARPS, int STAGES>
+static cudaError_t launch_tc(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeParams& p, int num_sms,
+                             cudaStream_t stream) {
+    using C = TileCfg<FP8, D>;
+    const int smem = WARPS * STAGES * C::kStageBytes + 1024;
+    auto kern = decode_tc_kernel<FP8, D, NT, WARPS, STAGES>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<num_sms, WARPS * 32, smem, stream>>>(tmK, tmV, p);
+    return cudaGetLastError();
+}
+
+// Warps per CTA of the tensor-core decode (one CTA per SM).
+constexpr int kTcWarps = 8;
+
+int decode_tc_warps() { return kTcWarps; }
+
+cudaError_t launch_decode_tc(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeParams& p, bool fp8,
+                             int num_sms, cudaStream_t stream) {
+    const int nt = (p.group + 7) / 8;
+    if (fp8) {
+        if (p.head_dim != 128) return cudaErrorInvalidValue;
+        return nt == 1 ? launch_tc<true, 128, 1, kTcWarps, 6>(tmK, tmV, p, num_sms, stream)
+                       : launch_tc<true, 128, 2, kTcWarps, 6>(tmK, tmV, p, num_sms, stream);
+    }
+    if (p.head_dim == 128)
+        return nt == 1 ? launch_tc<false, 128, 1, kTcWarps, 3>(tmK, tmV, p, num_sms, stream)
+                       : launch_tc<false, 128, 2, kTcWarps, 3>(tmK, tmV, p, num_sms, stream);
+    return nt == 1 ? launch_tc<false, 64, 1, kTcWarps, 6>(tmK, tmV, p, num_sms, stream)
+                   : launch_tc<false, 64, 2, kTcWarps, 6>(tmK, tmV, p, num_sms, stream);
+}
+
+}  // namespace pkv

@@ -1,0 +1,122 @@
+"""Parity of the native C++ block manager with the oracle's reference manager
+(CPU only; integer work, compared exactly)."""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle import RefBlockManager
+
+
+@pytest.fixture(scope="module")
+def BM():
+    from paged_kv_cache_404_b200 import build
+    build.build()
+    from paged_kv_cache_404_b200 import BlockManager
+    return BlockManager
+
+
+def test_worked_example(BM, golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "worked_example.json")))
+    bm = BM(g["pool_blocks"], g["block_size"], free_order=g["free_blocks"])
+    s = bm.alloc_seq(g["num_tokens"])
+    assert bm.block_table(s).tolist() == g["expected_block_table"]
+    assert bm.free_list().tolist() == g["expected_free_after"]
+    slots = bm.slots(s, 0, g["num_tokens"])
+    assert slots[0] == 41 * 16 and slots[16] == 7 * 16 and slots[39] == 19 * 16 + 7
+    assert len(bm.block_table(s)) * g["block_size"] - g["num_tokens"] == g["unused_slots_paged"]
+
+
+def _same_state(bm, ref, live):
+    assert bm.free_list().tolist() == list(ref.free)
+    for s in live:
+        assert bm.block_table(s).tolist() == ref.tables[s]
+        assert bm.seq_len(s) == ref.lens[s]
+    for b in range(ref.num_blocks):
+        assert bm.refcount(b) == ref.ref[b]
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_random_traces_match_reference(BM, seed):
+    rng = np.random.default_rng(seed)
+    NB = 300
+    order = rng.permutation(NB)
+    bm, ref = BM(NB, 16, free_order=order), RefBlockManager(NB, 16, free_order=order)
+    live = []
+    for step in range(2500):
+        op = int(rng.integers(0, 10))
+        if op == 0 or not live:
+            n = int(rng.integers(0, 70))
+            try:
+                r = ref.alloc_seq(n)
+            except MemoryError:
+                with pytest.raises(Exception):
+                    bm.alloc_seq(n)
+                continue
+            assert bm.alloc_seq(n) == r
+            live.append(r)
+        elif op == 1:
+            p = live[int(rng.integers(len(live)))]
+            r = ref.fork(p)
+            assert bm.fork(p) == r
+            live.append(r)
+        elif op == 2 and len(live) > 1:
+            s = live.pop(int(rng.integers(len(live))))
+            ref.free_seq(s)
+            bm.free_seq(s)
+        else:
+            k = int(rng.integers(1, 6))
+            seqs = [live[int(rng.integers(len(live)))] for _ in range(k)]
+            seqs = list(dict.fromkeys(seqs))
+            exp_slots, exp_pairs = [], []
+            ok = True
+            for s in seqs:
+                try:
+                    slot, cow = ref.append_token(s)
+                except MemoryError:
+                    ok = False
+                    break
+                exp_slots.append(slot)
+                if cow:
+                    exp_pairs.append(cow)
+            if not ok:
+                # the reference raised part-way; replay the successful prefix on the native side
+                done = len(exp_slots)
+                if done:
+                    slots, pairs = bm.append_tokens(seqs[:done])
+                    assert slots.tolist() == exp_slots
+                with pytest.raises(Exception):
+                    bm.append_tokens(seqs[done:done + 1])
+                continue
+            slots, pairs = bm.append_tokens(seqs)
+            assert slots.tolist() == exp_slots
+            assert [tuple(p) for p in pairs.tolist()] == exp_pairs
+        if step % 250 == 0:
+            _same_state(bm, ref, live)
+    _same_state(bm, ref, live)
+
+
+def test_parallel_sampling_trace(BM):
+    bm = BM(64, 16)
+    p = bm.alloc_seq(1000 % 64 + 40)          # 40 + 40 = 80 tokens: 5 blocks, last one full
+    q = bm.alloc_seq(40)                      # 3 blocks, last holds 8
+    kids = [bm.fork(q), bm.fork(q)]
+    slots, pairs = bm.append_tokens([q] + kids + [p])
+    assert [tuple(x) for x in pairs.tolist()] == [(7, 8), (7, 9)]
+    assert bm.refcount(7) == 1 and bm.refcount(5) == 3 and bm.refcount(6) == 3
+    assert slots[2] == 7 * 16 + 8             # the last holder writes in place
+    assert slots[3] == 10 * 16                # full last block: next free block
+
+
+def test_errors(BM):
+    from paged_kv_cache_404_b200 import PagedKVError
+    bm = BM(2, 16)
+    with pytest.raises(PagedKVError):
+        bm.alloc_seq(40)
+    with pytest.raises(PagedKVError):
+        bm.fork(7)
+    with pytest.raises(PagedKVError):
+        bm.free_seq(3)
+    with pytest.raises(PagedKVError):
+        BM(4, 16, free_order=[0, 0])
