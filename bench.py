@@ -438,6 +438,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="gqa70b", choices=sorted(DESCR))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--partition", type=int, default=0, help="partition tokens (0 = automatic)")
+    ap.add_argument("--num-seqs", type=int, default=0,
+                    help="fewer sequences of the same shape (small cases for profiling; not a bench line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args(argv)
@@ -445,6 +447,8 @@ def main(argv=None):
 
     rank, world, local = dist_env()
     w0 = W.WORKLOADS[args.workload]
+    if args.num_seqs:
+        w0 = W.scaled(w0, num_seqs=args.num_seqs, num_prompts=max(1, args.num_seqs // max(w0.samples, 1)))
     if args.impl == "reference":
         run_reference(args, w0, rank, world)
         return

@@ -257,8 +257,9 @@ def test_invalid_block_ids_are_skipped_and_counted():
     out = torch.empty_like(case.q)
     for P in (0, 16):
         err.zero_()
+        ws = pkv.decode_workspace(case.S, w.num_heads, w.head_dim, case.max_len, P)
         pkv.paged_attention_decode(out, case.q, case.k_pool, case.v_pool, g_t, case.g_lens, w.scale,
-                                   case.max_len, case.ws, partition_tokens=P, err_count=err)
+                                   case.max_len, ws, partition_tokens=P, err_count=err)
         torch.cuda.synchronize()
         assert int(err.item()) == 2
         # oracle semantics for the same bad ids: the tokens of those blocks are left out
