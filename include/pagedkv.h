@@ -171,6 +171,42 @@ int pkv_paged_attention_decode(void* out, const void* q, int q_dtype,
                                int32_t* err_count, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Decode attention that allocates nothing and takes no workspace.
+ * The pages have no counterpart to this call: it exists for callers that
+ * cannot allocate device memory where they run the decode (a plug-in inside a
+ * host program that owns all device memory, a loop that must not call
+ * cudaMalloc/cudaFree because they synchronise the device, a latency budget
+ * that allocation would break).
+ *
+ * Same arguments, layouts, computation and errors as
+ * pkv_paged_attention_decode, without `workspace` / `workspace_bytes`: the
+ * scratch is a device array of PKV_NOALLOC_SCRATCH_BYTES that the library
+ * declares at file scope.  Every GPU that loads the library's kernels holds
+ * that array until the process exits.
+ *  - Limit: returns PKV_EINVAL, before any CUDA call, when the scratch these
+ *    bounds need (pkv_decode_workspace_bytes(num_seqs, num_heads, head_dim,
+ *    max_context_len, partition_tokens)) exceeds PKV_NOALLOC_SCRATCH_BYTES;
+ *    a larger partition_tokens lowers the need.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *    first call before any stream capture.
+ *  - All calls share the one array and it keeps the last call's contents;
+ *    nothing in it needs clearing (each call's first kernel rewrites what the
+ *    others read).  Calls whose GPU work overlaps (different streams without
+ *    ordering between them) race on it: order them on one stream.
+ *  - Calls no cudaMalloc, cudaFree or allocating library routine.
+ * ---------------------------------------------------------------------- */
+#define PKV_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+int pkv_paged_attention_decode_noalloc(void* out, const void* q, int q_dtype,
+                                       const void* k_pool, const void* v_pool, int cache_dtype,
+                                       const int32_t* block_tables, int max_blocks_per_seq,
+                                       const int32_t* context_lens, int num_seqs, int max_context_len,
+                                       int num_blocks, int block_size, int num_heads, int num_kv_heads,
+                                       int head_dim, float scale, float k_scale, float v_scale,
+                                       int partition_tokens, int32_t* err_count, void* stream);
+
+/* ------------------------------------------------------------------------
  * Copy-on-write block copy: for every pair (src, dst) copy the whole physical
  * block src over block dst, in both pools.
  * Source: before a sequence writes into a block that other sequences still

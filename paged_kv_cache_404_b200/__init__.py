@@ -13,5 +13,6 @@ from .ops import (  # noqa: F401
     decode_workspace,
     decode_workspace_bytes,
     paged_attention_decode,
+    paged_attention_decode_noalloc,
     paged_kv_write,
 )

@@ -88,6 +88,25 @@ def paged_attention_decode(out, q, k_pool, v_pool, block_tables, context_lens, s
     return out
 
 
+def paged_attention_decode_noalloc(out, q, k_pool, v_pool, block_tables, context_lens, scale, max_context_len,
+                                   k_scale=1.0, v_scale=1.0, partition_tokens=0, err_count=None, stream=None):
+    """paged_attention_decode for callers that cannot allocate: no workspace argument;
+    the library's fixed device scratch (PKV_NOALLOC_SCRATCH_BYTES) is used instead."""
+    S, Hq, D = q.shape
+    NB, bs, Hkv, D2 = k_pool.shape
+    if D2 != D or out.shape != q.shape:
+        raise ValueError("shape mismatch")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    st = L.lib().pkv_paged_attention_decode_noalloc(
+        _ptr(out), _ptr(q), _dtype_code(q), _ptr(k_pool), _ptr(v_pool), _dtype_code(k_pool),
+        _ptr(block_tables), int(block_tables.shape[1]), _ptr(context_lens), S, int(max_context_len), NB, bs,
+        Hq, Hkv, D, float(scale), float(k_scale), float(v_scale), int(partition_tokens), _ptr(err_count),
+        _stream(stream))
+    L.check("pkv_paged_attention_decode_noalloc", st)
+    return out
+
+
 def copy_blocks(k_pool, v_pool, src_dst_pairs, err_count=None, stream=None):
     """Copy whole blocks src -> dst in both pools; src_dst_pairs int64 [n, 2] on the device."""
     if src_dst_pairs.dtype != torch.int64:
