@@ -14,11 +14,12 @@ cudaError_t launch_copy_blocks(void* k_pool, void* v_pool, size_t block_bytes, c
                                int num_blocks, int32_t* err, cudaStream_t stream);
 cudaError_t launch_decode_plan(const DecodeParams& p, int fixed_partition, int min_partition, int num_candidates,
                                int target_units, int out_dtype, cudaStream_t stream);
-cudaError_t launch_decode_merge(const DecodeParams& p, int out_dtype, cudaStream_t stream);
 cudaError_t launch_decode_tc(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeParams& p, bool fp8,
                              int num_sms, cudaStream_t stream);
 cudaError_t launch_decode_f32(const DecodeParams& p, int num_sms, cudaStream_t stream);
-int decode_tc_warps();
+int decode_tc_warps(bool fp8, int head_dim);
+float fp8_tile_value_scale();
+cudaError_t launch_decode_merge(const DecodeParams& p, int out_dtype, cudaStream_t stream);
 }  // namespace pkv
 
 using namespace pkv;
@@ -27,8 +28,11 @@ namespace {
 
 // Smallest partition the automatic plan considers, and how many units per
 // warp it aims for before it stops halving the partition.
+#ifndef PKV_UNITS_PER_WORKER
+#define PKV_UNITS_PER_WORKER 2
+#endif
 constexpr int kMinAutoPartition = 256;
-constexpr int kUnitsPerWorker = 8;
+constexpr int kUnitsPerWorker = PKV_UNITS_PER_WORKER;
 constexpr int kMaxCandidates = 12;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -184,8 +188,9 @@ int pkv_paged_attention_decode(void* out, const void* q, int q_dtype, const void
     p.group = group;
     p.head_dim = head_dim;
     const float log2e = 1.4426950408889634f;
-    p.score_scale = scale * log2e * (fp8 ? k_scale : 1.f);
-    p.out_scale = fp8 ? v_scale : 1.f;
+    const float tile = fp8 ? fp8_tile_value_scale() : 1.f;
+    p.score_scale = scale * log2e * (fp8 ? k_scale * tile : 1.f);
+    p.out_scale = fp8 ? v_scale * tile : 1.f;
     p.k_pool = k_pool;
     p.v_pool = v_pool;
     p.hdr = reinterpret_cast<WsHeader*>(w);
@@ -201,7 +206,7 @@ int pkv_paged_attention_decode(void* out, const void* q, int q_dtype, const void
     int ncand = 1;
     if (partition_tokens == 0)
         while (ncand < kMaxCandidates && ((long long)min_p << (ncand - 1)) < max_context_len) ++ncand;
-    const int warps_per_sm = f32 ? 32 : decode_tc_warps();
+    const int warps_per_sm = f32 ? 32 : decode_tc_warps(fp8, head_dim);
     const int target_units = num_sms * warps_per_sm * kUnitsPerWorker;
     const int out_dtype = f32 ? 0 : 1;
 
@@ -218,7 +223,8 @@ int pkv_paged_attention_decode(void* out, const void* q, int q_dtype, const void
         e = launch_decode_tc(tmK, tmV, p, fp8, num_sms, st);
     }
     if (e != cudaSuccess) return PKV_ECUDA;
-    // A split is possible only if the smallest partition is shorter than the longest context.
+    // a split (and so a merge) is possible only if the smallest partition is
+    // shorter than the longest context
     if (min_p < max_context_len) {
         e = launch_decode_merge(p, out_dtype, st);
         if (e != cudaSuccess) return PKV_ECUDA;

@@ -20,6 +20,8 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* __restrict__ k_
                                                           long long chunks_per_block,
                                                           const int64_t* __restrict__ pairs, int num_blocks,
                                                           int32_t* err) {
+    pdl_wait();
+    pdl_trigger();
     const int pair = blockIdx.y;
     const long long src = pairs[2 * pair];
     const long long dst = pairs[2 * pair + 1];
@@ -50,9 +52,8 @@ cudaError_t launch_copy_blocks(void* k_pool, void* v_pool, size_t block_bytes, c
     long long chunks = (long long)(block_bytes / 16);
     long long per_cta = (long long)threads * kCopyUnroll;
     dim3 grid((unsigned)((chunks + per_cta - 1) / per_cta), (unsigned)num_pairs, 2);
-    copy_blocks_kernel<<<grid, threads, 0, stream>>>(static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool),
-                                                     chunks, pairs, num_blocks, err);
-    return cudaGetLastError();
+    return launch_pdl(copy_blocks_kernel, grid, dim3(threads), 0, stream, static_cast<uint4*>(k_pool),
+                      static_cast<uint4*>(v_pool), chunks, pairs, num_blocks, err);
 }
 
 }  // namespace pkv

@@ -16,6 +16,8 @@ template <int D>
 __global__ void __launch_bounds__(256) decode_f32_kernel(const DecodeParams p) {
     constexpr int E = D / 32;
     const int lane = threadIdx.x & 31;
+    pdl_wait();
+    pdl_trigger();
     const int num_units = p.hdr->num_units;
     const int P = p.hdr->partition;
     const float* kpool = static_cast<const float*>(p.k_pool);
@@ -81,11 +83,8 @@ __global__ void __launch_bounds__(256) decode_f32_kernel(const DecodeParams p) {
 cudaError_t launch_decode_f32(const DecodeParams& p, int num_sms, cudaStream_t stream) {
     const int threads = 256;
     const int grid = num_sms * 4;
-    if (p.head_dim == 128)
-        decode_f32_kernel<128><<<grid, threads, 0, stream>>>(p);
-    else
-        decode_f32_kernel<64><<<grid, threads, 0, stream>>>(p);
-    return cudaGetLastError();
+    if (p.head_dim == 128) return launch_pdl(decode_f32_kernel<128>, dim3(grid), dim3(threads), 0, stream, p);
+    return launch_pdl(decode_f32_kernel<64>, dim3(grid), dim3(threads), 0, stream, p);
 }
 
 }  // namespace pkv

@@ -6,6 +6,9 @@
 // base-2 scores, sum of 2^(s - m), and the normalised output.  Partitions are
 // merged with weights l_p * 2^(m_p - M), M = max_p m_p.
 //
+// The merge runs as its own kernel after the decode, one warp per (sequence,
+// query head), so that no decode warp sits on a merge's memory latency.
+//
 // The plan runs on the device because the context lengths live there: one CTA
 // picks P from the actual lengths, then writes a work list of (sequence,
 // partition) items ordered by size, largest first (full partitions, then the
@@ -18,6 +21,7 @@ namespace pkv {
 
 constexpr int kPlanThreads = 1024;
 constexpr int kMaxBuckets = 1024;
+constexpr int kMaxCandidates = 12;
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
@@ -30,35 +34,47 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
                                                                    int num_candidates, int target_units,
                                                                    int zero_out_dtype) {
     __shared__ int hist[kMaxBuckets];
-    __shared__ unsigned long long red[kPlanThreads / 32];
+    __shared__ unsigned long long units_of[kMaxCandidates];
     __shared__ int chosen;
     const int tid = threadIdx.x;
 
-    // 1. partition size
+    // The workspace and the output may still be in use by the previous kernel.
+    pdl_wait();
+    pdl_trigger();
+
+    // 1. partition size: the largest candidate min_partition << c whose work
+    //    list still has target_units units (one pass over the lengths for all c)
+    if (tid < kMaxCandidates) units_of[tid] = 0;
+    __syncthreads();
     if (fixed_partition > 0) {
         if (tid == 0) chosen = fixed_partition;
     } else {
-        if (tid == 0) chosen = min_partition;
-        // largest candidate (min_partition << c) that still yields target_units units
-        for (int c = num_candidates - 1; c >= 0; --c) {
-            const int P = min_partition << c;
-            unsigned long long units = 0;
-            for (int s = tid; s < p.num_seqs; s += kPlanThreads)
-                units += (unsigned long long)ceil_div(clamped_len(p, s, false), P);
+        unsigned long long cnt[kMaxCandidates];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) units += __shfl_xor_sync(0xffffffffu, units, o);
-            if ((tid & 31) == 0) red[tid >> 5] = units;
-            __syncthreads();
-            if (tid < 32) {
-                unsigned long long u = red[tid];
+        for (int c = 0; c < kMaxCandidates; ++c) cnt[c] = 0;
+        for (int s = tid; s < p.num_seqs; s += kPlanThreads) {
+            const int L = clamped_len(p, s, false);
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) u += __shfl_xor_sync(0xffffffffu, u, o);
-                if (tid == 0 && u * (unsigned long long)p.num_kv_heads >= (unsigned long long)target_units &&
-                    chosen == min_partition)
-                    chosen = P;
-            }
-            __syncthreads();
-            if (chosen != min_partition) break;
+            for (int c = 0; c < kMaxCandidates; ++c)
+                if (c < num_candidates) cnt[c] += (unsigned long long)ceil_div(L, min_partition << c);
+        }
+#pragma unroll
+        for (int c = 0; c < kMaxCandidates; ++c) {
+            if (c >= num_candidates) break;
+            unsigned long long v = cnt[c];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            if ((tid & 31) == 0 && v) atomicAdd(&units_of[c], v);
+        }
+        __syncthreads();
+        if (tid == 0) {
+            int P = min_partition;
+            for (int c = num_candidates - 1; c >= 0; --c)
+                if (units_of[c] * (unsigned long long)p.num_kv_heads >= (unsigned long long)target_units) {
+                    P = min_partition << c;
+                    break;
+                }
+            chosen = P;
         }
     }
     __syncthreads();
@@ -130,20 +146,24 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
     }
 }
 
-// One warp per (sequence, query head): merge the partitions of a split context.
+// Merge of a split context, one warp per (sequence, query head): M = max_p m_p
+// over partitions with l_p > 0, w_p = l_p 2^(m_p - M), out = sum w_p o_p / sum w_p
+// (o_p normalised, m_p in base-2 units).  Sequences with one partition were
+// written by the decode kernel directly.
 template <int D, typename OutT>
 __global__ void __launch_bounds__(256) decode_merge_kernel(DecodeParams p) {
+    pdl_wait();
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (warp >= p.num_seqs * p.num_heads) return;
     const int s = warp / p.num_heads;
     const int n = p.nparts[s];
-    if (n <= 1) return;  // written directly by the decode kernel (or zero length)
+    if (n <= 1) return;
     const size_t base = (size_t)warp * p.max_parts;
-    constexpr int E = D / 32;  // elements per lane
+    constexpr int E = D / 32;
     float M = -INFINITY;
     for (int i = lane; i < n; i += 32) {
-        float2 ml = p.part_ml[base + i];
+        const float2 ml = p.part_ml[base + i];
         if (ml.y > 0.f) M = fmaxf(M, ml.x);
     }
 #pragma unroll
@@ -153,22 +173,14 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(DecodeParams p) {
     for (int e = 0; e < E; ++e) acc[e] = 0.f;
     float W = 0.f;
     if (M != -INFINITY) {
+#pragma unroll 4
         for (int i = 0; i < n; ++i) {
             const float2 ml = p.part_ml[base + i];
-            if (!(ml.y > 0.f)) continue;
-            const float w = ml.y * exp2f(ml.x - M);
+            const float w = ml.y > 0.f ? ml.y * exp2f(ml.x - M) : 0.f;
             W += w;
             const float* o = p.part_o + (base + i) * D + lane * E;
-            if constexpr (E == 4) {
-                float4 v = *reinterpret_cast<const float4*>(o);
-                acc[0] += w * v.x;
-                acc[1] += w * v.y;
-                acc[2] += w * v.z;
-                acc[3] += w * v.w;
-            } else {
 #pragma unroll
-                for (int e = 0; e < E; ++e) acc[e] += w * o[e];
-            }
+            for (int e = 0; e < E; ++e) acc[e] += w * o[e];
         }
     }
     const float inv = W > 0.f ? 1.f / W : 0.f;
@@ -182,29 +194,20 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(DecodeParams p) {
     }
 }
 
-cudaError_t launch_decode_plan(const DecodeParams& p, int fixed_partition, int min_partition, int num_candidates,
-                               int target_units, int out_dtype, cudaStream_t stream) {
-    decode_plan_kernel<<<1, kPlanThreads, 0, stream>>>(p, fixed_partition, min_partition, num_candidates,
-                                                        target_units, out_dtype);
-    return cudaGetLastError();
-}
-
 cudaError_t launch_decode_merge(const DecodeParams& p, int out_dtype, cudaStream_t stream) {
     const int warps = p.num_seqs * p.num_heads;
-    const int threads = 256;
-    const unsigned grid = (unsigned)((warps * 32 + threads - 1) / threads);
-    if (p.head_dim == 128) {
-        if (out_dtype == 0)
-            decode_merge_kernel<128, float><<<grid, threads, 0, stream>>>(p);
-        else
-            decode_merge_kernel<128, __nv_bfloat16><<<grid, threads, 0, stream>>>(p);
-    } else {
-        if (out_dtype == 0)
-            decode_merge_kernel<64, float><<<grid, threads, 0, stream>>>(p);
-        else
-            decode_merge_kernel<64, __nv_bfloat16><<<grid, threads, 0, stream>>>(p);
-    }
-    return cudaGetLastError();
+    const unsigned grid = (unsigned)((warps * 32 + 255) / 256);
+    if (p.head_dim == 128)
+        return out_dtype == 0 ? launch_pdl(decode_merge_kernel<128, float>, dim3(grid), dim3(256), 0, stream, p)
+                              : launch_pdl(decode_merge_kernel<128, __nv_bfloat16>, dim3(grid), dim3(256), 0, stream, p);
+    return out_dtype == 0 ? launch_pdl(decode_merge_kernel<64, float>, dim3(grid), dim3(256), 0, stream, p)
+                          : launch_pdl(decode_merge_kernel<64, __nv_bfloat16>, dim3(grid), dim3(256), 0, stream, p);
+}
+
+cudaError_t launch_decode_plan(const DecodeParams& p, int fixed_partition, int min_partition, int num_candidates,
+                               int target_units, int out_dtype, cudaStream_t stream) {
+    return launch_pdl(decode_plan_kernel, dim3(1), dim3(kPlanThreads), 0, stream, p, fixed_partition, min_partition,
+                      num_candidates, target_units, out_dtype);
 }
 
 }  // namespace pkv

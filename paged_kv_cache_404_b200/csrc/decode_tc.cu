@@ -33,6 +33,26 @@
 
 namespace pkv {
 
+// FP8 tiles: 1 = convert codes to f16 by moving bits (values scaled by 2^-8,
+// the factor folded into the scales); 0 = the cvt instruction.
+#ifndef PKV_FP8_BITCVT
+#define PKV_FP8_BITCVT 0
+#endif
+// FP8 scores: 1 = E4M3 tensor-core MMA on the stored codes with q split into
+// E4M3 hi + lo parts; 0 = codes converted to f16 and an f16 MMA.
+#ifndef PKV_FP8_QK_E4M3
+#define PKV_FP8_QK_E4M3 0
+#endif
+#if PKV_DEBUG_TIMELINE
+// Per-warp timeline for experiments: start, end (ns), units, merges, merge ns, blocks.
+__device__ unsigned long long g_timeline[4096][6];
+__device__ __forceinline__ unsigned long long now_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+#endif
+
 template <bool FP8, int D>
 struct TileCfg {
     static constexpr int kElem = FP8 ? 1 : 2;
@@ -43,13 +63,6 @@ struct TileCfg {
     static constexpr int kStageBytes = 2 * kTileBytes;      // K tile + V tile
     static_assert(kRowBytes % 128 == 0, "rows must be whole 128-byte swizzle atoms");
 };
-
-// Address of 16-byte chunk `chunk` (0..kSub*8-1) of row `row` in a swizzled tile.
-template <bool FP8, int D>
-__device__ __forceinline__ uint32_t tile_addr(uint32_t tile, int row, int chunk) {
-    const int sub = chunk >> 3, c = chunk & 7;
-    return tile + sub * (kBlockSize * 128) + row * 128 + ((c ^ (row & 7)) << 4);
-}
 
 template <bool FP8, int D, int NT, int WARPS, int STAGES>
 __global__ void __launch_bounds__(WARPS * 32, 1)
@@ -77,11 +90,41 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
         fence_barrier_init();
     }
     __syncwarp();
+    // everything above overlaps the plan kernel; its outputs are read below
+    pdl_wait();
+    pdl_trigger();
+
+    // Lane-dependent byte offsets inside a swizzled tile (chunk c of row r sits
+    // at r*128 + ((c ^ (r & 7)) << 4) within its 16-row x 128-byte atom), computed
+    // once; per block only the stage base is added.  Atoms of the tile (64-element
+    // halves of a bf16 D=128 row) add 2048 bytes each.
+    //  koff[j]: ldmatrix of K, matrices (rows 0-7 | 8-15) x (chunk 2j | 2j+1)
+    //  voff[j]: ldmatrix.trans of V, matrices (rows 0-7, 2j) (0-7, 2j+1) (8-15, 2j) (8-15, 2j+1)
+    //  foff[j][r]: FP8 V words at rows 2t (+r) of chunk 2j + (g >> 2), byte 4 (g & 3)
+    uint32_t koff[4], voff[4], foff[4][2];
+    {
+        const int krow = (lane & 7) + ((lane >> 3) & 1) * 8, kh = lane >> 4;
+        const int vrow = (lane & 7) + (lane >> 4) * 8, vh = (lane >> 3) & 1;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            koff[j] = krow * 128 + ((((2 * j + kh) & 7) ^ (krow & 7)) << 4);
+            voff[j] = vrow * 128 + ((((2 * j + vh) & 7) ^ (vrow & 7)) << 4);
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int row = 2 * t + r;
+                foff[j][r] = row * 128 + ((((2 * j + (g >> 2)) & 7) ^ (row & 7)) << 4) + (g & 3) * 4;
+            }
+        }
+    }
 
     const int num_units = p.hdr->num_units;
     const int P = p.hdr->partition;
     const int G = p.group;
     uint32_t seqno = 0;  // blocks this warp has consumed so far (stage = seqno % STAGES)
+#if PKV_DEBUG_TIMELINE
+    const unsigned long long dbg_t0 = now_ns();
+    unsigned long long dbg_units = 0, dbg_merges = 0, dbg_merge_ns = 0;
+#endif
 
     for (;;) {
         int u = 0;
@@ -133,6 +176,54 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
                 }
             }
         }
+
+#if PKV_FP8_QK_E4M3
+        // FP8 scores on the FP8 tensor path: q of head g scaled by a power of two
+        // s_g (max |q| s_g in [128, 256)) and split into E4M3 hi + lo words in
+        // the m16n8k32 B layout (k = head_dim 32kk + 4t..4t+3 and +16); the
+        // score columns are divided by s back in the softmax.
+        uint32_t qhi[NT][D / 32][2], qlo[NT][D / 32][2];
+        float col_scale[NT][2];
+        if constexpr (FP8) {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int hh = nt * 8 + g;
+                const bool hv = hh < G;
+                const __nv_bfloat16* qrow =
+                    static_cast<const __nv_bfloat16*>(p.q) + ((size_t)s * p.num_heads + hq0 + (hv ? hh : 0)) * D;
+                float x[D / 32][2][4];
+                float amax = 0.f;
+#pragma unroll
+                for (int kk = 0; kk < D / 32; ++kk)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint2 w = hv ? *reinterpret_cast<const uint2*>(qrow + 32 * kk + 16 * h + 4 * t)
+                                           : make_uint2(0u, 0u);
+                        x[kk][h][0] = __uint_as_float(w.x << 16);
+                        x[kk][h][1] = __uint_as_float(w.x & 0xFFFF0000u);
+                        x[kk][h][2] = __uint_as_float(w.y << 16);
+                        x[kk][h][3] = __uint_as_float(w.y & 0xFFFF0000u);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(x[kk][h][e]));
+                    }
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+                // s = 2^(7 - floor(log2 amax)); 1 for an all-zero (or padding) head
+                const int ex = amax > 0.f ? (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127 : 7;
+                const float sq = __uint_as_float((uint32_t)(127 + 7 - ex) << 23);
+#pragma unroll
+                for (int kk = 0; kk < D / 32; ++kk)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        split_e4m3x4(x[kk][h][0] * sq, x[kk][h][1] * sq, x[kk][h][2] * sq, x[kk][h][3] * sq,
+                                     qhi[nt][kk][h], qlo[nt][kk][h]);
+                // this thread's score columns are heads 2t and 2t+1 (held by lanes 8t and 8t+4)
+                const float inv = 1.f / sq;
+                col_scale[nt][0] = __shfl_sync(0xffffffffu, inv, 8 * t);
+                col_scale[nt][1] = __shfl_sync(0xffffffffu, inv, 8 * t + 4);
+            }
+        }
+#endif
 
         // Issue the TMA loads of block j of this unit into its stage (all lanes
         // call it: the block id is broadcast with a shuffle).
@@ -192,35 +283,82 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
             }
             float sc[NT][4];
             if (blk_ok) {
-                // ---- S^T = K Q^T
+                // ---- S^T = K Q^T, even and odd k-steps in two independent chains
+                float sc2[NT][4];
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) sc[nt][e] = sc2[nt][e] = 0.f;
                 if constexpr (!FP8) {
 #pragma unroll
                     for (int ks = 0; ks < KS; ++ks) {
-                        const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
-                        const int chunk = 2 * ks + (lane >> 4);
                         uint32_t a0, a1, a2, a3;
-                        ldmatrix_x4(tile_addr<FP8, D>(kt, row, chunk), a0, a1, a2, a3);
+                        ldmatrix_x4(kt + (ks >> 2) * (kBlockSize * 128) + koff[ks & 3], a0, a1, a2, a3);
 #pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) mma_bf16(sc[nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
+                        for (int nt = 0; nt < NT; ++nt)
+                            mma_bf16((ks & 1) ? sc2[nt] : sc[nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
                     }
                 } else {
+#if PKV_FP8_QK_E4M3
+                    // ldmatrix of 16 rows x 32 codes is exactly the m16n8k32 A fragment
+#pragma unroll
+                    for (int kk = 0; kk < D / 32; ++kk) {
+                        uint32_t r0, r1, r2, r3;
+                        ldmatrix_x4(kt + koff[kk], r0, r1, r2, r3);
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            mma_e4m3(sc[nt], r0, r1, r2, r3, qhi[nt][kk][0], qhi[nt][kk][1]);
+                            mma_e4m3(sc2[nt], r0, r1, r2, r3, qlo[nt][kk][0], qlo[nt][kk][1]);
+                        }
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        sc[nt][0] *= col_scale[nt][0];
+                        sc[nt][1] *= col_scale[nt][1];
+                        sc[nt][2] *= col_scale[nt][0];
+                        sc[nt][3] *= col_scale[nt][1];
+                        sc2[nt][0] *= col_scale[nt][0];
+                        sc2[nt][1] *= col_scale[nt][1];
+                        sc2[nt][2] *= col_scale[nt][0];
+                        sc2[nt][3] *= col_scale[nt][1];
+                    }
+#else
 #pragma unroll
                     for (int kp = 0; kp < KS / 2; ++kp) {
-                        const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
-                        const int chunk = 2 * kp + (lane >> 4);
                         uint32_t r0, r1, r2, r3;
-                        ldmatrix_x4(tile_addr<FP8, D>(kt, row, chunk), r0, r1, r2, r3);
+                        ldmatrix_x4(kt + koff[kp], r0, r1, r2, r3);
+#if PKV_FP8_BITCVT
+                        // codes (0,1) and (2,3) of each register, spread into the high
+                        // byte of each 16-bit lane, then moved into f16 fields (x 2^-8)
+                        const uint32_t k00 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(r0, 0, 0x1100));
+                        const uint32_t k01 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(r0, 0, 0x3322));
+                        const uint32_t k10 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(r1, 0, 0x1100));
+                        const uint32_t k11 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(r1, 0, 0x3322));
+                        const uint32_t k20 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(r2, 0, 0x1100));
+                        const uint32_t k21 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(r2, 0, 0x3322));
+                        const uint32_t k30 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(r3, 0, 0x1100));
+                        const uint32_t k31 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(r3, 0, 0x3322));
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            mma_f16(sc[nt], k00, k10, k01, k11, qf[nt][2 * kp][0], qf[nt][2 * kp][1]);
+                            mma_f16(sc2[nt], k20, k30, k21, k31, qf[nt][2 * kp + 1][0], qf[nt][2 * kp + 1][1]);
+                        }
+#else
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) {
                             mma_f16(sc[nt], e4m3x2_to_f16x2(r0), e4m3x2_to_f16x2(r1), e4m3x2_to_f16x2(r0 >> 16),
                                     e4m3x2_to_f16x2(r1 >> 16), qf[nt][2 * kp][0], qf[nt][2 * kp][1]);
-                            mma_f16(sc[nt], e4m3x2_to_f16x2(r2), e4m3x2_to_f16x2(r3), e4m3x2_to_f16x2(r2 >> 16),
+                            mma_f16(sc2[nt], e4m3x2_to_f16x2(r2), e4m3x2_to_f16x2(r3), e4m3x2_to_f16x2(r2 >> 16),
                                     e4m3x2_to_f16x2(r3 >> 16), qf[nt][2 * kp + 1][0], qf[nt][2 * kp + 1][1]);
                         }
+#endif
                     }
+#endif
                 }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) sc[nt][e] += sc2[nt][e];
             }
 
             if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar0 + 8 * (STAGES + st), par))) {
@@ -252,12 +390,16 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
                     l[nt][1] = l[nt][1] * al1 + (p1 + p3);
                     m[nt][0] = mn0;
                     m[nt][1] = mn1;
+                    // rescale the accumulator only if some running max moved (rare
+                    // after the first blocks); the test is warp-uniform
+                    if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
 #pragma unroll
-                    for (int i = 0; i < KS; ++i) {
-                        oacc[nt][i][0] *= al0;
-                        oacc[nt][i][1] *= al1;
-                        oacc[nt][i][2] *= al0;
-                        oacc[nt][i][3] *= al1;
+                        for (int i = 0; i < KS; ++i) {
+                            oacc[nt][i][0] *= al0;
+                            oacc[nt][i][1] *= al1;
+                            oacc[nt][i][2] *= al0;
+                            oacc[nt][i][3] *= al1;
+                        }
                     }
                     // accumulator fragment rows = tokens, cols = heads; transpose into
                     // the B fragment of P^T (rows = tokens as k, cols = heads as n)
@@ -288,23 +430,36 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
                 if constexpr (!FP8) {
 #pragma unroll
                     for (int i = 0; i < KS; ++i) {
-                        const int row = (lane & 7) + (lane >> 4) * 8;
-                        const int chunk = 2 * i + ((lane >> 3) & 1);
                         uint32_t a0, a1, a2, a3;
-                        ldmatrix_x4_trans(tile_addr<FP8, D>(vt, row, chunk), a0, a1, a2, a3);
+                        ldmatrix_x4_trans(vt + (i >> 2) * (kBlockSize * 128) + voff[i & 3], a0, a1, a2, a3);
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) mma_bf16(oacc[nt][i], a0, a1, a2, a3, pb0[nt], pb1[nt]);
                     }
                 } else {
 #pragma unroll
                     for (int q4 = 0; q4 < D / 32; ++q4) {
-                        // bytes 32*q4 + 4g .. +3 of token rows 2t, 2t+1, 2t+8, 2t+9
-                        const int chunk = 2 * q4 + (g >> 2);
-                        const int within = (g & 3) * 4;
-                        const uint32_t w0 = lds32(tile_addr<FP8, D>(vt, 2 * t, chunk) + within);
-                        const uint32_t w1 = lds32(tile_addr<FP8, D>(vt, 2 * t + 1, chunk) + within);
-                        const uint32_t w2 = lds32(tile_addr<FP8, D>(vt, 2 * t + 8, chunk) + within);
-                        const uint32_t w3 = lds32(tile_addr<FP8, D>(vt, 2 * t + 9, chunk) + within);
+                        // bytes 32*q4 + 4g .. +3 of token rows 2t, 2t+1, 2t+8, 2t+9 (rows r and
+                        // r+8 share a swizzle phase: +8 rows = +1024 bytes)
+                        const uint32_t w0 = lds32(vt + foff[q4][0]);
+                        const uint32_t w1 = lds32(vt + foff[q4][1]);
+                        const uint32_t w2 = lds32(vt + foff[q4][0] + 8 * 128);
+                        const uint32_t w3 = lds32(vt + foff[q4][1] + 8 * 128);
+#if PKV_FP8_BITCVT
+                        // (tok a, tok b) of head_dim column i, in the high bytes of the two lanes
+                        const uint32_t v0 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(w0, w1, 0x4400));
+                        const uint32_t v1 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(w0, w1, 0x5511));
+                        const uint32_t v2 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(w0, w1, 0x6622));
+                        const uint32_t v3 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(w0, w1, 0x7733));
+                        const uint32_t u0 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(w2, w3, 0x4400));
+                        const uint32_t u1 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(w2, w3, 0x5511));
+                        const uint32_t u2 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(w2, w3, 0x6622));
+                        const uint32_t u3 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(w2, w3, 0x7733));
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            mma_f16(oacc[nt][2 * q4], v0, v1, u0, u1, pb0[nt], pb1[nt]);
+                            mma_f16(oacc[nt][2 * q4 + 1], v2, v3, u2, u3, pb0[nt], pb1[nt]);
+                        }
+#else
                         // pair up the two tokens of each k-pair: (tok a, tok b) per head_dim column
                         const uint32_t x01lo = __byte_perm(w0, w1, 0x5140), x01hi = __byte_perm(w0, w1, 0x7362);
                         const uint32_t x23lo = __byte_perm(w2, w3, 0x5140), x23hi = __byte_perm(w2, w3, 0x7362);
@@ -317,6 +472,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
                             mma_f16(oacc[nt][2 * q4 + 1], e4m3x2_to_f16x2(x01hi), e4m3x2_to_f16x2(x01hi >> 16),
                                     e4m3x2_to_f16x2(x23hi), e4m3x2_to_f16x2(x23hi >> 16), pb0[nt], pb1[nt]);
                         }
+#endif
                     }
                 }
             }
@@ -397,7 +553,23 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
                     if (g == 0) p.part_ml[slot] = make_float2(m[nt][c], l[nt][c]);
                 }
             }
+#if PKV_DEBUG_TIMELINE
+        ++dbg_units;
+#endif
     }
+#if PKV_DEBUG_TIMELINE
+    if (lane == 0) {
+        const int w = blockIdx.x * WARPS + warp;
+        if (w < 4096) {
+            g_timeline[w][0] = dbg_t0;
+            g_timeline[w][1] = now_ns();
+            g_timeline[w][2] = dbg_units;
+            g_timeline[w][3] = dbg_merges;
+            g_timeline[w][4] = dbg_merge_ns;
+            g_timeline[w][5] = seqno;
+        }
+    }
+#endif
 }
 
 template <bool FP8, int D, int NT, int WARPS, int STAGES>
@@ -408,28 +580,60 @@ static cudaError_t launch_tc(const CUtensorMap& tmK, const CUtensorMap& tmV, con
     auto kern = decode_tc_kernel<FP8, D, NT, WARPS, STAGES>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kern<<<num_sms, WARPS * 32, smem, stream>>>(tmK, tmV, p);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(num_sms), dim3(WARPS * 32), smem, stream, tmK, tmV, p);
 }
 
-// Warps per CTA of the tensor-core decode (one CTA per SM).
-constexpr int kTcWarps = 8;
+#if PKV_DEBUG_TIMELINE
+extern "C" int pkv_debug_timeline(void* host, int rows) {
+    return cudaMemcpyFromSymbol(host, g_timeline, sizeof(unsigned long long) * 6 * rows) == cudaSuccess ? 0 : 3;
+}
+#endif
 
-int decode_tc_warps() { return kTcWarps; }
+// Warps per CTA (one CTA per SM) and ring depth per warp, per cache type.
+// Shared memory per CTA = warps * stages * 2 tiles (+1 KB alignment slack).
+#ifndef PKV_TC_WARPS_BF16
+#define PKV_TC_WARPS_BF16 12
+#endif
+#ifndef PKV_TC_STAGES_BF16
+#define PKV_TC_STAGES_BF16 2
+#endif
+#ifndef PKV_TC_WARPS_BF16_D64
+#define PKV_TC_WARPS_BF16_D64 8
+#endif
+#ifndef PKV_TC_STAGES_BF16_D64
+#define PKV_TC_STAGES_BF16_D64 6
+#endif
+#ifndef PKV_TC_WARPS_FP8
+#define PKV_TC_WARPS_FP8 12
+#endif
+#ifndef PKV_TC_STAGES_FP8
+#define PKV_TC_STAGES_FP8 4
+#endif
+
+// Factor by which the FP8 tile values the kernel multiplies are smaller than
+// the stored codes' values (folded into the score and output scales).
+float fp8_tile_value_scale() { return PKV_FP8_BITCVT ? 256.f : 1.f; }
+
+int decode_tc_warps(bool fp8, int head_dim) {
+    if (fp8) return PKV_TC_WARPS_FP8;
+    return head_dim == 128 ? PKV_TC_WARPS_BF16 : PKV_TC_WARPS_BF16_D64;
+}
 
 cudaError_t launch_decode_tc(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeParams& p, bool fp8,
                              int num_sms, cudaStream_t stream) {
     const int nt = (p.group + 7) / 8;
     if (fp8) {
         if (p.head_dim != 128) return cudaErrorInvalidValue;
-        return nt == 1 ? launch_tc<true, 128, 1, kTcWarps, 6>(tmK, tmV, p, num_sms, stream)
-                       : launch_tc<true, 128, 2, kTcWarps, 6>(tmK, tmV, p, num_sms, stream);
+        return nt == 1 ? launch_tc<true, 128, 1, PKV_TC_WARPS_FP8, PKV_TC_STAGES_FP8>(tmK, tmV, p, num_sms, stream)
+                       : launch_tc<true, 128, 2, PKV_TC_WARPS_FP8, PKV_TC_STAGES_FP8>(tmK, tmV, p, num_sms, stream);
     }
     if (p.head_dim == 128)
-        return nt == 1 ? launch_tc<false, 128, 1, kTcWarps, 3>(tmK, tmV, p, num_sms, stream)
-                       : launch_tc<false, 128, 2, kTcWarps, 3>(tmK, tmV, p, num_sms, stream);
-    return nt == 1 ? launch_tc<false, 64, 1, kTcWarps, 6>(tmK, tmV, p, num_sms, stream)
-                   : launch_tc<false, 64, 2, kTcWarps, 6>(tmK, tmV, p, num_sms, stream);
+        return nt == 1
+                   ? launch_tc<false, 128, 1, PKV_TC_WARPS_BF16, PKV_TC_STAGES_BF16>(tmK, tmV, p, num_sms, stream)
+                   : launch_tc<false, 128, 2, PKV_TC_WARPS_BF16, PKV_TC_STAGES_BF16>(tmK, tmV, p, num_sms, stream);
+    return nt == 1
+               ? launch_tc<false, 64, 1, PKV_TC_WARPS_BF16_D64, PKV_TC_STAGES_BF16_D64>(tmK, tmV, p, num_sms, stream)
+               : launch_tc<false, 64, 2, PKV_TC_WARPS_BF16_D64, PKV_TC_STAGES_BF16_D64>(tmK, tmV, p, num_sms, stream);
 }
 
 }  // namespace pkv

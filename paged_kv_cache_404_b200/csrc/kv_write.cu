@@ -22,6 +22,8 @@ __global__ void __launch_bounds__(256) kv_write_copy_kernel(const uint4* __restr
                                                             uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
                                                             long long num_slots, int chunks_per_row,
                                                             int32_t* err) {
+    pdl_wait();
+    pdl_trigger();
     long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     long long total = (long long)num_tokens * chunks_per_row;
     if (i >= total) return;
@@ -55,6 +57,8 @@ __global__ void __launch_bounds__(256) kv_write_fp8_kernel(const SrcT* __restric
                                                            uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
                                                            long long num_slots, int chunks_per_row, float k_scale,
                                                            float v_scale, int32_t* err) {
+    pdl_wait();
+    pdl_trigger();
     long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     long long total = (long long)num_tokens * chunks_per_row;
     if (i >= total) return;
@@ -113,23 +117,23 @@ cudaError_t launch_kv_write(const void* k, const void* v, int src_dtype, const i
         int chunks = row_elems * elem / 16;
         long long total = (long long)num_tokens * chunks;
         unsigned grid = (unsigned)((total + threads - 1) / threads);
-        kv_write_copy_kernel<<<grid, threads, 0, stream>>>(
-            static_cast<const uint4*>(k), static_cast<const uint4*>(v), slots, num_tokens,
-            static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), num_slots, chunks, err);
+        return launch_pdl(kv_write_copy_kernel, dim3(grid), dim3(threads), 0, stream, static_cast<const uint4*>(k),
+                          static_cast<const uint4*>(v), slots, num_tokens, static_cast<uint4*>(k_pool),
+                          static_cast<uint4*>(v_pool), num_slots, chunks, err);
     } else {
         int chunks = row_elems / 16;  // 16 output codes per thread
         long long total = (long long)num_tokens * chunks;
         unsigned grid = (unsigned)((total + threads - 1) / threads);
         if (src_dtype == 1)
-            kv_write_fp8_kernel<__nv_bfloat16><<<grid, threads, 0, stream>>>(
-                static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), slots, num_tokens,
-                static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), num_slots, chunks, k_scale, v_scale, err);
-        else
-            kv_write_fp8_kernel<float><<<grid, threads, 0, stream>>>(
-                static_cast<const float*>(k), static_cast<const float*>(v), slots, num_tokens,
-                static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), num_slots, chunks, k_scale, v_scale, err);
+            return launch_pdl(kv_write_fp8_kernel<__nv_bfloat16>, dim3(grid), dim3(threads), 0, stream,
+                              static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), slots,
+                              num_tokens, static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), num_slots, chunks,
+                              k_scale, v_scale, err);
+        return launch_pdl(kv_write_fp8_kernel<float>, dim3(grid), dim3(threads), 0, stream,
+                          static_cast<const float*>(k), static_cast<const float*>(v), slots, num_tokens,
+                          static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), num_slots, chunks, k_scale,
+                          v_scale, err);
     }
-    return cudaGetLastError();
 }
 
 }  // namespace pkv
