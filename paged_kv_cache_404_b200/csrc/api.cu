@@ -18,7 +18,6 @@ cudaError_t launch_decode_tc(const CUtensorMap& tmK, const CUtensorMap& tmV, con
                              int num_sms, cudaStream_t stream);
 cudaError_t launch_decode_f32(const DecodeParams& p, int num_sms, cudaStream_t stream);
 int decode_tc_warps(bool fp8, int head_dim);
-float fp8_tile_value_scale();
 cudaError_t launch_decode_merge(const DecodeParams& p, int out_dtype, cudaStream_t stream);
 }  // namespace pkv
 
@@ -29,7 +28,7 @@ namespace {
 // Smallest partition the automatic plan considers, and how many units per
 // warp it aims for before it stops halving the partition.
 #ifndef PKV_UNITS_PER_WORKER
-#define PKV_UNITS_PER_WORKER 2
+#define PKV_UNITS_PER_WORKER 3
 #endif
 constexpr int kMinAutoPartition = 256;
 constexpr int kUnitsPerWorker = PKV_UNITS_PER_WORKER;
@@ -188,9 +187,8 @@ int pkv_paged_attention_decode(void* out, const void* q, int q_dtype, const void
     p.group = group;
     p.head_dim = head_dim;
     const float log2e = 1.4426950408889634f;
-    const float tile = fp8 ? fp8_tile_value_scale() : 1.f;
-    p.score_scale = scale * log2e * (fp8 ? k_scale * tile : 1.f);
-    p.out_scale = fp8 ? v_scale * tile : 1.f;
+    p.score_scale = scale * log2e * (fp8 ? k_scale : 1.f);
+    p.out_scale = fp8 ? v_scale : 1.f;
     p.k_pool = k_pool;
     p.v_pool = v_pool;
     p.hdr = reinterpret_cast<WsHeader*>(w);

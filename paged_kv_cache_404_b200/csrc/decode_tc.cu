@@ -33,11 +33,6 @@
 
 namespace pkv {
 
-// FP8 tiles: 1 = convert codes to f16 by moving bits (values scaled by 2^-8,
-// the factor folded into the scales); 0 = the cvt instruction.
-#ifndef PKV_FP8_BITCVT
-#define PKV_FP8_BITCVT 0
-#endif
 // FP8 scores: 1 = E4M3 tensor-core MMA on the stored codes with q split into
 // E4M3 hi + lo parts; 0 = codes converted to f16 and an f16 MMA.
 #ifndef PKV_FP8_QK_E4M3
@@ -45,7 +40,7 @@ namespace pkv {
 #endif
 #if PKV_DEBUG_TIMELINE
 // Per-warp timeline for experiments: start, end (ns), units, merges, merge ns, blocks.
-__device__ unsigned long long g_timeline[4096][6];
+__device__ unsigned long long g_timeline[4096][7];
 __device__ __forceinline__ unsigned long long now_ns() {
     unsigned long long t;
     asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
@@ -64,19 +59,23 @@ struct TileCfg {
     static_assert(kRowBytes % 128 == 0, "rows must be whole 128-byte swizzle atoms");
 };
 
-template <bool FP8, int D, int NT, int WARPS, int STAGES>
+template <bool FP8, int D, int NT, int WARPS, int STAGES, int BPS>
 __global__ void __launch_bounds__(WARPS * 32, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const DecodeParams p) {
     using C = TileCfg<FP8, D>;
     constexpr int KS = D / 16;  // k-steps of the score MMA == m-tiles of the output MMA
     static_assert(STAGES >= 2 && STAGES < 64, "ring depth");
+    static_assert(BPS >= 1 && BPS <= STAGES, "blocks per step fit in the ring");
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t bars[WARPS][2 * STAGES];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
+#if PKV_DEBUG_TIMELINE
+    const unsigned long long dbg_entry = now_ns();
+#endif
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
     const uint32_t ring = base + warp * STAGES * C::kStageBytes;
     const uint32_t bar0 = smem_u32(&bars[warp][0]);  // K barrier of stage st at bar0 + 8*st, V at + 8*(STAGES+st)
@@ -268,114 +267,159 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
             for (int i = 0; i < KS; ++i) oacc[nt][i][0] = oacc[nt][i][1] = oacc[nt][i][2] = oacc[nt][i][3] = 0.f;
         }
 
-        bool dead = false;
-        int j = 0;
-        for (; j < nblk; ++j) {
-            const uint32_t st = (seqno + j) % STAGES;
-            const uint32_t par = ((seqno + j) / STAGES) & 1u;
-            const uint32_t kt = ring + st * C::kStageBytes, vt = kt + C::kTileBytes;
-            const bool blk_ok = (okmask >> (j & 63)) & 1ull;
-            const int nvalid = min(kBlockSize, t1 - (t0 + j * kBlockSize));
-
-            if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar0 + 8 * st, par))) {
-                dead = true;
-                break;
-            }
-            float sc[NT][4];
-            if (blk_ok) {
-                // ---- S^T = K Q^T, even and odd k-steps in two independent chains
-                float sc2[NT][4];
+        // ---- per-tile pieces ------------------------------------------------
+        // S^T[16 tok x 8 heads] of the K tile at `kt` (even and odd k-steps in two
+        // independent accumulation chains, summed at the end)
+        auto scores = [&](uint32_t kt, float (&sc)[NT][4]) {
+            float sc2[NT][4];
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
+            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) sc[nt][e] = sc2[nt][e] = 0.f;
-                if constexpr (!FP8) {
+                for (int e = 0; e < 4; ++e) sc[nt][e] = sc2[nt][e] = 0.f;
+            if constexpr (!FP8) {
 #pragma unroll
-                    for (int ks = 0; ks < KS; ++ks) {
-                        uint32_t a0, a1, a2, a3;
-                        ldmatrix_x4(kt + (ks >> 2) * (kBlockSize * 128) + koff[ks & 3], a0, a1, a2, a3);
+                for (int ks = 0; ks < KS; ++ks) {
+                    uint32_t a0, a1, a2, a3;
+                    ldmatrix_x4(kt + (ks >> 2) * (kBlockSize * 128) + koff[ks & 3], a0, a1, a2, a3);
 #pragma unroll
-                        for (int nt = 0; nt < NT; ++nt)
-                            mma_bf16((ks & 1) ? sc2[nt] : sc[nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
-                    }
-                } else {
+                    for (int nt = 0; nt < NT; ++nt)
+                        mma_bf16((ks & 1) ? sc2[nt] : sc[nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
+                }
+            } else {
 #if PKV_FP8_QK_E4M3
-                    // ldmatrix of 16 rows x 32 codes is exactly the m16n8k32 A fragment
+                // ldmatrix of 16 rows x 32 codes is exactly the m16n8k32 A fragment
 #pragma unroll
-                    for (int kk = 0; kk < D / 32; ++kk) {
-                        uint32_t r0, r1, r2, r3;
-                        ldmatrix_x4(kt + koff[kk], r0, r1, r2, r3);
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
-                            mma_e4m3(sc[nt], r0, r1, r2, r3, qhi[nt][kk][0], qhi[nt][kk][1]);
-                            mma_e4m3(sc2[nt], r0, r1, r2, r3, qlo[nt][kk][0], qlo[nt][kk][1]);
-                        }
-                    }
+                for (int kk = 0; kk < D / 32; ++kk) {
+                    uint32_t r0, r1, r2, r3;
+                    ldmatrix_x4(kt + koff[kk], r0, r1, r2, r3);
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
-                        sc[nt][0] *= col_scale[nt][0];
-                        sc[nt][1] *= col_scale[nt][1];
-                        sc[nt][2] *= col_scale[nt][0];
-                        sc[nt][3] *= col_scale[nt][1];
-                        sc2[nt][0] *= col_scale[nt][0];
-                        sc2[nt][1] *= col_scale[nt][1];
-                        sc2[nt][2] *= col_scale[nt][0];
-                        sc2[nt][3] *= col_scale[nt][1];
+                        mma_e4m3(sc[nt], r0, r1, r2, r3, qhi[nt][kk][0], qhi[nt][kk][1]);
+                        mma_e4m3(sc2[nt], r0, r1, r2, r3, qlo[nt][kk][0], qlo[nt][kk][1]);
                     }
-#else
-#pragma unroll
-                    for (int kp = 0; kp < KS / 2; ++kp) {
-                        uint32_t r0, r1, r2, r3;
-                        ldmatrix_x4(kt + koff[kp], r0, r1, r2, r3);
-#if PKV_FP8_BITCVT
-                        // codes (0,1) and (2,3) of each register, spread into the high
-                        // byte of each 16-bit lane, then moved into f16 fields (x 2^-8)
-                        const uint32_t k00 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(r0, 0, 0x1100));
-                        const uint32_t k01 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(r0, 0, 0x3322));
-                        const uint32_t k10 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(r1, 0, 0x1100));
-                        const uint32_t k11 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(r1, 0, 0x3322));
-                        const uint32_t k20 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(r2, 0, 0x1100));
-                        const uint32_t k21 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(r2, 0, 0x3322));
-                        const uint32_t k30 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(r3, 0, 0x1100));
-                        const uint32_t k31 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(r3, 0, 0x3322));
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
-                            mma_f16(sc[nt], k00, k10, k01, k11, qf[nt][2 * kp][0], qf[nt][2 * kp][1]);
-                            mma_f16(sc2[nt], k20, k30, k21, k31, qf[nt][2 * kp + 1][0], qf[nt][2 * kp + 1][1]);
-                        }
-#else
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
-                            mma_f16(sc[nt], e4m3x2_to_f16x2(r0), e4m3x2_to_f16x2(r1), e4m3x2_to_f16x2(r0 >> 16),
-                                    e4m3x2_to_f16x2(r1 >> 16), qf[nt][2 * kp][0], qf[nt][2 * kp][1]);
-                            mma_f16(sc2[nt], e4m3x2_to_f16x2(r2), e4m3x2_to_f16x2(r3), e4m3x2_to_f16x2(r2 >> 16),
-                                    e4m3x2_to_f16x2(r3 >> 16), qf[nt][2 * kp + 1][0], qf[nt][2 * kp + 1][1]);
-                        }
-#endif
-                    }
-#endif
                 }
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) sc[nt][e] += sc2[nt][e];
+                    for (int e = 0; e < 4; ++e) {
+                        sc[nt][e] *= col_scale[nt][e & 1];
+                        sc2[nt][e] *= col_scale[nt][e & 1];
+                    }
+#else
+#pragma unroll
+                for (int kp = 0; kp < KS / 2; ++kp) {
+                    uint32_t r0, r1, r2, r3;
+                    ldmatrix_x4(kt + koff[kp], r0, r1, r2, r3);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        mma_f16(sc[nt], e4m3x2_to_f16x2(r0), e4m3x2_to_f16x2(r1), e4m3x2_to_f16x2(r0 >> 16),
+                                e4m3x2_to_f16x2(r1 >> 16), qf[nt][2 * kp][0], qf[nt][2 * kp][1]);
+                        mma_f16(sc2[nt], e4m3x2_to_f16x2(r2), e4m3x2_to_f16x2(r3), e4m3x2_to_f16x2(r2 >> 16),
+                                e4m3x2_to_f16x2(r3 >> 16), qf[nt][2 * kp + 1][0], qf[nt][2 * kp + 1][1]);
+                    }
+                }
+#endif
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sc[nt][e] += sc2[nt][e];
+        };
+
+        // O^T[D x 8] += V^T[D x 16] P^T[16 x 8] for the V tile at `vt`
+        auto accumulate_pv = [&](uint32_t vt, const uint32_t (&pb0)[NT], const uint32_t (&pb1)[NT]) {
+            if constexpr (!FP8) {
+#pragma unroll
+                for (int i = 0; i < KS; ++i) {
+                    uint32_t a0, a1, a2, a3;
+                    ldmatrix_x4_trans(vt + (i >> 2) * (kBlockSize * 128) + voff[i & 3], a0, a1, a2, a3);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_bf16(oacc[nt][i], a0, a1, a2, a3, pb0[nt], pb1[nt]);
+                }
+            } else {
+#pragma unroll
+                for (int q4 = 0; q4 < D / 32; ++q4) {
+                    // bytes 32*q4 + 4g .. +3 of token rows 2t, 2t+1, 2t+8, 2t+9 (rows r and
+                    // r+8 share a swizzle phase: +8 rows = +1024 bytes)
+                    const uint32_t w0 = lds32(vt + foff[q4][0]);
+                    const uint32_t w1 = lds32(vt + foff[q4][1]);
+                    const uint32_t w2 = lds32(vt + foff[q4][0] + 8 * 128);
+                    const uint32_t w3 = lds32(vt + foff[q4][1] + 8 * 128);
+                    // pair up the two tokens of each k-pair: (tok a, tok b) per head_dim column
+                    const uint32_t x01lo = __byte_perm(w0, w1, 0x5140), x01hi = __byte_perm(w0, w1, 0x7362);
+                    const uint32_t x23lo = __byte_perm(w2, w3, 0x5140), x23hi = __byte_perm(w2, w3, 0x7362);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        // m-tile 2*q4: rows g -> column 32q4+4g, g+8 -> 32q4+4g+1
+                        mma_f16(oacc[nt][2 * q4], e4m3x2_to_f16x2(x01lo), e4m3x2_to_f16x2(x01lo >> 16),
+                                e4m3x2_to_f16x2(x23lo), e4m3x2_to_f16x2(x23lo >> 16), pb0[nt], pb1[nt]);
+                        // m-tile 2*q4+1: rows g -> column 32q4+4g+2, g+8 -> 32q4+4g+3
+                        mma_f16(oacc[nt][2 * q4 + 1], e4m3x2_to_f16x2(x01hi), e4m3x2_to_f16x2(x01hi >> 16),
+                                e4m3x2_to_f16x2(x23hi), e4m3x2_to_f16x2(x23hi >> 16), pb0[nt], pb1[nt]);
+                    }
+                }
+            }
+        };
+
+        // ---- main loop: BPS blocks per step (one softmax reduction per step) ----
+        bool dead = false;
+        int j = 0;
+        for (; j < nblk; j += BPS) {
+            const int nb = min(BPS, nblk - j);  // warp-uniform
+            uint32_t stb[BPS], parb[BPS], kt[BPS], vt[BPS];
+            bool okb[BPS];
+            int nvalid[BPS];
+            bool any_ok = false;
+#pragma unroll
+            for (int b = 0; b < BPS; ++b) {
+                const int jb = j + b;
+                stb[b] = (seqno + jb) % STAGES;
+                parb[b] = ((seqno + jb) / STAGES) & 1u;
+                kt[b] = ring + stb[b] * C::kStageBytes;
+                vt[b] = kt[b] + C::kTileBytes;
+                okb[b] = b < nb && ((okmask >> (jb & 63)) & 1ull);
+                nvalid[b] = b < nb ? min(kBlockSize, t1 - (t0 + jb * kBlockSize)) : 0;
+                any_ok = any_ok || okb[b];
             }
 
-            if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar0 + 8 * (STAGES + st), par))) {
+            bool waited = true;
+#pragma unroll
+            for (int b = 0; b < BPS; ++b)
+                if (b < nb) waited = waited && mbar_wait_bounded(bar0 + 8 * stb[b], parb[b]);
+            if (!__all_sync(0xffffffffu, waited)) {
                 dead = true;
                 break;
             }
-            if (blk_ok) {
-                // ---- online softmax over this block's tokens (rows g and g+8)
-                const bool vlo = g < nvalid, vhi = g + 8 < nvalid;
-                uint32_t pb0[NT], pb1[NT];
+            float sc[BPS][NT][4];
+#pragma unroll
+            for (int b = 0; b < BPS; ++b)
+                if (okb[b]) scores(kt[b], sc[b]);
+
+#pragma unroll
+            for (int b = 0; b < BPS; ++b)
+                if (b < nb) waited = waited && mbar_wait_bounded(bar0 + 8 * (STAGES + stb[b]), parb[b]);
+            if (!__all_sync(0xffffffffu, waited)) {
+                dead = true;
+                break;
+            }
+
+            if (any_ok) {
+                // ---- online softmax over the step's tokens (rows g and g+8 of each block)
+                uint32_t pb0[BPS][NT], pb1[BPS][NT];
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    const float x0 = vlo ? sc[nt][0] * p.score_scale : -INFINITY;
-                    const float x1 = vlo ? sc[nt][1] * p.score_scale : -INFINITY;
-                    const float x2 = vhi ? sc[nt][2] * p.score_scale : -INFINITY;
-                    const float x3 = vhi ? sc[nt][3] * p.score_scale : -INFINITY;
-                    float b0 = fmaxf(x0, x2), b1 = fmaxf(x1, x3);
+                    float x[BPS][4];
+                    float b0 = -INFINITY, b1 = -INFINITY;
+#pragma unroll
+                    for (int b = 0; b < BPS; ++b) {
+                        const bool vlo = okb[b] && g < nvalid[b], vhi = okb[b] && g + 8 < nvalid[b];
+                        x[b][0] = vlo ? sc[b][nt][0] * p.score_scale : -INFINITY;
+                        x[b][1] = vlo ? sc[b][nt][1] * p.score_scale : -INFINITY;
+                        x[b][2] = vhi ? sc[b][nt][2] * p.score_scale : -INFINITY;
+                        x[b][3] = vhi ? sc[b][nt][3] * p.score_scale : -INFINITY;
+                        b0 = fmaxf(b0, fmaxf(x[b][0], x[b][2]));
+                        b1 = fmaxf(b1, fmaxf(x[b][1], x[b][3]));
+                    }
 #pragma unroll
                     for (int o = 4; o < 32; o <<= 1) {
                         b0 = fmaxf(b0, __shfl_xor_sync(0xffffffffu, b0, o));
@@ -384,10 +428,25 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
                     const float mn0 = fmaxf(m[nt][0], b0), mn1 = fmaxf(m[nt][1], b1);
                     const float mu0 = mn0 == -INFINITY ? 0.f : mn0, mu1 = mn1 == -INFINITY ? 0.f : mn1;
                     const float al0 = fast_exp2(m[nt][0] - mu0), al1 = fast_exp2(m[nt][1] - mu1);
-                    const float p0 = fast_exp2(x0 - mu0), p2 = fast_exp2(x2 - mu0);
-                    const float p1 = fast_exp2(x1 - mu1), p3 = fast_exp2(x3 - mu1);
-                    l[nt][0] = l[nt][0] * al0 + (p0 + p2);
-                    l[nt][1] = l[nt][1] * al1 + (p1 + p3);
+                    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+                    for (int b = 0; b < BPS; ++b) {
+                        const float p0 = fast_exp2(x[b][0] - mu0), p2 = fast_exp2(x[b][2] - mu0);
+                        const float p1 = fast_exp2(x[b][1] - mu1), p3 = fast_exp2(x[b][3] - mu1);
+                        s0 += p0 + p2;
+                        s1 += p1 + p3;
+                        // accumulator fragment rows = tokens, cols = heads; transpose into
+                        // the B fragment of P^T (rows = tokens as k, cols = heads as n)
+                        if constexpr (!FP8) {
+                            pb0[b][nt] = movmatrix_trans(pack_bf16x2(p0, p1));
+                            pb1[b][nt] = movmatrix_trans(pack_bf16x2(p2, p3));
+                        } else {
+                            pb0[b][nt] = movmatrix_trans(pack_f16x2(p0, p1));
+                            pb1[b][nt] = movmatrix_trans(pack_f16x2(p2, p3));
+                        }
+                    }
+                    l[nt][0] = l[nt][0] * al0 + s0;
+                    l[nt][1] = l[nt][1] * al1 + s1;
                     m[nt][0] = mn0;
                     m[nt][1] = mn1;
                     // rescale the accumulator only if some running max moved (rare
@@ -401,86 +460,40 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
                             oacc[nt][i][3] *= al1;
                         }
                     }
-                    // accumulator fragment rows = tokens, cols = heads; transpose into
-                    // the B fragment of P^T (rows = tokens as k, cols = heads as n)
-                    if constexpr (!FP8) {
-                        pb0[nt] = movmatrix_trans(pack_bf16x2(p0, p1));
-                        pb1[nt] = movmatrix_trans(pack_bf16x2(p2, p3));
-                    } else {
-                        pb0[nt] = movmatrix_trans(pack_f16x2(p0, p1));
-                        pb1[nt] = movmatrix_trans(pack_f16x2(p2, p3));
-                    }
                 }
 
                 // Rows past the context hold stale data (possibly NaN): zero them so
                 // that a zero probability cannot meet a NaN in the MMA.
-                if (nvalid < kBlockSize) {
-                    const int per_row = C::kSub * 8;
-                    const int nz = (kBlockSize - nvalid) * per_row;
-                    for (int i = lane; i < nz; i += 32) {
-                        const int r = nvalid + i / per_row, c = i - (i / per_row) * per_row;
-                        const uint32_t a = vt + (c >> 3) * (kBlockSize * 128) + r * 128 + (c & 7) * 16;
-                        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0) : "memory");
+                bool zeroed = false;
+#pragma unroll
+                for (int b = 0; b < BPS; ++b) {
+                    if (okb[b] && nvalid[b] < kBlockSize) {
+                        const int per_row = C::kSub * 8;
+                        const int nz = (kBlockSize - nvalid[b]) * per_row;
+                        for (int i = lane; i < nz; i += 32) {
+                            const int r = nvalid[b] + i / per_row, c = i - (i / per_row) * per_row;
+                            const uint32_t a = vt[b] + (c >> 3) * (kBlockSize * 128) + r * 128 + (c & 7) * 16;
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0) : "memory");
+                        }
+                        zeroed = true;
                     }
+                }
+                if (zeroed) {
                     fence_proxy_async_smem();
                     __syncwarp();
                 }
 
-                // ---- O^T += V^T P^T
-                if constexpr (!FP8) {
 #pragma unroll
-                    for (int i = 0; i < KS; ++i) {
-                        uint32_t a0, a1, a2, a3;
-                        ldmatrix_x4_trans(vt + (i >> 2) * (kBlockSize * 128) + voff[i & 3], a0, a1, a2, a3);
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) mma_bf16(oacc[nt][i], a0, a1, a2, a3, pb0[nt], pb1[nt]);
-                    }
-                } else {
-#pragma unroll
-                    for (int q4 = 0; q4 < D / 32; ++q4) {
-                        // bytes 32*q4 + 4g .. +3 of token rows 2t, 2t+1, 2t+8, 2t+9 (rows r and
-                        // r+8 share a swizzle phase: +8 rows = +1024 bytes)
-                        const uint32_t w0 = lds32(vt + foff[q4][0]);
-                        const uint32_t w1 = lds32(vt + foff[q4][1]);
-                        const uint32_t w2 = lds32(vt + foff[q4][0] + 8 * 128);
-                        const uint32_t w3 = lds32(vt + foff[q4][1] + 8 * 128);
-#if PKV_FP8_BITCVT
-                        // (tok a, tok b) of head_dim column i, in the high bytes of the two lanes
-                        const uint32_t v0 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(w0, w1, 0x4400));
-                        const uint32_t v1 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(w0, w1, 0x5511));
-                        const uint32_t v2 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(w0, w1, 0x6622));
-                        const uint32_t v3 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(w0, w1, 0x7733));
-                        const uint32_t u0 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(w2, w3, 0x4400));
-                        const uint32_t u1 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(w2, w3, 0x5511));
-                        const uint32_t u2 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(w2, w3, 0x6622));
-                        const uint32_t u3 = e4m3_hi_bytes_to_f16x2_scaled(__byte_perm(w2, w3, 0x7733));
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
-                            mma_f16(oacc[nt][2 * q4], v0, v1, u0, u1, pb0[nt], pb1[nt]);
-                            mma_f16(oacc[nt][2 * q4 + 1], v2, v3, u2, u3, pb0[nt], pb1[nt]);
-                        }
-#else
-                        // pair up the two tokens of each k-pair: (tok a, tok b) per head_dim column
-                        const uint32_t x01lo = __byte_perm(w0, w1, 0x5140), x01hi = __byte_perm(w0, w1, 0x7362);
-                        const uint32_t x23lo = __byte_perm(w2, w3, 0x5140), x23hi = __byte_perm(w2, w3, 0x7362);
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
-                            // m-tile 2*q4: rows g -> column 32q4+4g, g+8 -> 32q4+4g+1
-                            mma_f16(oacc[nt][2 * q4], e4m3x2_to_f16x2(x01lo), e4m3x2_to_f16x2(x01lo >> 16),
-                                    e4m3x2_to_f16x2(x23lo), e4m3x2_to_f16x2(x23lo >> 16), pb0[nt], pb1[nt]);
-                            // m-tile 2*q4+1: rows g -> column 32q4+4g+2, g+8 -> 32q4+4g+3
-                            mma_f16(oacc[nt][2 * q4 + 1], e4m3x2_to_f16x2(x01hi), e4m3x2_to_f16x2(x01hi >> 16),
-                                    e4m3x2_to_f16x2(x23hi), e4m3x2_to_f16x2(x23hi >> 16), pb0[nt], pb1[nt]);
-                        }
-#endif
-                    }
-                }
+                for (int b = 0; b < BPS; ++b)
+                    if (okb[b]) accumulate_pv(vt[b], pb0[b], pb1[b]);
             }
             __syncwarp();
-            if (issued < nblk) {
-                issue(issued);
-                ++issued;
-            }
+#pragma unroll
+            for (int b = 0; b < BPS; ++b)
+                if (b < nb && issued < nblk) {
+                    issue(issued);
+                    ++issued;
+                }
         }
 
         if (dead) {
@@ -567,17 +580,18 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
             g_timeline[w][3] = dbg_merges;
             g_timeline[w][4] = dbg_merge_ns;
             g_timeline[w][5] = seqno;
+            g_timeline[w][6] = dbg_entry;
         }
     }
 #endif
 }
 
-template <bool FP8, int D, int NT, int WARPS, int STAGES>
+template <bool FP8, int D, int NT, int WARPS, int STAGES, int BPS>
 static cudaError_t launch_tc(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeParams& p, int num_sms,
                              cudaStream_t stream) {
     using C = TileCfg<FP8, D>;
     const int smem = WARPS * STAGES * C::kStageBytes + 1024;
-    auto kern = decode_tc_kernel<FP8, D, NT, WARPS, STAGES>;
+    auto kern = decode_tc_kernel<FP8, D, NT, WARPS, STAGES, BPS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3(num_sms), dim3(WARPS * 32), smem, stream, tmK, tmV, p);
@@ -585,7 +599,7 @@ static cudaError_t launch_tc(const CUtensorMap& tmK, const CUtensorMap& tmV, con
 
 #if PKV_DEBUG_TIMELINE
 extern "C" int pkv_debug_timeline(void* host, int rows) {
-    return cudaMemcpyFromSymbol(host, g_timeline, sizeof(unsigned long long) * 6 * rows) == cudaSuccess ? 0 : 3;
+    return cudaMemcpyFromSymbol(host, g_timeline, sizeof(unsigned long long) * 7 * rows) == cudaSuccess ? 0 : 3;
 }
 #endif
 
@@ -604,15 +618,19 @@ extern "C" int pkv_debug_timeline(void* host, int rows) {
 #define PKV_TC_STAGES_BF16_D64 6
 #endif
 #ifndef PKV_TC_WARPS_FP8
-#define PKV_TC_WARPS_FP8 12
+#define PKV_TC_WARPS_FP8 16
 #endif
 #ifndef PKV_TC_STAGES_FP8
-#define PKV_TC_STAGES_FP8 4
+#define PKV_TC_STAGES_FP8 3
+#endif
+// Blocks per step of the main loop (one softmax reduction per step).
+#ifndef PKV_TC_BPS_BF16
+#define PKV_TC_BPS_BF16 1
+#endif
+#ifndef PKV_TC_BPS_FP8
+#define PKV_TC_BPS_FP8 2
 #endif
 
-// Factor by which the FP8 tile values the kernel multiplies are smaller than
-// the stored codes' values (folded into the score and output scales).
-float fp8_tile_value_scale() { return PKV_FP8_BITCVT ? 256.f : 1.f; }
 
 int decode_tc_warps(bool fp8, int head_dim) {
     if (fp8) return PKV_TC_WARPS_FP8;
@@ -624,16 +642,16 @@ cudaError_t launch_decode_tc(const CUtensorMap& tmK, const CUtensorMap& tmV, con
     const int nt = (p.group + 7) / 8;
     if (fp8) {
         if (p.head_dim != 128) return cudaErrorInvalidValue;
-        return nt == 1 ? launch_tc<true, 128, 1, PKV_TC_WARPS_FP8, PKV_TC_STAGES_FP8>(tmK, tmV, p, num_sms, stream)
-                       : launch_tc<true, 128, 2, PKV_TC_WARPS_FP8, PKV_TC_STAGES_FP8>(tmK, tmV, p, num_sms, stream);
+        return nt == 1 ? launch_tc<true, 128, 1, PKV_TC_WARPS_FP8, PKV_TC_STAGES_FP8, PKV_TC_BPS_FP8>(tmK, tmV, p, num_sms, stream)
+                       : launch_tc<true, 128, 2, PKV_TC_WARPS_FP8, PKV_TC_STAGES_FP8, PKV_TC_BPS_FP8>(tmK, tmV, p, num_sms, stream);
     }
     if (p.head_dim == 128)
         return nt == 1
-                   ? launch_tc<false, 128, 1, PKV_TC_WARPS_BF16, PKV_TC_STAGES_BF16>(tmK, tmV, p, num_sms, stream)
-                   : launch_tc<false, 128, 2, PKV_TC_WARPS_BF16, PKV_TC_STAGES_BF16>(tmK, tmV, p, num_sms, stream);
+                   ? launch_tc<false, 128, 1, PKV_TC_WARPS_BF16, PKV_TC_STAGES_BF16, PKV_TC_BPS_BF16>(tmK, tmV, p, num_sms, stream)
+                   : launch_tc<false, 128, 2, PKV_TC_WARPS_BF16, PKV_TC_STAGES_BF16, PKV_TC_BPS_BF16>(tmK, tmV, p, num_sms, stream);
     return nt == 1
-               ? launch_tc<false, 64, 1, PKV_TC_WARPS_BF16_D64, PKV_TC_STAGES_BF16_D64>(tmK, tmV, p, num_sms, stream)
-               : launch_tc<false, 64, 2, PKV_TC_WARPS_BF16_D64, PKV_TC_STAGES_BF16_D64>(tmK, tmV, p, num_sms, stream);
+               ? launch_tc<false, 64, 1, PKV_TC_WARPS_BF16_D64, PKV_TC_STAGES_BF16_D64, PKV_TC_BPS_BF16>(tmK, tmV, p, num_sms, stream)
+               : launch_tc<false, 64, 2, PKV_TC_WARPS_BF16_D64, PKV_TC_STAGES_BF16_D64, PKV_TC_BPS_BF16>(tmK, tmV, p, num_sms, stream);
 }
 
 }  // namespace pkv

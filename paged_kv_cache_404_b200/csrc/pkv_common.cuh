@@ -280,18 +280,6 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
     return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
 }
 
-// E4M3 -> f16 by moving bits: for a 16-bit lane holding an E4M3 code c in its
-// high byte (low byte ignored), (c & 0x80) << 8 | (c & 0x7F) << 7 is the f16
-// whose value is exactly value(c) * 2^-8 for every finite code, subnormals
-// included (both formats place the exponent right after the sign, and f16's
-// bias is 8 more than E4M3's).  The 2^8 is folded into the per-tensor scales.
-// Codes 0x7F / 0xFF (NaN) become 480 * 2^-8 instead of NaN.
-// `spread` holds two codes in bytes 1 and 3: the result is the f16x2 pair.
-__device__ __forceinline__ uint32_t e4m3_hi_bytes_to_f16x2_scaled(uint32_t spread) {
-    const uint32_t mag = (spread & 0x7F007F00u) >> 1;
-    return (spread & 0x80008000u) | mag;
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
