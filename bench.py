@@ -88,7 +88,7 @@ def measured_peak_hbm():
 
 def kernel_source_hash():
     h = hashlib.sha256()
-    for f in ("decode_tc.cu", "pkv_common.cuh", "decode_plan.cu"):
+    for f in ("decode_tc.cu", "pkv_common.cuh", "decode_plan.cu", "api.cu"):
         with open(os.path.join(ROOT, "paged_kv_cache_404_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -295,41 +295,66 @@ def time_steps(step: Step, steps: int, warmup: int, world: int, device):
 
 
 def time_e2e(step: Step, steps: int, warmup: int, world: int):
-    """The same step through the public API from pinned HOST buffers: every step
-    copies its inputs (q, new K/V, slots, tables, lengths, copy pairs) host->device
-    and reads the output back device->host, all inside the timed region."""
-    stream = torch.cuda.current_stream()
-    host = {
-        "q": step.q.cpu().pin_memory(), "k_new": step.k_new.cpu().pin_memory(),
-        "v_new": step.v_new.cpu().pin_memory(), "g_slots": step.g_slots.cpu().pin_memory(),
-        "g_tables": step.g_tables.cpu().pin_memory(), "g_lens": step.g_lens.cpu().pin_memory(),
-    }
-    if step.g_pairs is not None:
-        host["g_pairs"] = step.g_pairs.cpu().pin_memory()
-    out_host = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    """The same step through the public API from pinned HOST buffers.  Every
+    step copies its inputs (q, new K/V, slots, tables, lengths, copy pairs)
+    host->device and reads its output back device->host inside the timed
+    region.  The copies run on a second stream with two device input sets, so
+    step i+1's uploads and step i-1's download overlap step i's kernels, as in
+    a serving loop; the KV pools stay resident (they are the cache, not a
+    per-step input).  Uploads and downloads use separate streams."""
+    compute = torch.cuda.current_stream()
+    up = torch.cuda.Stream(device=step.device)
+    down = torch.cuda.Stream(device=step.device)
+    names = ["q", "k_new", "v_new", "g_slots", "g_tables", "g_lens"] + (["g_pairs"] if step.g_pairs is not None else [])
+    host = {n: getattr(step, n).cpu().pin_memory() for n in names}
+    dev = [{n: getattr(step, n) for n in names}, {n: torch.empty_like(getattr(step, n)) for n in names}]
+    outs = [step.out, torch.empty_like(step.out)]
+    out_host = [torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory() for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out_host.numel() * out_host.element_size()
+    d2h = out_host[0].numel() * out_host[0].element_size()
+    uploaded = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    consumed = [torch.cuda.Event() for _ in range(2)]   # set b's inputs no longer needed
 
-    def one():
-        for name, t in host.items():
-            getattr(step, name).copy_(t, non_blocking=True)
-        step.run()
-        out_host.copy_(step.out, non_blocking=True)
+    def run(n_steps):
+        for i in range(n_steps):
+            b = i & 1
+            with torch.cuda.stream(up):
+                if i >= 2:
+                    up.wait_event(consumed[b])
+                for n in names:
+                    dev[b][n].copy_(host[n], non_blocking=True)
+                uploaded[b].record(up)
+            compute.wait_event(uploaded[b])
+            for n in names:
+                setattr(step, n, dev[b][n])
+            step.out = outs[b]
+            step.run()
+            computed[b].record(compute)
+            consumed[b].record(compute)
+            with torch.cuda.stream(down):
+                down.wait_event(computed[b])
+                out_host[b].copy_(outs[b], non_blocking=True)
+        compute.wait_stream(up)
+        compute.wait_stream(down)
 
-    for _ in range(warmup):
-        one()
+    run(warmup)
     torch.cuda.synchronize()
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
     a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(steps):
-        one()
-    b.record(stream)
+    z = torch.cuda.Event(enable_timing=True)
+    a.record(compute)
+    up.wait_event(a)
+    down.wait_event(a)
+    run(steps)
+    z.record(compute)
     torch.cuda.synchronize()
-    return a.elapsed_time(b), h2d, d2h
+    for n in names:
+        setattr(step, n, dev[0][n])
+    step.out = outs[0]
+    return a.elapsed_time(z), h2d, d2h
 
 
 # ------------------------------------------------------------------ CPU oracle timing

@@ -193,7 +193,7 @@ int pkv_paged_attention_decode(void* out, const void* q, int q_dtype, const void
     p.v_pool = v_pool;
     p.hdr = reinterpret_cast<WsHeader*>(w);
     p.nparts = reinterpret_cast<int*>(w + ws.nparts);
-    p.items = reinterpret_cast<int2*>(w + ws.items);
+    p.items = reinterpret_cast<int4*>(w + ws.items);
     p.part_ml = reinterpret_cast<float2*>(w + ws.part_ml);
     p.part_o = reinterpret_cast<float*>(w + ws.part_o);
     p.max_parts = max_parts;

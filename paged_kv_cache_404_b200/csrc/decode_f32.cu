@@ -19,7 +19,6 @@ __global__ void __launch_bounds__(256) decode_f32_kernel(const DecodeParams p) {
     pdl_wait();
     pdl_trigger();
     const int num_units = p.hdr->num_units;
-    const int P = p.hdr->partition;
     const float* kpool = static_cast<const float*>(p.k_pool);
     const float* vpool = static_cast<const float*>(p.v_pool);
     for (;;) {
@@ -27,11 +26,11 @@ __global__ void __launch_bounds__(256) decode_f32_kernel(const DecodeParams p) {
         if (lane == 0) u = atomicAdd(&p.hdr->counter, 1);
         u = __shfl_sync(0xffffffffu, u, 0);
         if (u >= num_units) break;
-        const int2 item = p.items[u / p.num_kv_heads];
+        const int4 item = p.items[u / p.num_kv_heads];
         const int kvh = u % p.num_kv_heads;
         const int s = item.x, part = item.y;
         const int L = clamped_len(p, s, false);
-        const int t0 = part * P, t1 = min(L, t0 + P);
+        const int t0 = item.z * kBlockSize, t1 = min(L, t0 + item.w * kBlockSize);
         const int32_t* tab = p.block_tables + (size_t)s * p.max_blocks_per_seq;
         const bool split = p.nparts[s] > 1;
         for (int hh = 0; hh < p.group; ++hh) {

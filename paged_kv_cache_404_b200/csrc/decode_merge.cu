@@ -1,0 +1,97 @@
+// decode_merge.cu -- log-sum-exp merge of split-context partitions.
+//
+// A long context is cut into partitions (FlashAttention-2 parallelises over
+// the context; iplexlaw.co.kr, section on technical differences); partition p
+// of (sequence, query head) left (m_p, l_p, o_p): the max of its base-2 scores,
+// the sum of 2^(s - m_p) and its normalised output.  The merge is
+//   M = max_p m_p over partitions with l_p > 0,  w_p = l_p 2^(m_p - M),
+//   out = sum_p w_p o_p / sum_p w_p,
+// and a sequence with a single partition was written by the decode kernel.
+//
+// One warp per (sequence, query head).  Lanes are 4 partition groups x 8
+// head_dim slices (16 elements each): group r takes partitions r, r+4, ...,
+// so a 60-partition context costs 15 dependent load rounds instead of 60; the
+// four groups are combined with shuffles at the end.  Deterministic: the order
+// of additions depends only on the partition count.
+#include "pkv_common.cuh"
+
+namespace pkv {
+
+template <int D, typename OutT>
+__global__ void __launch_bounds__(256) decode_merge_kernel(DecodeParams p) {
+    pdl_wait();
+    constexpr int SL = D / 8;  // head_dim elements per lane
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (warp >= p.num_seqs * p.num_heads) return;
+    const int s = warp / p.num_heads;
+    const int n = p.nparts[s];
+    if (n <= 1) return;
+    const size_t base = (size_t)warp * p.max_parts;
+    const int grp = lane >> 3, slice = lane & 7;
+
+    float M = -INFINITY;
+    for (int i = lane; i < n; i += 32) {
+        const float2 ml = p.part_ml[base + i];
+        if (ml.y > 0.f) M = fmaxf(M, ml.x);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+
+    float acc[SL];
+#pragma unroll
+    for (int e = 0; e < SL; ++e) acc[e] = 0.f;
+    float W = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll 2
+        for (int i = grp; i < n; i += 4) {
+            const float2 ml = p.part_ml[base + i];
+            const float w = ml.y > 0.f ? ml.y * exp2f(ml.x - M) : 0.f;
+            W += w;
+            const float4* src = reinterpret_cast<const float4*>(p.part_o + (base + i) * D + slice * SL);
+#pragma unroll
+            for (int v = 0; v < SL / 4; ++v) {
+                const float4 x = src[v];
+                acc[4 * v] += w * x.x;
+                acc[4 * v + 1] += w * x.y;
+                acc[4 * v + 2] += w * x.z;
+                acc[4 * v + 3] += w * x.w;
+            }
+        }
+    }
+    // combine the four partition groups (lanes slice, slice+8, slice+16, slice+24)
+#pragma unroll
+    for (int o = 8; o < 32; o <<= 1) {
+        W += __shfl_xor_sync(0xffffffffu, W, o);
+#pragma unroll
+        for (int e = 0; e < SL; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+    }
+    if (grp != 0) return;
+    const float inv = W > 0.f ? 1.f / W : 0.f;
+    OutT* out = static_cast<OutT*>(p.out) + (size_t)warp * D + slice * SL;
+    if constexpr (sizeof(OutT) == 4) {
+#pragma unroll
+        for (int v = 0; v < SL / 4; ++v)
+            reinterpret_cast<float4*>(out)[v] =
+                make_float4(acc[4 * v] * inv, acc[4 * v + 1] * inv, acc[4 * v + 2] * inv, acc[4 * v + 3] * inv);
+    } else {
+#pragma unroll
+        for (int v = 0; v < SL / 4; ++v) {
+            const uint32_t lo = pack_bf16x2(acc[4 * v] * inv, acc[4 * v + 1] * inv);
+            const uint32_t hi = pack_bf16x2(acc[4 * v + 2] * inv, acc[4 * v + 3] * inv);
+            reinterpret_cast<uint2*>(out)[v] = make_uint2(lo, hi);
+        }
+    }
+}
+
+cudaError_t launch_decode_merge(const DecodeParams& p, int out_dtype, cudaStream_t stream) {
+    const int warps = p.num_seqs * p.num_heads;
+    const unsigned grid = (unsigned)((warps * 32 + 255) / 256);
+    if (p.head_dim == 128)
+        return out_dtype == 0 ? launch_pdl(decode_merge_kernel<128, float>, dim3(grid), dim3(256), 0, stream, p)
+                              : launch_pdl(decode_merge_kernel<128, __nv_bfloat16>, dim3(grid), dim3(256), 0, stream, p);
+    return out_dtype == 0 ? launch_pdl(decode_merge_kernel<64, float>, dim3(grid), dim3(256), 0, stream, p)
+                          : launch_pdl(decode_merge_kernel<64, __nv_bfloat16>, dim3(grid), dim3(256), 0, stream, p);
+}
+
+}  // namespace pkv

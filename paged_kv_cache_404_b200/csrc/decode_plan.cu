@@ -6,15 +6,14 @@
 // base-2 scores, sum of 2^(s - m), and the normalised output.  Partitions are
 // merged with weights l_p * 2^(m_p - M), M = max_p m_p.
 //
-// The merge runs as its own kernel after the decode, one warp per (sequence,
-// query head), so that no decode warp sits on a merge's memory latency.
+// The merge runs as its own kernel after the decode (decode_merge.cu), so
+// that no decode warp sits on a merge's memory latency.
 //
 // The plan runs on the device because the context lengths live there: one CTA
-// picks P from the actual lengths, then writes a work list of (sequence,
-// partition) items ordered by size, largest first (full partitions, then the
-// tails by decreasing length), so that a persistent kernel handing out items
-// through an atomic counter finishes with small items (longest processing
-// time first).
+// picks the partition size from the actual lengths, then writes a work list of
+// (sequence, partition, block range) items ordered by size, largest first, so
+// that a persistent kernel handing out items through an atomic counter
+// finishes with small items (longest processing time first).
 #include "pkv_common.cuh"
 
 namespace pkv {
@@ -23,11 +22,46 @@ constexpr int kPlanThreads = 1024;
 constexpr int kMaxBuckets = 1024;
 constexpr int kMaxCandidates = 12;
 
+// Automatic partitioning ends each context with geometrically shrinking pieces.
+#ifndef PKV_PLAN_GEOMETRIC
+#define PKV_PLAN_GEOMETRIC 1
+#endif
+
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 __device__ __forceinline__ int bucket_of(int nblk, int nb_top, int nbuckets) {
-    // bucket 0 = one block ... nbuckets-1 = a full partition
+    // bucket 0 = one block ... nbuckets-1 = a largest partition
     return (int)(((long long)(nblk - 1) * nbuckets) / nb_top);
+}
+
+// Partitions of one sequence of B blocks, in order along the context.
+//  uniform (user-fixed size): pieces of nb blocks, the last one shorter;
+//  geometric (automatic): whole pieces of nb blocks, then the remaining chunk T
+//  (1..nb blocks) halved while it exceeds 2*mb: T/2, T/4, ..., then the rest.
+//  Each piece is >= mb blocks unless the sequence is shorter, so a sequence of
+//  B blocks has at most ceil(B / mb) pieces; under longest-first scheduling the
+//  last units handed out are the small ones, which evens out the finish times.
+// Calls emit(first_block, blocks) for each piece and returns the count.
+template <typename F>
+__device__ __forceinline__ int for_each_piece(int B, int nb, int mb, bool geometric, F&& emit) {
+    if (B <= 0) return 0;
+    int count = 0, at = 0;
+    if (!geometric) {
+        for (; at < B; at += nb, ++count) emit(at, min(nb, B - at));
+        return count;
+    }
+    const int body = (B - 1) / nb;  // whole pieces before the last chunk
+    for (int i = 0; i < body; ++i, at += nb, ++count) emit(at, nb);
+    int T = B - at;
+    while (T > 2 * mb) {
+        const int piece = T / 2;
+        emit(at, piece);
+        at += piece;
+        T -= piece;
+        ++count;
+    }
+    emit(at, T);
+    return count + 1;
 }
 
 __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams p, int fixed_partition, int min_partition,
@@ -37,12 +71,14 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
     __shared__ unsigned long long units_of[kMaxCandidates];
     __shared__ int chosen;
     const int tid = threadIdx.x;
+    const bool geometric = fixed_partition == 0 && PKV_PLAN_GEOMETRIC;
+    const int mb = min_partition / kBlockSize;
 
     // The workspace and the output may still be in use by the previous kernel.
     pdl_wait();
     pdl_trigger();
 
-    // 1. partition size: the largest candidate min_partition << c whose work
+    // 1. largest partition: the largest candidate min_partition << c whose work
     //    list still has target_units units (one pass over the lengths for all c)
     if (tid < kMaxCandidates) units_of[tid] = 0;
     __syncthreads();
@@ -53,10 +89,12 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
 #pragma unroll
         for (int c = 0; c < kMaxCandidates; ++c) cnt[c] = 0;
         for (int s = tid; s < p.num_seqs; s += kPlanThreads) {
-            const int L = clamped_len(p, s, false);
+            const int B = ceil_div(clamped_len(p, s, false), kBlockSize);
 #pragma unroll
             for (int c = 0; c < kMaxCandidates; ++c)
-                if (c < num_candidates) cnt[c] += (unsigned long long)ceil_div(L, min_partition << c);
+                if (c < num_candidates)
+                    cnt[c] += (unsigned long long)for_each_piece(B, (min_partition << c) / kBlockSize, mb, geometric,
+                                                                 [](int, int) {});
         }
 #pragma unroll
         for (int c = 0; c < kMaxCandidates; ++c) {
@@ -87,10 +125,9 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
     __syncthreads();
     for (int s = tid; s < p.num_seqs; s += kPlanThreads) {
         const int L = clamped_len(p, s, true);
-        const int nfull = L / P, tail = L - nfull * P;
-        p.nparts[s] = nfull + (tail > 0);
-        if (nfull) atomicAdd(&hist[nbuckets - 1], nfull);
-        if (tail) atomicAdd(&hist[bucket_of(ceil_div(tail, kBlockSize), nb_top, nbuckets)], 1);
+        const int B = ceil_div(L, kBlockSize);
+        p.nparts[s] = for_each_piece(B, nb_top, mb, geometric,
+                                     [&](int, int n) { atomicAdd(&hist[bucket_of(n, nb_top, nbuckets)], 1); });
         if (L == 0) {
             // an empty context produces a zero output row (nothing else writes it)
             const size_t row = (size_t)s * p.num_heads * p.head_dim;
@@ -131,77 +168,14 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
     __syncthreads();
 
     // 4. scatter the items (order inside a bucket does not affect results)
-    int2* items = p.items;
     for (int s = tid; s < p.num_seqs; s += kPlanThreads) {
-        const int L = clamped_len(p, s, false);
-        const int nfull = L / P, tail = L - nfull * P;
-        if (nfull) {
-            const int base = atomicAdd(&hist[nbuckets - 1], nfull);
-            for (int j = 0; j < nfull; ++j) items[base + j] = make_int2(s, j);
-        }
-        if (tail) {
-            const int pos = atomicAdd(&hist[bucket_of(ceil_div(tail, kBlockSize), nb_top, nbuckets)], 1);
-            items[pos] = make_int2(s, nfull);
-        }
+        const int B = ceil_div(clamped_len(p, s, false), kBlockSize);
+        int part = 0;
+        for_each_piece(B, nb_top, mb, geometric, [&](int first, int n) {
+            const int pos = atomicAdd(&hist[bucket_of(n, nb_top, nbuckets)], 1);
+            p.items[pos] = make_int4(s, part++, first, n);
+        });
     }
-}
-
-// Merge of a split context, one warp per (sequence, query head): M = max_p m_p
-// over partitions with l_p > 0, w_p = l_p 2^(m_p - M), out = sum w_p o_p / sum w_p
-// (o_p normalised, m_p in base-2 units).  Sequences with one partition were
-// written by the decode kernel directly.
-template <int D, typename OutT>
-__global__ void __launch_bounds__(256) decode_merge_kernel(DecodeParams p) {
-    pdl_wait();
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (warp >= p.num_seqs * p.num_heads) return;
-    const int s = warp / p.num_heads;
-    const int n = p.nparts[s];
-    if (n <= 1) return;
-    const size_t base = (size_t)warp * p.max_parts;
-    constexpr int E = D / 32;
-    float M = -INFINITY;
-    for (int i = lane; i < n; i += 32) {
-        const float2 ml = p.part_ml[base + i];
-        if (ml.y > 0.f) M = fmaxf(M, ml.x);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float acc[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] = 0.f;
-    float W = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll 4
-        for (int i = 0; i < n; ++i) {
-            const float2 ml = p.part_ml[base + i];
-            const float w = ml.y > 0.f ? ml.y * exp2f(ml.x - M) : 0.f;
-            W += w;
-            const float* o = p.part_o + (base + i) * D + lane * E;
-#pragma unroll
-            for (int e = 0; e < E; ++e) acc[e] += w * o[e];
-        }
-    }
-    const float inv = W > 0.f ? 1.f / W : 0.f;
-    OutT* out = static_cast<OutT*>(p.out) + (size_t)warp * D + lane * E;
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-        if constexpr (sizeof(OutT) == 4)
-            out[e] = acc[e] * inv;
-        else
-            out[e] = __float2bfloat16(acc[e] * inv);
-    }
-}
-
-cudaError_t launch_decode_merge(const DecodeParams& p, int out_dtype, cudaStream_t stream) {
-    const int warps = p.num_seqs * p.num_heads;
-    const unsigned grid = (unsigned)((warps * 32 + 255) / 256);
-    if (p.head_dim == 128)
-        return out_dtype == 0 ? launch_pdl(decode_merge_kernel<128, float>, dim3(grid), dim3(256), 0, stream, p)
-                              : launch_pdl(decode_merge_kernel<128, __nv_bfloat16>, dim3(grid), dim3(256), 0, stream, p);
-    return out_dtype == 0 ? launch_pdl(decode_merge_kernel<64, float>, dim3(grid), dim3(256), 0, stream, p)
-                          : launch_pdl(decode_merge_kernel<64, __nv_bfloat16>, dim3(grid), dim3(256), 0, stream, p);
 }
 
 cudaError_t launch_decode_plan(const DecodeParams& p, int fixed_partition, int min_partition, int num_candidates,

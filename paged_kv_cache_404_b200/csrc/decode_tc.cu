@@ -117,7 +117,6 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
     }
 
     const int num_units = p.hdr->num_units;
-    const int P = p.hdr->partition;
     const int G = p.group;
     uint32_t seqno = 0;  // blocks this warp has consumed so far (stage = seqno % STAGES)
 #if PKV_DEBUG_TIMELINE
@@ -130,14 +129,14 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
         if (lane == 0) u = atomicAdd(&p.hdr->counter, 1);
         u = __shfl_sync(0xffffffffu, u, 0);
         if (u >= num_units) break;
-        const int2 item = p.items[u / p.num_kv_heads];
+        const int4 item = p.items[u / p.num_kv_heads];
         const int kvh = u - (u / p.num_kv_heads) * p.num_kv_heads;
         const int s = item.x, part = item.y;
         const int L = clamped_len(p, s, false);
-        const int t0 = part * P;
-        const int t1 = min(L, t0 + P);
+        const int blk0 = item.z;
+        const int t0 = blk0 * kBlockSize;
+        const int t1 = min(L, t0 + item.w * kBlockSize);
         const int nblk = (t1 - t0 + kBlockSize - 1) / kBlockSize;
-        const int blk0 = t0 / kBlockSize;
         const int32_t* tab = p.block_tables + (size_t)s * p.max_blocks_per_seq + blk0;
 
         // Block ids, 32 at a time: lane i holds block (32*chunk + i); the next

@@ -24,15 +24,15 @@ constexpr int kBlockSize = 16;
 // Decode workspace (caller-allocated device memory), in this order:
 //   WsHeader                       256 bytes
 //   nparts   int32 [num_seqs]      partitions of each sequence (written by the plan)
-//   items    int2  [num_seqs * max_parts]   (seq, partition) work list
+//   items    int4  [num_seqs * max_parts]   (seq, partition, first block, blocks) work list
 //   part_ml  float2[num_seqs * num_heads * max_parts]   (m, l) per partition
 //   part_o   float [num_seqs * num_heads * max_parts * head_dim]
 // Each region starts on a 256-byte boundary.
 struct WsHeader {
     int counter;        // next unit to hand out (zeroed by the plan kernel)
-    int num_items;      // (seq, partition) items in the work list
+    int num_items;      // (seq, partition, block range) items in the work list
     int num_units;      // num_items * num_kv_heads
-    int partition;      // partition size in tokens chosen for this call
+    int partition;      // largest partition in tokens chosen for this call
     int timeout;        // set when a bounded wait ran out
     int pad[59];
 };
@@ -52,7 +52,7 @@ __host__ __device__ inline WsLayout ws_layout(int num_seqs, int num_heads, int h
     L.nparts = off;
     off = pkv_align256(off + sizeof(int) * (size_t)num_seqs);
     L.items = off;
-    off = pkv_align256(off + sizeof(int2) * (size_t)num_seqs * max_parts);
+    off = pkv_align256(off + sizeof(int4) * (size_t)num_seqs * max_parts);
     L.part_ml = off;
     off = pkv_align256(off + sizeof(float2) * (size_t)num_seqs * num_heads * max_parts);
     L.part_o = off;
@@ -81,7 +81,7 @@ struct DecodeParams {
     const void* v_pool;
     WsHeader* hdr;
     int* nparts;         // written by the plan kernel
-    int2* items;         // written by the plan kernel
+    int4* items;         // written by the plan kernel: {seq, partition, first block, blocks}
     float2* part_ml;
     float* part_o;
     int max_parts;
