@@ -49,6 +49,8 @@ def lib():
                                    C.c_int, C.c_int, C.c_float, C.c_float]
         L.orc_copy_blocks.restype = C.c_int
         L.orc_copy_blocks.argtypes = [p, p, C.c_size_t, p, C.c_int, C.c_int]
+        L.orc_swap_blocks.restype = C.c_int
+        L.orc_swap_blocks.argtypes = [p, p, C.c_int, p, p, C.c_int, C.c_size_t, p, C.c_int]
         L.orc_gather.restype = C.c_int
         L.orc_gather.argtypes = [p, C.c_size_t, p, C.c_int, C.c_int, C.c_int, p]
         L.orc_paged_attention_decode.restype = C.c_int
@@ -121,6 +123,22 @@ def copy_blocks(k_pool, v_pool, pairs):
     r = lib().orc_copy_blocks(_ptr(k_pool), _ptr(v_pool), block_bytes, _ptr(pairs), pairs.shape[0], NB)
     if r < 0:
         raise ValueError("overlapping copy pairs have no defined result")
+    return r
+
+
+def swap_blocks(dst_k, dst_v, src_k, src_v, pairs):
+    """Copy whole blocks src (of the source pools) -> dst (of the destination pools).
+
+    pairs: int64 [n, 2].  Returns the number of out-of-range pairs skipped;
+    raises on a repeated dst.
+    """
+    pairs = _c(np.asarray(pairs, dtype=np.int64).reshape(-1, 2))
+    assert dst_k.shape[1:] == src_k.shape[1:] and dst_k.dtype == src_k.dtype
+    block_bytes = src_k.nbytes // src_k.shape[0]
+    r = lib().orc_swap_blocks(_ptr(dst_k), _ptr(dst_v), dst_k.shape[0], _ptr(src_k), _ptr(src_v),
+                              src_k.shape[0], block_bytes, _ptr(pairs), pairs.shape[0])
+    if r < 0:
+        raise ValueError("a repeated destination block has no defined result")
     return r
 
 

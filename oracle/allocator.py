@@ -16,12 +16,18 @@ Written from the pages' description of the host side of PagedAttention:
   only the block that must split is copied; blocks with no references are freed.
 - same glossary page, "Tecnicas relacionadas" (continuous batching): a finished
   sequence's blocks return to the free pool at once.
+- "Le cache KV et PagedAttention" (gyaansetu.com), fine-grained eviction: when
+  memory runs out, a sequence's small pages can go to the CPU instead of the
+  whole sequence being dropped, and come back later.
 
 Readings where the pages are silent: the free list is first-in first-out (pop
 from the front, freed blocks appended to the back in table order); a
 copy-on-write copies the whole block and moves the writer to the copy, leaving
 the last holder (reference count 1) to write in place; running out of free
-blocks raises MemoryError and leaves the state unchanged.
+blocks raises MemoryError and leaves the state unchanged.  Swap moves all of a
+sequence's pages at once to a host pool with its own first-in first-out free
+list (ids 0..n-1); a page shared with another sequence is copied out and comes
+back as a private block; a swapped sequence can only be swapped in or freed.
 """
 from collections import deque
 
@@ -42,6 +48,8 @@ class RefBlockManager:
         self.tables = {}
         self.lens = {}
         self._next = 0
+        self.host_free = deque()
+        self.swapped = set()
 
     # -- allocation ---------------------------------------------------------
     def _pop(self):
@@ -98,11 +106,59 @@ class RefBlockManager:
 
     def free_seq(self, seq):
         """Drop a finished sequence; blocks whose count reaches 0 return to the pool."""
-        for b in self.tables.pop(seq):
+        table = self.tables.pop(seq)
+        del self.lens[seq]
+        if seq in self.swapped:
+            self.swapped.discard(seq)
+            self.host_free.extend(table)
+            return
+        for b in table:
             self.ref[b] -= 1
             if self.ref[b] == 0:
                 self.free.append(b)
-        del self.lens[seq]
+
+    # -- swap to a host pool --------------------------------------------------
+    def set_host_pool(self, num_host_blocks):
+        assert not self.swapped, "host blocks still in use"
+        self.host_free = deque(range(num_host_blocks))
+
+    def swap_out(self, seq):
+        """Move every page of a resident sequence to host blocks.
+
+        Returns the (device block, host block) copies, in table order.
+        """
+        assert seq not in self.swapped
+        table = self.tables[seq]
+        if len(table) > len(self.host_free):
+            raise MemoryError("not enough free host blocks")
+        pairs = []
+        for i, b in enumerate(table):
+            h = self.host_free.popleft()
+            pairs.append((b, h))
+            self.ref[b] -= 1
+            if self.ref[b] == 0:
+                self.free.append(b)
+            table[i] = h
+        self.swapped.add(seq)
+        return pairs
+
+    def swap_in(self, seq):
+        """Bring a swapped sequence back into fresh device blocks.
+
+        Returns the (host block, device block) copies, in table order.
+        """
+        assert seq in self.swapped
+        table = self.tables[seq]
+        if len(table) > len(self.free):
+            raise MemoryError("not enough free blocks")
+        pairs = []
+        for i, h in enumerate(table):
+            b = self._pop()
+            pairs.append((h, b))
+            self.host_free.append(h)
+            table[i] = b
+        self.swapped.discard(seq)
+        return pairs
 
     # -- queries ------------------------------------------------------------
     def slot(self, seq, pos):

@@ -217,6 +217,29 @@ int orc_copy_blocks(void* k_pool, void* v_pool, size_t block_bytes, const int64_
     return bad;
 }
 
+/* Swap between pools (fine-grained eviction: pages move to host memory and
+ * back, "Le cache KV et PagedAttention", gyaansetu.com): for every (src, dst)
+ * pair copy block src of the source pools over block dst of the destination
+ * pools.  The pools are distinct, so only a repeated dst is order-dependent
+ * (refused: -1).  Pairs outside their pool's range are skipped and counted. */
+int orc_swap_blocks(void* dst_k, void* dst_v, int dst_blocks, const void* src_k, const void* src_v,
+                    int src_blocks, size_t block_bytes, const int64_t* pairs, int num_pairs) {
+    int i, j, bad = 0;
+    for (i = 0; i < num_pairs; i++)
+        for (j = i + 1; j < num_pairs; j++)
+            if (pairs[2 * i + 1] == pairs[2 * j + 1]) return -1;
+    for (i = 0; i < num_pairs; i++) {
+        int64_t s = pairs[2 * i], d = pairs[2 * i + 1];
+        if (s < 0 || s >= src_blocks || d < 0 || d >= dst_blocks) {
+            bad++;
+            continue;
+        }
+        memcpy((char*)dst_k + (size_t)d * block_bytes, (const char*)src_k + (size_t)s * block_bytes, block_bytes);
+        memcpy((char*)dst_v + (size_t)d * block_bytes, (const char*)src_v + (size_t)s * block_bytes, block_bytes);
+    }
+    return bad;
+}
+
 /* ---------------------------------------------------------------- gather */
 
 /* The worked example's read-back: the bytes of a request's first `len` tokens

@@ -36,6 +36,10 @@ MUTANTS = {
                              "load_src_float(v, src_dtype, (size_t)i * row + e), k_scale)"),
     "write_slot_row": ("(char*)k_pool + (size_t)slot * row * es", "(char*)k_pool + (size_t)(slot + 1) * row * es"),
     "copy_only_k": ("memcpy((char*)v_pool + (size_t)d * block_bytes", "if (0) memcpy((char*)v_pool + (size_t)d * block_bytes"),
+    "swap_only_k": ("memcpy((char*)dst_v", "if (0) memcpy((char*)dst_v"),
+    "swap_accepts_repeated_dst": ("for (j = i + 1; j < num_pairs; j++)", "for (j = num_pairs; j < num_pairs; j++)"),
+    "swap_half_block": ("(const char*)src_k + (size_t)s * block_bytes, block_bytes);",
+                        "(const char*)src_k + (size_t)s * block_bytes, block_bytes / 2);"),
     "gather_wrong_slot": ("((size_t)blk * block_size + (size_t)(t % block_size)) * row_bytes, row_bytes);",
                           "((size_t)blk * block_size + (size_t)(t / block_size)) * row_bytes, row_bytes);"),
 }
@@ -57,6 +61,7 @@ def _pins(golden):
         P.test_e4m3_encode_matches_brute_force_sweep,
         P.test_kv_write_bf16_is_raw_copy_and_touches_nothing_else,
         P.test_kv_write_fp8_matches_library_cast, P.test_copy_blocks_semantics,
+        P.test_swap_blocks_between_pools_of_different_sizes,
     ]
     return fns
 
@@ -97,7 +102,7 @@ def test_pins_reject_planted_mistake(name, golden_dir, tmp_path):
         for fn in _pins(golden_dir):
             try:
                 fn()
-            except Exception as e:  # noqa: BLE001 - any failure counts as a catch
+            except (Exception, pytest.fail.Exception) as e:  # noqa: BLE001 - any failure counts as a catch
                 caught.append(repr(e)[:80])
                 break
     finally:
@@ -132,3 +137,48 @@ def test_pins_reject_allocator_copying_for_last_holder(monkeypatch):
     monkeypatch.setattr(allocator.RefBlockManager, "append_token", bad_append)
     with pytest.raises(AssertionError):
         A.test_parallel_sampling_cow_trace()
+
+
+def test_pins_reject_swap_out_that_keeps_device_blocks(monkeypatch):
+    """Planted mistake in the reference block manager: swap-out copies the pages
+    but never returns the device blocks to the free list."""
+    from oracle import allocator
+
+    def bad_swap_out(self, seq):
+        table = self.tables[seq]
+        if len(table) > len(self.host_free):
+            raise MemoryError("not enough free host blocks")
+        pairs = []
+        for i, b in enumerate(table):
+            h = self.host_free.popleft()
+            pairs.append((b, h))
+            self.ref[b] -= 1               # the planted mistake: no return to the free list
+            table[i] = h
+        self.swapped.add(seq)
+        return pairs
+
+    monkeypatch.setattr(allocator.RefBlockManager, "swap_out", bad_swap_out)
+    with pytest.raises(AssertionError):
+        A.test_swap_round_trip_restores_every_token()
+
+
+def test_pins_reject_swap_in_that_restores_old_block_ids(monkeypatch):
+    """Planted mistake: swap-in writes the pages back to the block ids they left,
+    which other sequences may own by then."""
+    from oracle import allocator
+
+    def bad_swap_in(self, seq):
+        table = self.tables[seq]
+        pairs = []
+        for i, h in enumerate(table):
+            b = h                          # the planted mistake: host id reused as device id
+            self.ref[b] += 1
+            pairs.append((h, b))
+            self.host_free.append(h)
+            table[i] = b
+        self.swapped.discard(seq)
+        return pairs
+
+    monkeypatch.setattr(allocator.RefBlockManager, "swap_in", bad_swap_in)
+    with pytest.raises(AssertionError):
+        A.test_swap_round_trip_restores_every_token()

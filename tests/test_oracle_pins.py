@@ -445,3 +445,26 @@ def test_copy_blocks_semantics():
         oracle.copy_blocks(kp, vp, [[1, 5], [2, 5]])
     with pytest.raises(ValueError):
         oracle.copy_blocks(kp, vp, [[1, 5], [5, 6]])
+
+
+def test_swap_blocks_between_pools_of_different_sizes():
+    """Cross-pool page copy: block src of the source pool lands in block dst of the
+    destination pool, nothing else changes (fancy indexing is the brute force)."""
+    rng = np.random.default_rng(19)
+    dk = rng.standard_normal((6, 16, 2, 8)).astype(np.float32)
+    dv = rng.standard_normal((6, 16, 2, 8)).astype(np.float32)
+    hk = np.zeros((9, 16, 2, 8), np.float32)
+    hv = np.zeros((9, 16, 2, 8), np.float32)
+    pairs = np.array([[5, 8], [0, 2], [3, 0], [6, 1], [1, 9], [-2, 3]])
+    assert oracle.swap_blocks(hk, hv, dk, dv, pairs) == 3
+    ek, ev = np.zeros_like(hk), np.zeros_like(hv)
+    ek[[8, 2, 0]], ev[[8, 2, 0]] = dk[[5, 0, 3]], dv[[5, 0, 3]]
+    assert np.array_equal(hk, ek) and np.array_equal(hv, ev)
+    d0 = dk.copy()
+    assert oracle.swap_blocks(dk, dv, hk, hv, [[8, 1]]) == 0      # and back, into another block
+    assert np.array_equal(dk[1], d0[5]) and np.array_equal(np.delete(dk, 1, 0), np.delete(d0, 1, 0))
+    with pytest.raises(ValueError):
+        oracle.swap_blocks(hk, hv, dk, dv, [[0, 4], [1, 4]])
+    # the same src twice is fine (two copies of one page)
+    assert oracle.swap_blocks(hk, hv, dk, dv, [[2, 4], [2, 5]]) == 0
+    assert np.array_equal(hk[4], dk[2]) and np.array_equal(hk[5], dk[2])
