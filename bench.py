@@ -20,6 +20,12 @@ the max over ranks and the value the sum over ranks (weak scaling).
 
 --impl reference times the CPU oracle (the plain fp64 reference) on a bounded
 sample of the same workload, on this host's cores.
+
+--swap measures block swap instead (a separate line, not the headline): a
+quarter of the gqa70b batch (64 sequences x 4,096 tokens, 1 GiB of K+V) moves
+from scattered device blocks to a page-locked host pool and back through
+pkv_swap_blocks; the roofline is one contiguous copy-engine transfer of the
+same bytes in the same direction, measured in the same run.
 """
 import argparse
 import hashlib
@@ -315,6 +321,7 @@ def time_e2e(step: Step, steps: int, warmup: int, world: int):
     uploaded = [torch.cuda.Event() for _ in range(2)]
     computed = [torch.cuda.Event() for _ in range(2)]
     consumed = [torch.cuda.Event() for _ in range(2)]   # set b's inputs no longer needed
+    downloaded = [torch.cuda.Event() for _ in range(2)]  # output b read back: free to overwrite
 
     def run(n_steps):
         for i in range(n_steps):
@@ -326,6 +333,8 @@ def time_e2e(step: Step, steps: int, warmup: int, world: int):
                     dev[b][n].copy_(host[n], non_blocking=True)
                 uploaded[b].record(up)
             compute.wait_event(uploaded[b])
+            if i >= 2:
+                compute.wait_event(downloaded[b])
             for n in names:
                 setattr(step, n, dev[b][n])
             step.out = outs[b]
@@ -335,6 +344,7 @@ def time_e2e(step: Step, steps: int, warmup: int, world: int):
             with torch.cuda.stream(down):
                 down.wait_event(computed[b])
                 out_host[b].copy_(outs[b], non_blocking=True)
+                downloaded[b].record(down)
         compute.wait_stream(up)
         compute.wait_stream(down)
 
@@ -460,6 +470,84 @@ def run_reference(args, w, rank, world):
 
 # ------------------------------------------------------------------ main
 
+def run_swap(args, device):
+    """Swap-out and swap-in throughput of pkv_swap_blocks over the host link."""
+    import paged_kv_cache_404_b200 as pkv
+    w = W.WORKLOADS["gqa70b"]
+    nseq = args.num_seqs or 64
+    per_seq = -(-w.len_lo // 16)
+    blocks = nseq * per_seq
+    NB = int(blocks * 2)
+    bm = pkv.BlockManager(NB, 16, free_order=W.free_order(w, NB))
+    others = bm.alloc_seq((NB - blocks) * 16 // 2)          # scatter: half the pool held elsewhere
+    ids = [bm.alloc_seq(w.len_lo) for _ in range(nseq)]
+    bm.set_host_pool(blocks)
+    out_pairs = np.concatenate([bm.swap_out(s) for s in ids])
+    in_pairs = np.concatenate([bm.swap_in(s) for s in ids])
+    del others
+    shape = (16, w.num_kv_heads, w.head_dim)
+    dk = torch.randn((NB,) + shape, device=device).to(torch.bfloat16)
+    dv = torch.randn((NB,) + shape, device=device).to(torch.bfloat16)
+    hk = torch.empty((blocks,) + shape, dtype=torch.bfloat16).pin_memory()
+    hv = torch.empty((blocks,) + shape, dtype=torch.bfloat16).pin_memory()
+    g_out = torch.from_numpy(out_pairs).to(device)
+    g_in = torch.from_numpy(in_pairs).to(device)
+    nbytes = 2 * blocks * dk[0].numel() * 2
+    err = torch.zeros(1, dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, reps):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms.append(a.elapsed_time(b))
+        return statistics.median(ms)
+
+    reps = max(3, min(args.steps, 20))
+    with ClockSampler(device) as clk:
+        out_ms = timed(lambda: pkv.swap_blocks(hk, hv, dk, dv, g_out, err_count=err), reps)
+        in_ms = timed(lambda: pkv.swap_blocks(dk, dv, hk, hv, g_in, err_count=err), reps)
+        # copy-engine reference: the same bytes as two contiguous transfers per direction
+        ck, cv = dk[:blocks], dv[:blocks]
+        d2h_ms = timed(lambda: (hk.copy_(ck, non_blocking=True), hv.copy_(cv, non_blocking=True)), reps)
+        h2d_ms = timed(lambda: (ck.copy_(hk, non_blocking=True), cv.copy_(hv, non_blocking=True)), reps)
+    torch.cuda.synchronize()
+    # bytes check: after a swap-out and a swap-in, sampled blocks hold what the host pool holds
+    pkv.swap_blocks(hk, hv, dk, dv, g_out, err_count=err)
+    pkv.swap_blocks(dk, dv, hk, hv, g_in, err_count=err)
+    torch.cuda.synchronize()
+    probe = in_pairs[:: max(1, blocks // 64)]
+    ok = bool(torch.equal(dk[torch.from_numpy(probe[:, 1]).to(device)].cpu(), hk[torch.from_numpy(probe[:, 0])]))
+    ok = ok and int(err.item()) == 0
+    gbs = lambda ms: round(nbytes / (ms / 1e3) / 1e9, 2)  # noqa: E731
+    line = {
+        "metric": "block swap over the host link: GB/s (K+V bytes moved / time)",
+        "value": round(2 * nbytes / ((out_ms + in_ms) / 1e3) / 1e9, 2),
+        "unit": "GB/s", "n_gpus": 1, "steps": reps, "warmup": 3, "ms_per_step": round(out_ms + in_ms, 4),
+        "higher_is_better": True, "dtype": "bf16 (byte copy)", "data": "synthetic",
+        "config": {"workload": "swap: %d sequences x %d tokens of gqa70b (8 kv heads, head_dim 128, bf16), "
+                               "%d scattered device blocks <-> page-locked host pool" % (nseq, w.len_lo, blocks),
+                   "bytes_per_direction": nbytes},
+        "swap_out": {"ms": round(out_ms, 4), "GB/s": gbs(out_ms), "copy_engine_GB/s": gbs(d2h_ms),
+                     "frac": round(d2h_ms / out_ms, 4)},
+        "swap_in": {"ms": round(in_ms, 4), "GB/s": gbs(in_ms), "copy_engine_GB/s": gbs(h2d_ms),
+                    "frac": round(h2d_ms / in_ms, 4)},
+        "roofline": {"bound": "host link", "achieved": round(2 * nbytes / ((out_ms + in_ms) / 1e3) / 1e9, 2),
+                     "peak": round(2 * nbytes / ((d2h_ms + h2d_ms) / 1e3) / 1e9, 2), "unit": "GB/s",
+                     "frac": round((d2h_ms + h2d_ms) / (out_ms + in_ms), 4),
+                     "peak_source": "contiguous cudaMemcpyAsync of the same bytes, measured in this run"},
+        "gpu_launches": 2 * reps, "bytes_restored": ok, "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -472,6 +560,7 @@ def main(argv=None):
                     help="fewer sequences of the same shape (small cases for profiling; not a bench line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--swap", action="store_true", help="measure block swap to a host pool instead")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
 
@@ -487,6 +576,9 @@ def main(argv=None):
     if rank == 0:
         pkv_build.build()
     torch.cuda.set_device(local)
+    if args.swap:
+        run_swap(args, torch.device("cuda", local))
+        return
     device = torch.device("cuda", local)
     if world > 1:
         import datetime

@@ -70,7 +70,8 @@ typedef enum pkv_status {
     PKV_EUNSUPPORTED = 2,  /* valid but not implemented: block_size, head_dim, dtype combination, group */
     PKV_ECUDA = 3,         /* a CUDA runtime/driver call failed (launch error, no device) */
     PKV_ENOMEM = 4,        /* block manager: not enough free blocks */
-    PKV_ENOENT = 5         /* block manager: no such sequence */
+    PKV_ENOENT = 5,        /* block manager: no such sequence */
+    PKV_ESWAPPED = 6       /* block manager: the sequence is swapped out to the host pool */
 } pkv_status;
 
 typedef enum pkv_dtype {
@@ -228,6 +229,29 @@ int pkv_copy_blocks(void* k_pool, void* v_pool, size_t block_bytes,
                     int32_t* err_count, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Block swap between pools: for every pair (src, dst) copy the whole block src
+ * of the source pools over block dst of the destination pools (K and V).
+ * Source: when memory runs out, small pages are moved to the CPU instead of
+ * whole sequences, and brought back later ("Le cache KV et PagedAttention",
+ * gyaansetu.com, section "Comment PagedAttention resout ce probleme": fine-
+ * grained eviction); with pkv_copy_blocks it is the copy of one page.
+ *
+ *   dst_k_pool, dst_v_pool  dst_num_blocks blocks of block_bytes each
+ *   src_k_pool, src_v_pool  src_num_blocks blocks of block_bytes each
+ *   src_dst_pairs           int64 [num_pairs][2], device-accessible
+ * Any pointer may be device memory or page-locked host memory that the device
+ * can address (cudaHostAlloc, torch pin_memory): the GPU moves the bytes over
+ * the host link itself, so swap-out is (device pool -> host pool) and swap-in
+ * (host pool -> device pool).  Pageable host memory is refused (PKV_EINVAL).
+ * Pairs out of range are skipped and counted; a dst that repeats gives an
+ * undefined result.  num_pairs == 0 launches nothing.
+ * ---------------------------------------------------------------------- */
+int pkv_swap_blocks(void* dst_k_pool, void* dst_v_pool, int dst_num_blocks,
+                    const void* src_k_pool, const void* src_v_pool, int src_num_blocks,
+                    size_t block_bytes, const int64_t* src_dst_pairs, int num_pairs,
+                    int32_t* err_count, void* stream);
+
+/* ------------------------------------------------------------------------
  * Host block manager (CPU only; no CUDA calls).  It decides where tokens go:
  * lazy allocation of a new block only when the last one is full, taken from
  * the front of a first-in first-out free list (glossary entry, worked example
@@ -271,6 +295,28 @@ int pkv_bm_tables(const pkv_block_manager* bm, const int32_t* seqs, int n, int32
                   int max_blocks, int32_t pad, int32_t* lens);
 /* Current free list, front first (n_out entries). */
 int pkv_bm_free_list(const pkv_block_manager* bm, int32_t* out, int cap, int* n_out);
+
+/* Host pool for swapping (fine-grained eviction, see pkv_swap_blocks): give the
+ * manager num_host_blocks host blocks (ids 0..n-1, free list in id order).
+ * swap_out moves a resident sequence's pages to host blocks: it appends one
+ * (device block, host block) pair per table entry to pairs_out (capacity =
+ * table length), drops the sequence's references to its device blocks (a block
+ * another sequence still uses stays on the device) and leaves the sequence
+ * "swapped" (its table now holds host ids).  swap_in is the reverse: fresh
+ * device blocks from the free list, (host block, device block) pairs, host
+ * blocks freed.  Both return PKV_ENOMEM, with nothing changed, if the target
+ * pool has too few free blocks, and PKV_EINVAL if cap is below the table
+ * length.  A page shared with another sequence is copied out like any other,
+ * and comes back as a private block: sharing is not restored.  A swapped
+ * sequence can be swapped in, freed (its host blocks return to the host free
+ * list) or queried (seq_len, block_table: host ids, is_swapped); fork,
+ * append_tokens, slots and tables return PKV_ESWAPPED.  set_host_pool returns
+ * PKV_EINVAL while any host block is in use. */
+int pkv_bm_set_host_pool(pkv_block_manager* bm, int num_host_blocks);
+int pkv_bm_swap_out(pkv_block_manager* bm, int32_t seq, int64_t* pairs_out, int cap, int* num_pairs_out);
+int pkv_bm_swap_in(pkv_block_manager* bm, int32_t seq, int64_t* pairs_out, int cap, int* num_pairs_out);
+int pkv_bm_is_swapped(const pkv_block_manager* bm, int32_t seq, int* swapped_out);
+int pkv_bm_num_free_host(const pkv_block_manager* bm);
 
 #ifdef __cplusplus
 }

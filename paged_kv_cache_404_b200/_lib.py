@@ -9,7 +9,7 @@ import os
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libpagedkv.so")
 
-PKV_OK, PKV_EINVAL, PKV_EUNSUPPORTED, PKV_ECUDA, PKV_ENOMEM, PKV_ENOENT = range(6)
+PKV_OK, PKV_EINVAL, PKV_EUNSUPPORTED, PKV_ECUDA, PKV_ENOMEM, PKV_ENOENT, PKV_ESWAPPED = range(7)
 PKV_F32, PKV_BF16, PKV_FP8_E4M3 = 0, 1, 2
 
 # Every exported symbol of include/pagedkv.h with (restype, argtypes).
@@ -24,6 +24,7 @@ SIGNATURES = {
     "pkv_paged_attention_decode_noalloc": (_i, [_p, _p, _i, _p, _p, _i, _p, _i, _p, _i, _i, _i, _i, _i, _i, _i,
                                                 _f, _f, _f, _i, _p, _p]),
     "pkv_copy_blocks": (_i, [_p, _p, _z, _p, _i, _i, _p, _p]),
+    "pkv_swap_blocks": (_i, [_p, _p, _i, _p, _p, _i, _z, _p, _i, _p, _p]),
     "pkv_bm_create": (_i, [_i, _i, _p, _i, C.POINTER(_p)]),
     "pkv_bm_destroy": (None, [_p]),
     "pkv_bm_alloc_seq": (_i, [_p, _i, _p]),
@@ -37,6 +38,11 @@ SIGNATURES = {
     "pkv_bm_slots": (_i, [_p, C.c_int32, _i, _i, _p]),
     "pkv_bm_tables": (_i, [_p, _p, _i, _p, _i, C.c_int32, _p]),
     "pkv_bm_free_list": (_i, [_p, _p, _i, _p]),
+    "pkv_bm_set_host_pool": (_i, [_p, _i]),
+    "pkv_bm_swap_out": (_i, [_p, C.c_int32, _p, _i, _p]),
+    "pkv_bm_swap_in": (_i, [_p, C.c_int32, _p, _i, _p]),
+    "pkv_bm_is_swapped": (_i, [_p, C.c_int32, _p]),
+    "pkv_bm_num_free_host": (_i, [_p]),
 }
 
 _lib = None

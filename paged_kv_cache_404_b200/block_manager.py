@@ -106,3 +106,31 @@ class BlockManager:
         out = np.empty(max(n.value, 1), dtype=np.int32)
         L.check("pkv_bm_free_list", self._lib.pkv_bm_free_list(self._h, out.ctypes.data, out.size, C.byref(n)))
         return out[:n.value].copy()
+
+    # --- host pool and swap (fine-grained eviction) -------------------------
+
+    def set_host_pool(self, num_host_blocks):
+        L.check("pkv_bm_set_host_pool", self._lib.pkv_bm_set_host_pool(self._h, int(num_host_blocks)))
+
+    def _swap(self, fn, name, seq):
+        n = C.c_int()
+        cap = max(len(self.block_table(seq)), 1)
+        pairs = np.empty((cap, 2), dtype=np.int64)
+        L.check(name, fn(self._h, int(seq), pairs.ctypes.data, cap, C.byref(n)))
+        return pairs[:n.value].copy()
+
+    def swap_out(self, seq):
+        """Move a sequence to host blocks; returns (device block, host block) pairs int64 [k, 2]."""
+        return self._swap(self._lib.pkv_bm_swap_out, "pkv_bm_swap_out", seq)
+
+    def swap_in(self, seq):
+        """Bring a swapped sequence back; returns (host block, device block) pairs int64 [k, 2]."""
+        return self._swap(self._lib.pkv_bm_swap_in, "pkv_bm_swap_in", seq)
+
+    def is_swapped(self, seq):
+        out = C.c_int()
+        L.check("pkv_bm_is_swapped", self._lib.pkv_bm_is_swapped(self._h, int(seq), C.byref(out)))
+        return bool(out.value)
+
+    def num_free_host(self):
+        return self._lib.pkv_bm_num_free_host(self._h)

@@ -10,8 +10,9 @@ namespace pkv {
 cudaError_t launch_kv_write(const void* k, const void* v, int src_dtype, const int64_t* slots, int num_tokens,
                             void* k_pool, void* v_pool, int cache_dtype, long long num_slots, int row_elems,
                             float k_scale, float v_scale, int32_t* err, cudaStream_t stream);
-cudaError_t launch_copy_blocks(void* k_pool, void* v_pool, size_t block_bytes, const int64_t* pairs, int num_pairs,
-                               int num_blocks, int32_t* err, cudaStream_t stream);
+cudaError_t launch_copy_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v, size_t block_bytes,
+                               const int64_t* pairs, int num_pairs, int src_blocks, int dst_blocks, int32_t* err,
+                               cudaStream_t stream);
 cudaError_t launch_decode_plan(const DecodeParams& p, int fixed_partition, int min_partition, int num_candidates,
                                int target_units, int out_dtype, cudaStream_t stream);
 cudaError_t launch_decode_tc(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeParams& p, bool fp8,
@@ -98,6 +99,7 @@ const char* pkv_status_string(int status) {
         case PKV_ECUDA: return "CUDA error";
         case PKV_ENOMEM: return "out of free blocks";
         case PKV_ENOENT: return "no such sequence";
+        case PKV_ESWAPPED: return "sequence is swapped out to the host pool";
         default: return "unknown status";
     }
 }
@@ -240,8 +242,56 @@ int pkv_copy_blocks(void* k_pool, void* v_pool, size_t block_bytes, const int64_
     // grid.y carries the pair index: launch in slices of at most 65535 pairs
     for (int first = 0; first < num_pairs; first += 65535) {
         const int n = num_pairs - first < 65535 ? num_pairs - first : 65535;
-        cudaError_t e = launch_copy_blocks(k_pool, v_pool, block_bytes, src_dst_pairs + 2 * (size_t)first, n,
-                                           num_blocks, err_count, static_cast<cudaStream_t>(stream));
+        cudaError_t e = launch_copy_blocks(k_pool, v_pool, k_pool, v_pool, block_bytes,
+                                           src_dst_pairs + 2 * (size_t)first, n, num_blocks, num_blocks, err_count,
+                                           static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return PKV_ECUDA;
+    }
+    return PKV_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+// Address the device uses for `p`: device or managed memory as is, page-locked
+// host memory through its device mapping; nullptr if the device cannot reach it
+// (pageable host memory, unknown pointer).
+const void* device_view(const void* p) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();  // clear the error this query left as the runtime's last error
+        return nullptr;
+    }
+    if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) return p;
+    if (a.type == cudaMemoryTypeHost) return a.devicePointer;
+    return nullptr;
+}
+
+}  // namespace
+
+extern "C" {
+
+int pkv_swap_blocks(void* dst_k_pool, void* dst_v_pool, int dst_num_blocks, const void* src_k_pool,
+                    const void* src_v_pool, int src_num_blocks, size_t block_bytes, const int64_t* src_dst_pairs,
+                    int num_pairs, int32_t* err_count, void* stream) {
+    if (num_pairs < 0 || dst_num_blocks <= 0 || src_num_blocks <= 0 || block_bytes == 0 || block_bytes % 16 != 0)
+        return PKV_EINVAL;
+    if (num_pairs == 0) return PKV_OK;
+    if (!dst_k_pool || !dst_v_pool || !src_k_pool || !src_v_pool || !src_dst_pairs) return PKV_EINVAL;
+    if (!aligned(dst_k_pool, 16) || !aligned(dst_v_pool, 16) || !aligned(src_k_pool, 16) ||
+        !aligned(src_v_pool, 16) || !aligned(src_dst_pairs, 8) || !aligned(err_count, 4))
+        return PKV_EINVAL;
+    void* dk = const_cast<void*>(device_view(dst_k_pool));
+    void* dv = const_cast<void*>(device_view(dst_v_pool));
+    const void* sk = device_view(src_k_pool);
+    const void* sv = device_view(src_v_pool);
+    const int64_t* pr = static_cast<const int64_t*>(device_view(src_dst_pairs));
+    if (!dk || !dv || !sk || !sv || !pr) return PKV_EINVAL;
+    for (int first = 0; first < num_pairs; first += 65535) {
+        const int n = num_pairs - first < 65535 ? num_pairs - first : 65535;
+        cudaError_t e = launch_copy_blocks(dk, dv, sk, sv, block_bytes, pr + 2 * (size_t)first, n, src_num_blocks,
+                                           dst_num_blocks, err_count, static_cast<cudaStream_t>(stream));
         if (e != cudaSuccess) return PKV_ECUDA;
     }
     return PKV_OK;

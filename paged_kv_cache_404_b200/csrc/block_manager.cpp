@@ -15,7 +15,11 @@
 //    (iplexlaw.co.kr, "two answers to one request");
 //  - release: a finished sequence drops its references and blocks whose count
 //    reaches zero return to the back of the free list at once (glossary entry,
-//    continuous batching).
+//    continuous batching);
+//  - swap: a sequence's pages can move to a host pool and back, page by page,
+//    instead of evicting whole sequences ("Le cache KV et PagedAttention",
+//    fine-grained eviction); the manager decides the block pairs, the copies
+//    run on the GPU (pkv_swap_blocks).
 // Plain C++ with host memory only; exported through the C ABI in pagedkv.h.
 #include <cstdint>
 #include <cstring>
@@ -33,8 +37,17 @@ struct pkv_block_manager {
     std::vector<std::vector<int32_t>> tables;   // per sequence id
     std::vector<int32_t> lens;                  // tokens per sequence
     std::vector<uint8_t> alive;
+    std::vector<uint8_t> swapped;               // table holds host block ids
+    int num_host_blocks = 0;
+    std::deque<int32_t> host_free;
+    std::vector<uint8_t> host_used;
 
     bool valid_seq(int32_t s) const { return s >= 0 && (size_t)s < tables.size() && alive[s]; }
+    // resident (on the device) sequence: PKV_OK, else the error to return
+    int resident(int32_t s) const {
+        if (!valid_seq(s)) return PKV_ENOENT;
+        return swapped[s] ? PKV_ESWAPPED : PKV_OK;
+    }
 
     int32_t take_block() {
         const int32_t b = free_list.front();
@@ -47,6 +60,7 @@ struct pkv_block_manager {
         tables.push_back(std::move(table));
         lens.push_back(len);
         alive.push_back(1);
+        swapped.push_back(0);
         return (int32_t)(tables.size() - 1);
     }
 };
@@ -94,7 +108,7 @@ int pkv_bm_alloc_seq(pkv_block_manager* bm, int num_tokens, int32_t* seq_out) {
 
 int pkv_bm_fork(pkv_block_manager* bm, int32_t parent, int32_t* child_out) {
     if (bm == nullptr || child_out == nullptr) return PKV_EINVAL;
-    if (!bm->valid_seq(parent)) return PKV_ENOENT;
+    if (int st = bm->resident(parent)) return st;
     std::vector<int32_t> table = bm->tables[parent];
     for (int32_t b : table) ++bm->refs[b];
     *child_out = bm->new_seq(std::move(table), bm->lens[parent]);
@@ -110,8 +124,8 @@ int pkv_bm_append_tokens(pkv_block_manager* bm, const int32_t* seqs, int n, int6
     int status = PKV_OK;
     for (; done < n; ++done) {
         const int32_t s = seqs[done];
-        if (!bm->valid_seq(s)) {
-            status = PKV_ENOENT;
+        if (int st = bm->resident(s)) {
+            status = st;
             break;
         }
         std::vector<int32_t>& table = bm->tables[s];
@@ -149,13 +163,21 @@ int pkv_bm_append_tokens(pkv_block_manager* bm, const int32_t* seqs, int n, int6
 int pkv_bm_free_seq(pkv_block_manager* bm, int32_t seq) {
     if (bm == nullptr) return PKV_EINVAL;
     if (!bm->valid_seq(seq)) return PKV_ENOENT;
-    for (int32_t b : bm->tables[seq]) {
-        if (--bm->refs[b] == 0) bm->free_list.push_back(b);
+    if (bm->swapped[seq]) {
+        for (int32_t h : bm->tables[seq]) {
+            bm->host_used[h] = 0;
+            bm->host_free.push_back(h);
+        }
+    } else {
+        for (int32_t b : bm->tables[seq]) {
+            if (--bm->refs[b] == 0) bm->free_list.push_back(b);
+        }
     }
     bm->tables[seq].clear();
     bm->tables[seq].shrink_to_fit();
     bm->lens[seq] = 0;
     bm->alive[seq] = 0;
+    bm->swapped[seq] = 0;
     return PKV_OK;
 }
 
@@ -186,7 +208,7 @@ int pkv_bm_block_table(const pkv_block_manager* bm, int32_t seq, int32_t* out, i
 
 int pkv_bm_slots(const pkv_block_manager* bm, int32_t seq, int start, int count, int64_t* out) {
     if (bm == nullptr || start < 0 || count < 0 || (count > 0 && out == nullptr)) return PKV_EINVAL;
-    if (!bm->valid_seq(seq)) return PKV_ENOENT;
+    if (int st = bm->resident(seq)) return st;
     const std::vector<int32_t>& t = bm->tables[seq];
     if ((size_t)start + count > t.size() * (size_t)bm->block_size) return PKV_EINVAL;
     for (int i = 0; i < count; ++i) {
@@ -201,7 +223,7 @@ int pkv_bm_tables(const pkv_block_manager* bm, const int32_t* seqs, int n, int32
     if (bm == nullptr || n < 0 || max_blocks <= 0 || (n > 0 && (seqs == nullptr || tables == nullptr)))
         return PKV_EINVAL;
     for (int i = 0; i < n; ++i) {
-        if (!bm->valid_seq(seqs[i])) return PKV_ENOENT;
+        if (int st = bm->resident(seqs[i])) return st;
         const std::vector<int32_t>& t = bm->tables[seqs[i]];
         if ((int)t.size() > max_blocks) return PKV_EINVAL;
         int32_t* row = tables + (size_t)i * max_blocks;
@@ -219,5 +241,72 @@ int pkv_bm_free_list(const pkv_block_manager* bm, int32_t* out, int cap, int* n_
     for (int32_t b : bm->free_list) out[i++] = b;
     return PKV_OK;
 }
+
+int pkv_bm_set_host_pool(pkv_block_manager* bm, int num_host_blocks) {
+    if (bm == nullptr || num_host_blocks < 0) return PKV_EINVAL;
+    for (uint8_t u : bm->host_used)
+        if (u) return PKV_EINVAL;  // host blocks still hold swapped pages
+    bm->num_host_blocks = num_host_blocks;
+    bm->host_used.assign(num_host_blocks, 0);
+    bm->host_free.clear();
+    for (int h = 0; h < num_host_blocks; ++h) bm->host_free.push_back(h);
+    return PKV_OK;
+}
+
+int pkv_bm_swap_out(pkv_block_manager* bm, int32_t seq, int64_t* pairs_out, int cap, int* num_pairs_out) {
+    if (bm == nullptr || num_pairs_out == nullptr || cap < 0) return PKV_EINVAL;
+    if (int st = bm->resident(seq)) return st;
+    std::vector<int32_t>& table = bm->tables[seq];
+    const int k = (int)table.size();
+    *num_pairs_out = 0;
+    if (k > cap || (k > 0 && pairs_out == nullptr)) return PKV_EINVAL;
+    if ((size_t)k > bm->host_free.size()) return PKV_ENOMEM;
+    for (int i = 0; i < k; ++i) {
+        const int32_t h = bm->host_free.front();
+        bm->host_free.pop_front();
+        bm->host_used[h] = 1;
+        const int32_t d = table[i];
+        pairs_out[2 * i] = d;
+        pairs_out[2 * i + 1] = h;
+        // a page another sequence still uses stays on the device
+        if (--bm->refs[d] == 0) bm->free_list.push_back(d);
+        table[i] = h;
+    }
+    bm->swapped[seq] = 1;
+    *num_pairs_out = k;
+    return PKV_OK;
+}
+
+int pkv_bm_swap_in(pkv_block_manager* bm, int32_t seq, int64_t* pairs_out, int cap, int* num_pairs_out) {
+    if (bm == nullptr || num_pairs_out == nullptr || cap < 0) return PKV_EINVAL;
+    if (!bm->valid_seq(seq)) return PKV_ENOENT;
+    if (!bm->swapped[seq]) return PKV_EINVAL;
+    std::vector<int32_t>& table = bm->tables[seq];
+    const int k = (int)table.size();
+    *num_pairs_out = 0;
+    if (k > cap || (k > 0 && pairs_out == nullptr)) return PKV_EINVAL;
+    if ((size_t)k > bm->free_list.size()) return PKV_ENOMEM;
+    for (int i = 0; i < k; ++i) {
+        const int32_t h = table[i];
+        const int32_t d = bm->take_block();
+        pairs_out[2 * i] = h;
+        pairs_out[2 * i + 1] = d;
+        bm->host_used[h] = 0;
+        bm->host_free.push_back(h);
+        table[i] = d;
+    }
+    bm->swapped[seq] = 0;
+    *num_pairs_out = k;
+    return PKV_OK;
+}
+
+int pkv_bm_is_swapped(const pkv_block_manager* bm, int32_t seq, int* swapped_out) {
+    if (bm == nullptr || swapped_out == nullptr) return PKV_EINVAL;
+    if (!bm->valid_seq(seq)) return PKV_ENOENT;
+    *swapped_out = bm->swapped[seq];
+    return PKV_OK;
+}
+
+int pkv_bm_num_free_host(const pkv_block_manager* bm) { return bm ? (int)bm->host_free.size() : -1; }
 
 }  // extern "C"

@@ -116,3 +116,28 @@ def copy_blocks(k_pool, v_pool, src_dst_pairs, err_count=None, stream=None):
     st = L.lib().pkv_copy_blocks(_ptr(k_pool), _ptr(v_pool), block_bytes, _ptr(src_dst_pairs),
                                  int(src_dst_pairs.numel() // 2), NB, _ptr(err_count), _stream(stream))
     L.check("pkv_copy_blocks", st)
+
+
+def _pool_ptr(t):
+    """Pointer of a pool that may live on the device or in page-locked host memory."""
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    if not t.is_cuda and not t.is_pinned():
+        raise ValueError("a host pool must be page-locked (pin_memory)")
+    return C.c_void_p(t.data_ptr())
+
+
+def swap_blocks(dst_k, dst_v, src_k, src_v, src_dst_pairs, err_count=None, stream=None):
+    """Copy whole blocks between pools (device <-> pinned host).
+
+    src_dst_pairs: int64 [n, 2], on the device or in page-locked host memory.
+    """
+    if src_dst_pairs.dtype != torch.int64:
+        raise TypeError("src_dst_pairs must be int64")
+    if dst_k.shape[1:] != src_k.shape[1:] or dst_k.dtype != src_k.dtype:
+        raise ValueError("pools differ in block shape or dtype")
+    block_bytes = src_k[0].numel() * src_k.element_size()
+    st = L.lib().pkv_swap_blocks(_pool_ptr(dst_k), _pool_ptr(dst_v), dst_k.shape[0], _pool_ptr(src_k),
+                                 _pool_ptr(src_v), src_k.shape[0], block_bytes, _pool_ptr(src_dst_pairs),
+                                 int(src_dst_pairs.numel() // 2), _ptr(err_count), _stream(stream))
+    L.check("pkv_swap_blocks", st)

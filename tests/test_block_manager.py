@@ -33,8 +33,10 @@ def _same_state(bm, ref, live):
     for s in live:
         assert bm.block_table(s).tolist() == ref.tables[s]
         assert bm.seq_len(s) == ref.lens[s]
+        assert bm.is_swapped(s) == (s in ref.swapped)
     for b in range(ref.num_blocks):
         assert bm.refcount(b) == ref.ref[b]
+    assert bm.num_free_host() == len(ref.host_free)
 
 
 @pytest.mark.parametrize("seed", [0, 1, 2])
@@ -120,3 +122,91 @@ def test_errors(BM):
         bm.free_seq(3)
     with pytest.raises(PagedKVError):
         BM(4, 16, free_order=[0, 0])
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_random_traces_with_swaps_match_reference(BM, seed):
+    """Allocation, fork, copy-on-write, release and swap to a host pool: the
+    native manager emits the same pairs and reaches the same state."""
+    from paged_kv_cache_404_b200 import PagedKVError
+    rng = np.random.default_rng(100 + seed)
+    NB, NH = 160, 120
+    order = rng.permutation(NB)
+    bm, ref = BM(NB, 16, free_order=order), RefBlockManager(NB, 16, free_order=order)
+    bm.set_host_pool(NH)
+    ref.set_host_pool(NH)
+    live = []
+    for step in range(2500):
+        op = int(rng.integers(0, 12))
+        if op == 0 or not live:
+            n = int(rng.integers(0, 70))
+            try:
+                r = ref.alloc_seq(n)
+            except MemoryError:
+                with pytest.raises(PagedKVError):
+                    bm.alloc_seq(n)
+                continue
+            assert bm.alloc_seq(n) == r
+            live.append(r)
+            continue
+        s = live[int(rng.integers(len(live)))]
+        if op == 1 and len(live) > 1:
+            live.remove(s)
+            ref.free_seq(s)
+            bm.free_seq(s)
+        elif op == 2:
+            swap = ref.swap_in if s in ref.swapped else ref.swap_out
+            native = bm.swap_in if s in ref.swapped else bm.swap_out
+            try:
+                exp = swap(s)
+            except MemoryError:
+                with pytest.raises(PagedKVError) as e:
+                    native(s)
+                assert e.value.status == 4                    # PKV_ENOMEM, state unchanged
+                continue
+            assert [tuple(p) for p in native(s).tolist()] == exp
+        elif s in ref.swapped:
+            # a swapped sequence cannot be forked or grown
+            with pytest.raises(PagedKVError) as e:
+                (bm.fork if op == 3 else bm.append_token)(s)
+            assert e.value.status == 6                        # PKV_ESWAPPED
+        elif op == 3:
+            r = ref.fork(s)
+            assert bm.fork(s) == r
+            live.append(r)
+        else:
+            try:
+                exp = ref.append_token(s)
+            except MemoryError:
+                with pytest.raises(PagedKVError):
+                    bm.append_token(s)
+                continue
+            assert bm.append_token(s) == exp
+        if step % 200 == 0:
+            _same_state(bm, ref, live)
+    _same_state(bm, ref, live)
+
+
+def test_swap_errors(BM):
+    from paged_kv_cache_404_b200 import PagedKVError
+    bm = BM(8, 16)
+    a = bm.alloc_seq(40)
+    with pytest.raises(PagedKVError):
+        bm.swap_out(a)                 # no host pool yet: ENOMEM
+    bm.set_host_pool(4)
+    with pytest.raises(PagedKVError):
+        bm.swap_in(a)                  # not swapped
+    pairs = bm.swap_out(a)
+    assert pairs.tolist() == [[0, 0], [1, 1], [2, 2]]
+    assert bm.block_table(a).tolist() == [0, 1, 2] and bm.seq_len(a) == 40
+    for call in (lambda: bm.slots(a, 0, 1), lambda: bm.tables([a], 4), lambda: bm.append_token(a)):
+        with pytest.raises(PagedKVError):
+            call()
+    with pytest.raises(PagedKVError):
+        bm.set_host_pool(8)            # host blocks in use
+    with pytest.raises(PagedKVError):
+        bm.swap_out(a)                 # already swapped
+    bm.free_seq(a)
+    assert bm.num_free_host() == 4 and bm.num_free() == 8
+    bm.set_host_pool(8)
+    assert bm.num_free_host() == 8
