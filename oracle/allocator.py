@@ -160,6 +160,34 @@ class RefBlockManager:
         self.swapped.discard(seq)
         return pairs
 
+    # -- shared prefixes ------------------------------------------------------
+    def prefix_groups(self, seqs):
+        """Sequences of a batch that start with the same physical block.
+
+        Returns (offsets, members, shared): group g has batch indices
+        members[offsets[g]:offsets[g+1]] (batch order) and shares its first
+        shared[g] table entries, each a full block in every member.  Only
+        groups of two or more are listed, in order of first appearance.
+        """
+        firsts = {}
+        for i, s in enumerate(seqs):
+            assert s not in self.swapped
+            if self.lens[s] >= self.block_size:
+                firsts.setdefault(self.tables[s][0], []).append(i)
+        offsets, members, shared = [0], [], []
+        for group in firsts.values():
+            if len(group) < 2:
+                continue
+            tabs = [self.tables[seqs[i]] for i in group]
+            full = min(self.lens[seqs[i]] // self.block_size for i in group)
+            k = 0
+            while k < full and all(t[k] == tabs[0][k] for t in tabs):
+                k += 1
+            members += group
+            shared.append(k)
+            offsets.append(len(members))
+        return offsets, members, shared
+
     # -- queries ------------------------------------------------------------
     def slot(self, seq, pos):
         t = self.tables[seq]

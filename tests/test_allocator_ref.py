@@ -240,3 +240,37 @@ def test_random_trace_with_swaps_invariants():
             host_used = sum(len(bm.tables[s]) for s in bm.swapped)
             assert host_used + len(bm.host_free) == 150
     _check_invariants(bm)
+
+
+# -- shared-prefix groups -----------------------------------------------------------
+
+def test_prefix_groups_of_parallel_samples():
+    """Parallel sampling shares the prompt's blocks (glossary entry, sharing
+    section): the three samples form one group over the prompt's full blocks;
+    the partly filled block does not count, and neither does a lone sequence."""
+    bm = RefBlockManager(32, 16)
+    lone = bm.alloc_seq(50)                       # blocks 0..3
+    p = bm.alloc_seq(40)                          # blocks 4, 5, 6 (6 holds 8 tokens)
+    kids = [bm.fork(p), bm.fork(p)]
+    short = bm.alloc_seq(9)                       # block 7: no full block
+    assert bm.prefix_groups([lone, p] + kids + [short]) == ([0, 3], [1, 2, 3], [2])
+    bm.append_token(kids[0])                      # copy-on-write of block 6
+    for _ in range(30):
+        bm.append_token(p)                        # p fills block 6 and takes another
+    assert bm.prefix_groups([kids[1], lone, p, kids[0]]) == ([0, 3], [0, 2, 3], [2])
+    # a second family after the first, members in batch order
+    q = bm.alloc_seq(33)
+    qk = bm.fork(q)
+    assert bm.prefix_groups([q, p, qk, kids[0]]) == ([0, 2, 4], [0, 2, 1, 3], [2, 2])
+
+
+def test_prefix_groups_stop_at_first_different_block():
+    bm = RefBlockManager(64, 16)
+    a = bm.alloc_seq(64)                          # 4 full blocks
+    b = bm.fork(a)
+    c = bm.fork(a)
+    # give b a different third block by hand (as a later copy-on-write would)
+    bm.ref[bm.tables[b][2]] -= 1
+    bm.tables[b][2] = bm._pop()
+    assert bm.prefix_groups([a, b, c]) == ([0, 3], [0, 1, 2], [2])
+    assert bm.prefix_groups([a, c]) == ([0, 2], [0, 1], [4])
