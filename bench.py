@@ -176,12 +176,13 @@ class ClockSampler:
 class Step:
     """Device-resident inputs of one decode step and the calls that run it."""
 
-    def __init__(self, w: W.Workload, device, partition=0):
+    def __init__(self, w: W.Workload, device, partition=0, prefix_groups=True):
         import paged_kv_cache_404_b200 as pkv
         self.pkv = pkv
         self.w = w
         self.device = device
         self.partition = partition
+        self.groups = None
         if w.lens == "shared":
             self._setup_shared()
         else:
@@ -191,14 +192,23 @@ class Step:
         self.g_tables = torch.from_numpy(self.tables).to(device)
         self.g_lens = torch.from_numpy(self.lens).to(device)
         self.g_pairs = torch.from_numpy(self.pairs).to(device) if len(self.pairs) else None
-        self.ws = pkv.decode_workspace(self.S, w.num_heads, w.head_dim, self.max_len, partition, device=device)
+        if self.groups is not None and prefix_groups:
+            # shared-prefix decode: each prompt's blocks are read once for its samples
+            offs, mem, sh = self.groups
+            self.g_offs = torch.from_numpy(offs).to(device)
+            self.g_mem = torch.from_numpy(mem).to(device)
+            self.g_sh = torch.from_numpy(sh).to(device)
+        else:
+            self.groups = None
+        self.ws = pkv.decode_workspace(self.S, w.num_heads, w.head_dim, self.max_len, partition, device=device,
+                                       shared=self.groups is not None)
         self.out = torch.empty_like(self.q)
         self.err = torch.zeros(1, dtype=torch.int32, device=device)
         elem = 1 if w.cache_dtype == "fp8" else 2
         self.kv_bytes = int(self.lens.astype(np.int64).sum()) * w.num_kv_heads * w.head_dim * 2 * elem
         self.seq_tokens = int(self.lens.astype(np.int64).sum())
         # write + plan + decode (+ merge when a split is possible) (+ copy-on-write copy)
-        merge = (partition or 256) < self.max_len
+        merge = (partition or 256) < self.max_len or self.groups is not None
         self.launches = 3 + int(merge) + int(self.g_pairs is not None)
 
     def _setup_flat(self):
@@ -245,6 +255,7 @@ class Step:
             cur += len(act)
         self.slots, self.pairs = bm.append_tokens(ids)
         self.tables, self.lens = bm.tables(ids, max(-(-int(bm.seq_len(s)) // 16) for s in ids), pad=-1)
+        self.groups = bm.prefix_groups(ids)
         self.k_pool, self.v_pool, self.k_scale, self.v_scale = kp, vp, 1.0, 1.0
         self.q = W.queries(w, S, dev)
         self.k_new, self.v_new = W.new_tokens(w, S, dev)
@@ -258,6 +269,12 @@ class Step:
                                 self.v_scale, err_count=self.err)
 
     def decode(self):
+        if self.groups is not None:
+            self.pkv.paged_attention_decode_shared(self.out, self.q, self.k_pool, self.v_pool, self.g_tables,
+                                                   self.g_lens, self.w.scale, self.max_len, self.ws, self.g_offs,
+                                                   self.g_mem, self.g_sh, self.k_scale, self.v_scale,
+                                                   partition_tokens=self.partition, err_count=self.err)
+            return
         self.pkv.paged_attention_decode(self.out, self.q, self.k_pool, self.v_pool, self.g_tables, self.g_lens,
                                         self.w.scale, self.max_len, self.ws, self.k_scale, self.v_scale,
                                         partition_tokens=self.partition, err_count=self.err)
@@ -312,6 +329,8 @@ def time_e2e(step: Step, steps: int, warmup: int, world: int):
     up = torch.cuda.Stream(device=step.device)
     down = torch.cuda.Stream(device=step.device)
     names = ["q", "k_new", "v_new", "g_slots", "g_tables", "g_lens"] + (["g_pairs"] if step.g_pairs is not None else [])
+    if step.groups is not None:
+        names += ["g_offs", "g_mem", "g_sh"]
     host = {n: getattr(step, n).cpu().pin_memory() for n in names}
     dev = [{n: getattr(step, n) for n in names}, {n: torch.empty_like(getattr(step, n)) for n in names}]
     outs = [step.out, torch.empty_like(step.out)]
@@ -561,6 +580,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--swap", action="store_true", help="measure block swap to a host pool instead")
+    ap.add_argument("--no-prefix-groups", action="store_true",
+                    help="shared_prefix: plain decode (each sample reads the prompt's blocks itself)")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
 
@@ -588,7 +609,7 @@ def main(argv=None):
         pkv_build.build()
 
     w = rank_workload(w0, rank)
-    step = Step(w, device, partition=args.partition)
+    step = Step(w, device, partition=args.partition, prefix_groups=not args.no_prefix_groups)
     torch.cuda.synchronize()
 
     with ClockSampler(device) as clk:
@@ -630,7 +651,8 @@ def main(argv=None):
                        "seq_len": step.max_len, "parallelism": "replicas: sequences sharded by rank, no collective",
                        "l2": "inputs larger than L2 (pools %.1f GiB per GPU vs 126 MB L2)" % (
                            2 * step.k_pool.numel() * step.k_pool.element_size() / 2**30),
-                       "partition_tokens": args.partition or "auto"},
+                       "partition_tokens": args.partition or "auto",
+                       "prefix_groups": step.groups is not None},
             "seq_tokens_per_s": round(step.seq_tokens * world * args.steps / (max_ms / 1e3), 1),
             "us_per_step_per_layer": round(1e3 * ms_per_step, 2),
             "us_decode": round(1e3 * dec_ms, 2), "us_write": round(1e3 * statistics.mean(write_ms), 2),

@@ -208,6 +208,48 @@ int pkv_paged_attention_decode_noalloc(void* out, const void* q, int q_dtype,
                                        int partition_tokens, int32_t* err_count, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Shared-prefix decode: the same attention as pkv_paged_attention_decode, but
+ * sequences that begin with the same physical blocks read those blocks once
+ * for all of them.  Source: block tables let several sequences point at the
+ * same physical blocks -- parallel samples, beams, requests that start with the
+ * same system prompt reuse one copy of the shared prefix (glossary entry
+ * "PagedAttention", section "Compartir bloques entre secuencias"; full-block
+ * hashing extends this across requests, same section).
+ *
+ * Extra arguments (device pointers, int32):
+ *   group_offsets        [num_groups + 1]  group g is group_seqs[offsets[g] .. offsets[g+1])
+ *   group_seqs           [num_group_seqs]  batch indices (0 .. num_seqs-1) of its members
+ *   group_shared_blocks  [num_groups]      leading blocks the members are said to share
+ * These are hints (pkv_bm_prefix_groups computes them): the kernels keep a
+ * member only if it is in range and in no earlier-claimed group, and cut a
+ * group's shared blocks to those every kept member holds in full (16 tokens
+ * within its context) with the same physical id in every member's table.  A
+ * wrong hint costs time, never correctness.  Up to 1024 members per group are
+ * considered.  The result equals pkv_paged_attention_decode's up to rounding
+ * (partitions are cut differently: each sequence's shared and own blocks
+ * separately).  Grouping applies to bf16 caches with head_dim 128 and at most 8
+ * query heads per KV head (a member's heads and its group-mates' fill 16 score
+ * columns); other configurations ignore the hints and run the plain decode.
+ *
+ * workspace: pkv_decode_workspace_bytes_shared(...) bytes (a little more than
+ * the plain decode's).  num_groups == 0 runs the plain decode in that layout.
+ * ---------------------------------------------------------------------- */
+size_t pkv_decode_workspace_bytes_shared(int num_seqs, int num_heads, int head_dim, int max_context_len,
+                                         int partition_tokens);
+
+int pkv_paged_attention_decode_shared(void* out, const void* q, int q_dtype,
+                                      const void* k_pool, const void* v_pool, int cache_dtype,
+                                      const int32_t* block_tables, int max_blocks_per_seq,
+                                      const int32_t* context_lens, int num_seqs, int max_context_len,
+                                      int num_blocks, int block_size, int num_heads, int num_kv_heads,
+                                      int head_dim, float scale, float k_scale, float v_scale,
+                                      int partition_tokens,
+                                      const int32_t* group_offsets, const int32_t* group_seqs,
+                                      int num_group_seqs, const int32_t* group_shared_blocks, int num_groups,
+                                      void* workspace, size_t workspace_bytes,
+                                      int32_t* err_count, void* stream);
+
+/* ------------------------------------------------------------------------
  * Copy-on-write block copy: for every pair (src, dst) copy the whole physical
  * block src over block dst, in both pools.
  * Source: before a sequence writes into a block that other sequences still
@@ -295,6 +337,19 @@ int pkv_bm_tables(const pkv_block_manager* bm, const int32_t* seqs, int n, int32
                   int max_blocks, int32_t pad, int32_t* lens);
 /* Current free list, front first (n_out entries). */
 int pkv_bm_free_list(const pkv_block_manager* bm, int32_t* out, int cap, int* n_out);
+
+/* Shared-prefix hints for pkv_paged_attention_decode_shared, for the batch
+ * seqs[0..n) (in that order: members are given as batch indices 0..n-1).
+ * Resident sequences holding at least one full block are grouped by the
+ * physical id of their first block, in order of first appearance; groups of at
+ * least two members are emitted, members in batch order, and a group's shared
+ * count is the number of leading table entries equal in all its members and
+ * full (16 tokens) in every member.  Outputs: group_offsets [n + 1],
+ * group_seqs [n], group_shared_blocks [n] (capacity n each),
+ * *num_groups_out groups, group_offsets[*num_groups_out] = members written.
+ * Unknown sequences return PKV_ENOENT, swapped ones PKV_ESWAPPED. */
+int pkv_bm_prefix_groups(const pkv_block_manager* bm, const int32_t* seqs, int n, int32_t* group_offsets,
+                         int32_t* group_seqs, int32_t* group_shared_blocks, int* num_groups_out);
 
 /* Host pool for swapping (fine-grained eviction, see pkv_swap_blocks): give the
  * manager num_host_blocks host blocks (ids 0..n-1, free list in id order).

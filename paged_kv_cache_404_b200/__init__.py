@@ -12,7 +12,9 @@ from .ops import (  # noqa: F401
     copy_blocks,
     decode_workspace,
     decode_workspace_bytes,
+    decode_workspace_bytes_shared,
     paged_attention_decode,
+    paged_attention_decode_shared,
     paged_attention_decode_noalloc,
     paged_kv_write,
     swap_blocks,

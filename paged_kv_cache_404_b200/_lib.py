@@ -23,6 +23,9 @@ SIGNATURES = {
                                         _f, _f, _f, _i, _p, _z, _p, _p]),
     "pkv_paged_attention_decode_noalloc": (_i, [_p, _p, _i, _p, _p, _i, _p, _i, _p, _i, _i, _i, _i, _i, _i, _i,
                                                 _f, _f, _f, _i, _p, _p]),
+    "pkv_decode_workspace_bytes_shared": (_z, [_i, _i, _i, _i, _i]),
+    "pkv_paged_attention_decode_shared": (_i, [_p, _p, _i, _p, _p, _i, _p, _i, _p, _i, _i, _i, _i, _i, _i, _i,
+                                               _f, _f, _f, _i, _p, _p, _i, _p, _i, _p, _z, _p, _p]),
     "pkv_copy_blocks": (_i, [_p, _p, _z, _p, _i, _i, _p, _p]),
     "pkv_swap_blocks": (_i, [_p, _p, _i, _p, _p, _i, _z, _p, _i, _p, _p]),
     "pkv_bm_create": (_i, [_i, _i, _p, _i, C.POINTER(_p)]),
@@ -38,6 +41,7 @@ SIGNATURES = {
     "pkv_bm_slots": (_i, [_p, C.c_int32, _i, _i, _p]),
     "pkv_bm_tables": (_i, [_p, _p, _i, _p, _i, C.c_int32, _p]),
     "pkv_bm_free_list": (_i, [_p, _p, _i, _p]),
+    "pkv_bm_prefix_groups": (_i, [_p, _p, _i, _p, _p, _p, _p]),
     "pkv_bm_set_host_pool": (_i, [_p, _i]),
     "pkv_bm_swap_out": (_i, [_p, C.c_int32, _p, _i, _p]),
     "pkv_bm_swap_in": (_i, [_p, C.c_int32, _p, _i, _p]),

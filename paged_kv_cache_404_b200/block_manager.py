@@ -107,6 +107,19 @@ class BlockManager:
         L.check("pkv_bm_free_list", self._lib.pkv_bm_free_list(self._h, out.ctypes.data, out.size, C.byref(n)))
         return out[:n.value].copy()
 
+    def prefix_groups(self, seqs):
+        """Shared-prefix hints of a batch: (offsets int32 [g+1], members int32 [m], shared int32 [g])."""
+        seqs = np.ascontiguousarray(seqs, dtype=np.int32)
+        n = seqs.size
+        offs = np.zeros(n + 1, dtype=np.int32)
+        mem = np.zeros(max(n, 1), dtype=np.int32)
+        sh = np.zeros(max(n, 1), dtype=np.int32)
+        ng = C.c_int()
+        L.check("pkv_bm_prefix_groups", self._lib.pkv_bm_prefix_groups(
+            self._h, seqs.ctypes.data, n, offs.ctypes.data, mem.ctypes.data, sh.ctypes.data, C.byref(ng)))
+        g = ng.value
+        return offs[:g + 1].copy(), mem[:offs[g]].copy(), sh[:g].copy()
+
     # --- host pool and swap (fine-grained eviction) -------------------------
 
     def set_host_pool(self, num_host_blocks):

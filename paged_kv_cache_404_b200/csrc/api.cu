@@ -18,7 +18,8 @@ cudaError_t launch_decode_plan(const DecodeParams& p, int fixed_partition, int m
 cudaError_t launch_decode_tc(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeParams& p, bool fp8,
                              int num_sms, cudaStream_t stream);
 cudaError_t launch_decode_f32(const DecodeParams& p, int num_sms, cudaStream_t stream);
-int decode_tc_warps(bool fp8, int head_dim);
+int decode_tc_warps(bool fp8, int head_dim, bool grouped);
+bool decode_tc_groupable(bool fp8, int head_dim, int group);
 cudaError_t launch_decode_merge(const DecodeParams& p, int out_dtype, cudaStream_t stream);
 }  // namespace pkv
 
@@ -87,6 +88,22 @@ int max_parts_of(int max_context_len, int partition_tokens) {
     return n > 0 ? n : 1;
 }
 
+// Optional shared-prefix hints of pkv_paged_attention_decode_shared.
+struct PrefixGroups {
+    const int32_t* offsets = nullptr;
+    const int32_t* seqs = nullptr;
+    const int32_t* shared_blocks = nullptr;
+    int num_seqs = 0;
+    int num_groups = 0;
+    bool layout = false;  // workspace laid out by ws_layout_shared
+};
+
+int decode_impl(void* out, const void* q, int q_dtype, const void* k_pool, const void* v_pool, int cache_dtype,
+                const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
+                int max_context_len, int num_blocks, int block_size, int num_heads, int num_kv_heads, int head_dim,
+                float scale, float k_scale, float v_scale, int partition_tokens, const PrefixGroups& pg,
+                void* workspace, size_t workspace_bytes, int32_t* err_count, void* stream);
+
 }  // namespace
 
 extern "C" {
@@ -145,6 +162,55 @@ int pkv_paged_attention_decode(void* out, const void* q, int q_dtype, const void
                                int block_size, int num_heads, int num_kv_heads, int head_dim, float scale,
                                float k_scale, float v_scale, int partition_tokens, void* workspace,
                                size_t workspace_bytes, int32_t* err_count, void* stream) {
+    return decode_impl(out, q, q_dtype, k_pool, v_pool, cache_dtype, block_tables, max_blocks_per_seq, context_lens,
+                       num_seqs, max_context_len, num_blocks, block_size, num_heads, num_kv_heads, head_dim, scale,
+                       k_scale, v_scale, partition_tokens, PrefixGroups(), workspace, workspace_bytes, err_count,
+                       stream);
+}
+
+size_t pkv_decode_workspace_bytes_shared(int num_seqs, int num_heads, int head_dim, int max_context_len,
+                                         int partition_tokens) {
+    if (num_seqs < 0 || num_heads <= 0 || head_dim <= 0 || max_context_len < 0 || partition_tokens < 0 ||
+        partition_tokens % kBlockSize != 0)
+        return 0;
+    return ws_layout_shared(num_seqs, num_heads, head_dim, max_parts_of(max_context_len, partition_tokens)).total;
+}
+
+int pkv_paged_attention_decode_shared(void* out, const void* q, int q_dtype, const void* k_pool, const void* v_pool,
+                                      int cache_dtype, const int32_t* block_tables, int max_blocks_per_seq,
+                                      const int32_t* context_lens, int num_seqs, int max_context_len,
+                                      int num_blocks, int block_size, int num_heads, int num_kv_heads, int head_dim,
+                                      float scale, float k_scale, float v_scale, int partition_tokens,
+                                      const int32_t* group_offsets, const int32_t* group_seqs, int num_group_seqs,
+                                      const int32_t* group_shared_blocks, int num_groups, void* workspace,
+                                      size_t workspace_bytes, int32_t* err_count, void* stream) {
+    if (num_groups < 0 || num_group_seqs < 0) return PKV_EINVAL;
+    PrefixGroups pg;
+    pg.layout = true;
+    if (num_groups > 0 && num_group_seqs > 0) {
+        if (!group_offsets || !group_seqs || !group_shared_blocks) return PKV_EINVAL;
+        if (!aligned(group_offsets, 4) || !aligned(group_seqs, 4) || !aligned(group_shared_blocks, 4))
+            return PKV_EINVAL;
+        pg.offsets = group_offsets;
+        pg.seqs = group_seqs;
+        pg.shared_blocks = group_shared_blocks;
+        pg.num_seqs = num_group_seqs;
+        pg.num_groups = num_groups;
+    }
+    return decode_impl(out, q, q_dtype, k_pool, v_pool, cache_dtype, block_tables, max_blocks_per_seq, context_lens,
+                       num_seqs, max_context_len, num_blocks, block_size, num_heads, num_kv_heads, head_dim, scale,
+                       k_scale, v_scale, partition_tokens, pg, workspace, workspace_bytes, err_count, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+int decode_impl(void* out, const void* q, int q_dtype, const void* k_pool, const void* v_pool, int cache_dtype,
+                const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
+                int max_context_len, int num_blocks, int block_size, int num_heads, int num_kv_heads, int head_dim,
+                float scale, float k_scale, float v_scale, int partition_tokens, const PrefixGroups& pg,
+                void* workspace, size_t workspace_bytes, int32_t* err_count, void* stream) {
     if (num_seqs < 0 || max_blocks_per_seq <= 0 || max_context_len < 0 || num_blocks <= 0 || block_size <= 0 ||
         num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || partition_tokens < 0)
         return PKV_EINVAL;
@@ -167,8 +233,11 @@ int pkv_paged_attention_decode(void* out, const void* q, int q_dtype, const void
         !aligned(err_count, 4))
         return PKV_EINVAL;
     const int max_parts = max_parts_of(max_context_len, partition_tokens);
-    const WsLayout ws = ws_layout(num_seqs, num_heads, head_dim, max_parts);
+    const WsLayout ws = pg.layout ? ws_layout_shared(num_seqs, num_heads, head_dim, max_parts)
+                                  : ws_layout(num_seqs, num_heads, head_dim, max_parts);
     if (workspace_bytes < ws.total) return PKV_EINVAL;
+    // groups only where a grouped kernel exists and two members fit in 16 columns
+    const bool grouped = pg.num_groups > 0 && !f32 && decode_tc_groupable(fp8, head_dim, group);
 
     const int num_sms = sm_count();
     if (num_sms <= 0) return PKV_ECUDA;
@@ -198,15 +267,25 @@ int pkv_paged_attention_decode(void* out, const void* q, int q_dtype, const void
     p.items = reinterpret_cast<int4*>(w + ws.items);
     p.part_ml = reinterpret_cast<float2*>(w + ws.part_ml);
     p.part_o = reinterpret_cast<float*>(w + ws.part_o);
-    p.max_parts = max_parts;
+    p.max_parts = ws.max_parts;
     p.err = err_count;
+    p.group_offsets = grouped ? pg.offsets : nullptr;
+    p.group_seqs = grouped ? pg.seqs : nullptr;
+    p.group_shared_blocks = grouped ? pg.shared_blocks : nullptr;
+    p.num_groups = grouped ? pg.num_groups : 0;
+    p.num_group_seqs = grouped ? pg.num_seqs : 0;
+    p.group_cap = 16 / group;
+    p.seq_sub = pg.layout ? reinterpret_cast<int*>(w + ws.seq_sub) : nullptr;
+    p.seq_k = pg.layout ? reinterpret_cast<int*>(w + ws.seq_k) : nullptr;
+    p.sub_info = pg.layout ? reinterpret_cast<int4*>(w + ws.sub_info) : nullptr;
+    p.sub_members = pg.layout ? reinterpret_cast<int*>(w + ws.sub_members) : nullptr;
 
     // Partition candidates: min_partition << c, up to the first that covers max_context_len.
     const int min_p = min_partition_of(partition_tokens);
     int ncand = 1;
     if (partition_tokens == 0)
         while (ncand < kMaxCandidates && ((long long)min_p << (ncand - 1)) < max_context_len) ++ncand;
-    const int warps_per_sm = f32 ? 32 : decode_tc_warps(fp8, head_dim);
+    const int warps_per_sm = f32 ? 32 : decode_tc_warps(fp8, head_dim, grouped);
     const int target_units = num_sms * warps_per_sm * kUnitsPerWorker;
     const int out_dtype = f32 ? 0 : 1;
 
@@ -224,13 +303,18 @@ int pkv_paged_attention_decode(void* out, const void* q, int q_dtype, const void
     }
     if (e != cudaSuccess) return PKV_ECUDA;
     // a split (and so a merge) is possible only if the smallest partition is
-    // shorter than the longest context
-    if (min_p < max_context_len) {
+    // shorter than the longest context, or if a sequence's shared and own
+    // blocks are cut apart
+    if (grouped || min_p < max_context_len) {
         e = launch_decode_merge(p, out_dtype, st);
         if (e != cudaSuccess) return PKV_ECUDA;
     }
     return PKV_OK;
 }
+
+}  // namespace
+
+extern "C" {
 
 int pkv_copy_blocks(void* k_pool, void* v_pool, size_t block_bytes, const int64_t* src_dst_pairs, int num_pairs,
                     int num_blocks, int32_t* err_count, void* stream) {

@@ -25,6 +25,7 @@
 #include <cstring>
 #include <deque>
 #include <new>
+#include <unordered_map>
 #include <vector>
 
 #include "pagedkv.h"
@@ -239,6 +240,50 @@ int pkv_bm_free_list(const pkv_block_manager* bm, int32_t* out, int cap, int* n_
     if ((int)bm->free_list.size() > cap) return PKV_EINVAL;
     int i = 0;
     for (int32_t b : bm->free_list) out[i++] = b;
+    return PKV_OK;
+}
+
+int pkv_bm_prefix_groups(const pkv_block_manager* bm, const int32_t* seqs, int n, int32_t* group_offsets,
+                         int32_t* group_seqs, int32_t* group_shared_blocks, int* num_groups_out) {
+    if (bm == nullptr || n < 0 || num_groups_out == nullptr ||
+        (n > 0 && (seqs == nullptr || group_offsets == nullptr || group_seqs == nullptr ||
+                   group_shared_blocks == nullptr)))
+        return PKV_EINVAL;
+    for (int i = 0; i < n; ++i)
+        if (int st = bm->resident(seqs[i])) return st;
+    // batch indices grouped by the physical id of their first block
+    std::unordered_map<int32_t, int> by_first;
+    std::vector<std::vector<int>> groups;
+    for (int i = 0; i < n; ++i) {
+        if (bm->lens[seqs[i]] < bm->block_size) continue;  // no full block
+        const int32_t b0 = bm->tables[seqs[i]][0];
+        auto it = by_first.find(b0);
+        if (it == by_first.end()) {
+            by_first.emplace(b0, (int)groups.size());
+            groups.push_back({i});
+        } else {
+            groups[it->second].push_back(i);
+        }
+    }
+    int ng = 0, pos = 0;
+    if (n > 0) group_offsets[0] = 0;
+    for (const std::vector<int>& g : groups) {
+        if (g.size() < 2) continue;
+        const std::vector<int32_t>& t0 = bm->tables[seqs[g[0]]];
+        int k = bm->lens[seqs[g[0]]] / bm->block_size;
+        for (int m : g) {
+            const std::vector<int32_t>& tm = bm->tables[seqs[m]];
+            const int full = bm->lens[seqs[m]] / bm->block_size;
+            if (full < k) k = full;
+            int j = 0;
+            while (j < k && tm[j] == t0[j]) ++j;
+            k = j;
+        }
+        for (int m : g) group_seqs[pos++] = m;
+        group_shared_blocks[ng++] = k;
+        group_offsets[ng] = pos;
+    }
+    *num_groups_out = ng;
     return PKV_OK;
 }
 

@@ -64,12 +64,120 @@ __device__ __forceinline__ int for_each_piece(int B, int nb, int mb, bool geomet
     return count + 1;
 }
 
+// Shared-prefix groups.  Sequences that start with the same physical blocks
+// (parallel samples of one prompt, requests with a common system prompt: the
+// glossary entry "PagedAttention", "Compartir bloques entre secuencias") can
+// read those blocks once for all of them.  The caller's hints are checked
+// here, never trusted: a member is kept only if it is in range and not already
+// in another group; the shared count is cut to the leading blocks that every
+// kept member holds in full and that are the same physical block in all their
+// tables.  A kept group is split into subgroups of at most group_cap members
+// (balanced sizes).  A wrong hint costs speed, not correctness.
+constexpr int kMaxGroupChunks = 32;  // members per group considered: 32 * 32
+
+__device__ void build_groups(const DecodeParams& p, int* n_subs, int* n_members) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int s = tid; s < p.num_seqs; s += kPlanThreads) {
+        p.seq_sub[s] = -1;
+        p.seq_k[s] = 0;
+    }
+    __syncthreads();
+    for (int gi = warp; gi < p.num_groups; gi += kPlanThreads / 32) {
+        const int beg = p.group_offsets[gi];
+        if (beg < 0 || beg >= p.num_group_seqs) continue;
+        const int end = min(min(p.group_offsets[gi + 1], p.num_group_seqs), beg + 32 * kMaxGroupChunks);
+        int k = min(p.group_shared_blocks[gi], p.max_blocks_per_seq);
+        if (end <= beg + 1 || k <= 0) continue;
+        const int nchunks = (end - beg + 31) >> 5;
+
+        // claim the members (bit c of `mine`: member beg + 32c + lane is ours)
+        uint32_t mine = 0;
+        int count = 0, s0 = -1;
+        for (int c = 0; c < nchunks; ++c) {
+            const int i = beg + 32 * c + lane;
+            const int s = i < end ? p.group_seqs[i] : -1;
+            bool got = false;
+            if (s >= 0 && s < p.num_seqs && atomicCAS(&p.seq_sub[s], -1, -2) == -1) {
+                got = true;
+                k = min(k, clamped_len(p, s, false) / kBlockSize);
+            }
+            const unsigned b = __ballot_sync(0xffffffffu, got);
+            if (got) mine |= 1u << c;
+            if (s0 < 0 && b) s0 = __shfl_sync(0xffffffffu, s, __ffs(b) - 1);
+            count += __popc(b);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) k = min(k, __shfl_xor_sync(0xffffffffu, k, o));
+
+        // cut k at the first block where a member's table differs from s0's
+        if (count >= 2 && k > 0) {
+            const int32_t* ref = p.block_tables + (size_t)s0 * p.max_blocks_per_seq;
+            for (int j0 = 0; j0 < k; j0 += 32) {
+                const int j = j0 + lane;
+                const int r = j < k ? __ldg(ref + j) : 0;
+                bool diff = false;
+                for (int c = 0; c < nchunks; ++c) {
+                    const int i = beg + 32 * c + lane;
+                    const int sl = ((mine >> c) & 1u) ? p.group_seqs[i] : -1;
+                    unsigned b = __ballot_sync(0xffffffffu, sl >= 0);
+                    while (b) {
+                        const int src = __ffs(b) - 1;
+                        b &= b - 1;
+                        const int sm = __shfl_sync(0xffffffffu, sl, src);
+                        if (j < k && __ldg(p.block_tables + (size_t)sm * p.max_blocks_per_seq + j) != r) diff = true;
+                    }
+                }
+                const unsigned d = __ballot_sync(0xffffffffu, diff);
+                if (d) {
+                    k = j0 + __ffs(d) - 1;
+                    break;
+                }
+            }
+        }
+
+        const bool keep = count >= 2 && k > 0;
+        const int nsub = keep ? (count + p.group_cap - 1) / p.group_cap : 0;
+        int mbase = 0, sbase = 0;
+        if (keep && lane == 0) {
+            mbase = atomicAdd(n_members, count);
+            sbase = atomicAdd(n_subs, nsub);
+        }
+        mbase = __shfl_sync(0xffffffffu, mbase, 0);
+        sbase = __shfl_sync(0xffffffffu, sbase, 0);
+        if (keep)
+            for (int q = lane; q < nsub; q += 32) {
+                const int a = (int)(((long long)q * count) / nsub), b = (int)(((long long)(q + 1) * count) / nsub);
+                p.sub_info[sbase + q] = make_int4(mbase + a, b - a, k, 0);
+            }
+        // members in claim order; member of rank r goes to subgroup ((r+1)*nsub - 1) / count
+        int rank0 = 0;
+        for (int c = 0; c < nchunks; ++c) {
+            const bool own = (mine >> c) & 1u;
+            const unsigned b = __ballot_sync(0xffffffffu, own);
+            if (own) {
+                const int s = p.group_seqs[beg + 32 * c + lane];
+                if (keep) {
+                    const int r = rank0 + __popc(b & ((1u << lane) - 1u));
+                    p.sub_members[mbase + r] = s;
+                    p.seq_sub[s] = sbase + (int)(((long long)(r + 1) * nsub - 1) / count);
+                    p.seq_k[s] = k;
+                } else {
+                    p.seq_sub[s] = -1;  // release
+                }
+            }
+            rank0 += __popc(b);
+        }
+    }
+    __syncthreads();
+}
+
 __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams p, int fixed_partition, int min_partition,
                                                                    int num_candidates, int target_units,
                                                                    int zero_out_dtype) {
     __shared__ int hist[kMaxBuckets];
     __shared__ unsigned long long units_of[kMaxCandidates];
     __shared__ int chosen;
+    __shared__ int n_subs, n_members;
     const int tid = threadIdx.x;
     const bool geometric = fixed_partition == 0 && PKV_PLAN_GEOMETRIC;
     const int mb = min_partition / kBlockSize;
@@ -77,6 +185,15 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
     // The workspace and the output may still be in use by the previous kernel.
     pdl_wait();
     pdl_trigger();
+
+    // 0. shared-prefix subgroups: sequence s then owns blocks [seq_k[s], B) and
+    //    its subgroup computes blocks [0, seq_k[s]) once for all its members
+    if (tid == 0) n_subs = n_members = 0;
+    __syncthreads();
+    const bool grouped = p.num_groups > 0;
+    if (grouped) build_groups(p, &n_subs, &n_members);
+    const int num_subs = n_subs;
+    auto own_k = [&](int s) { return grouped ? p.seq_k[s] : 0; };
 
     // 1. largest partition: the largest candidate min_partition << c whose work
     //    list still has target_units units (one pass over the lengths for all c)
@@ -89,11 +206,19 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
 #pragma unroll
         for (int c = 0; c < kMaxCandidates; ++c) cnt[c] = 0;
         for (int s = tid; s < p.num_seqs; s += kPlanThreads) {
-            const int B = ceil_div(clamped_len(p, s, false), kBlockSize);
+            const int B = ceil_div(clamped_len(p, s, false), kBlockSize) - own_k(s);
 #pragma unroll
             for (int c = 0; c < kMaxCandidates; ++c)
                 if (c < num_candidates)
                     cnt[c] += (unsigned long long)for_each_piece(B, (min_partition << c) / kBlockSize, mb, geometric,
+                                                                 [](int, int) {});
+        }
+        for (int q = tid; q < num_subs; q += kPlanThreads) {
+            const int k = p.sub_info[q].z;
+#pragma unroll
+            for (int c = 0; c < kMaxCandidates; ++c)
+                if (c < num_candidates)
+                    cnt[c] += (unsigned long long)for_each_piece(k, (min_partition << c) / kBlockSize, mb, geometric,
                                                                  [](int, int) {});
         }
 #pragma unroll
@@ -125,8 +250,10 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
     __syncthreads();
     for (int s = tid; s < p.num_seqs; s += kPlanThreads) {
         const int L = clamped_len(p, s, true);
-        const int B = ceil_div(L, kBlockSize);
-        p.nparts[s] = for_each_piece(B, nb_top, mb, geometric,
+        const int k = own_k(s);
+        const int B = ceil_div(L, kBlockSize) - k;
+        p.nparts[s] = for_each_piece(k, nb_top, mb, geometric, [](int, int) {}) +
+                      for_each_piece(B, nb_top, mb, geometric,
                                      [&](int, int n) { atomicAdd(&hist[bucket_of(n, nb_top, nbuckets)], 1); });
         if (L == 0) {
             // an empty context produces a zero output row (nothing else writes it)
@@ -140,6 +267,9 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
             }
         }
     }
+    for (int q = tid; q < num_subs; q += kPlanThreads)
+        for_each_piece(p.sub_info[q].z, nb_top, mb, geometric,
+                       [&](int, int n) { atomicAdd(&hist[bucket_of(n, nb_top, nbuckets)], 1); });
     __syncthreads();
 
     // 3. exclusive scan, largest bucket first (serial over <= 1024 buckets by one warp)
@@ -163,17 +293,29 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
             p.hdr->partition = P;
             p.hdr->counter = 0;
             p.hdr->timeout = 0;
+            p.hdr->num_subs = num_subs;
+            p.hdr->num_members = n_members;
         }
     }
     __syncthreads();
 
-    // 4. scatter the items (order inside a bucket does not affect results)
+    // 4. scatter the items (order inside a bucket does not affect results);
+    //    a sequence's shared partitions come first, then its own
     for (int s = tid; s < p.num_seqs; s += kPlanThreads) {
-        const int B = ceil_div(clamped_len(p, s, false), kBlockSize);
-        int part = 0;
+        const int k = own_k(s);
+        const int B = ceil_div(clamped_len(p, s, false), kBlockSize) - k;
+        int part = for_each_piece(k, nb_top, mb, geometric, [](int, int) {});
         for_each_piece(B, nb_top, mb, geometric, [&](int first, int n) {
             const int pos = atomicAdd(&hist[bucket_of(n, nb_top, nbuckets)], 1);
-            p.items[pos] = make_int4(s, part++, first, n);
+            p.items[pos] = make_int4(s, part++, k + first, n);
+        });
+    }
+    // subgroup items carry -(subgroup + 1) in place of the sequence
+    for (int q = tid; q < num_subs; q += kPlanThreads) {
+        int part = 0;
+        for_each_piece(p.sub_info[q].z, nb_top, mb, geometric, [&](int first, int n) {
+            const int pos = atomicAdd(&hist[bucket_of(n, nb_top, nbuckets)], 1);
+            p.items[pos] = make_int4(-(q + 1), part++, first, n);
         });
     }
 }

@@ -59,7 +59,7 @@ struct TileCfg {
     static_assert(kRowBytes % 128 == 0, "rows must be whole 128-byte swizzle atoms");
 };
 
-template <bool FP8, int D, int NT, int WARPS, int STAGES, int BPS>
+template <bool FP8, int D, int NT, int WARPS, int STAGES, int BPS, bool GROUPED>
 __global__ void __launch_bounds__(WARPS * 32, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const DecodeParams p) {
@@ -131,7 +131,22 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
         if (u >= num_units) break;
         const int4 item = p.items[u / p.num_kv_heads];
         const int kvh = u - (u / p.num_kv_heads) * p.num_kv_heads;
-        const int s = item.x, part = item.y;
+        int s = item.x;
+        const int part = item.y;
+        // A subgroup item (shared-prefix decode) serves M sequences that hold the
+        // same physical blocks: one read of each K/V tile, M*G score columns
+        // (member i's query heads are columns i*G .. i*G+G-1).
+        int M = 1, mbase = 0;
+        if constexpr (GROUPED) {
+            if (s < 0) {
+                const int4 si = p.sub_info[-s - 1];
+                mbase = si.x;
+                M = si.y;
+                s = p.sub_members[mbase];
+            }
+        }
+        const int ncols = M * G;
+        const int nt_act = GROUPED ? (ncols + 7) >> 3 : NT;  // n-tiles holding a column
         const int L = clamped_len(p, s, false);
         const int blk0 = item.z;
         const int t0 = blk0 * kBlockSize;
@@ -155,10 +170,17 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
         const int hq0 = kvh * G;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            const int hh = nt * 8 + g;
-            const bool hv = hh < G;
+            int hh = nt * 8 + g, sq = s;
+            bool hv = hh < G;
+            if constexpr (GROUPED) {
+                const int c = hh;
+                hv = c < ncols;
+                const int mi = hv ? c / G : 0;
+                hh = c - mi * G;
+                if (mi > 0) sq = p.sub_members[mbase + mi];
+            }
             const __nv_bfloat16* qrow =
-                static_cast<const __nv_bfloat16*>(p.q) + ((size_t)s * p.num_heads + hq0 + (hv ? hh : 0)) * D;
+                static_cast<const __nv_bfloat16*>(p.q) + ((size_t)sq * p.num_heads + hq0 + (hv ? hh : 0)) * D;
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) {
                 if constexpr (!FP8) {
@@ -282,7 +304,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
                     ldmatrix_x4(kt + (ks >> 2) * (kBlockSize * 128) + koff[ks & 3], a0, a1, a2, a3);
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt)
-                        mma_bf16((ks & 1) ? sc2[nt] : sc[nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
+                        if (nt < nt_act)
+                            mma_bf16((ks & 1) ? sc2[nt] : sc[nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
                 }
             } else {
 #if PKV_FP8_QK_E4M3
@@ -311,6 +334,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
                     ldmatrix_x4(kt + koff[kp], r0, r1, r2, r3);
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
+                        if (nt >= nt_act) continue;
                         mma_f16(sc[nt], e4m3x2_to_f16x2(r0), e4m3x2_to_f16x2(r1), e4m3x2_to_f16x2(r0 >> 16),
                                 e4m3x2_to_f16x2(r1 >> 16), qf[nt][2 * kp][0], qf[nt][2 * kp][1]);
                         mma_f16(sc2[nt], e4m3x2_to_f16x2(r2), e4m3x2_to_f16x2(r3), e4m3x2_to_f16x2(r2 >> 16),
@@ -333,7 +357,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
                     uint32_t a0, a1, a2, a3;
                     ldmatrix_x4_trans(vt + (i >> 2) * (kBlockSize * 128) + voff[i & 3], a0, a1, a2, a3);
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) mma_bf16(oacc[nt][i], a0, a1, a2, a3, pb0[nt], pb1[nt]);
+                    for (int nt = 0; nt < NT; ++nt)
+                        if (nt < nt_act) mma_bf16(oacc[nt][i], a0, a1, a2, a3, pb0[nt], pb1[nt]);
                 }
             } else {
 #pragma unroll
@@ -349,6 +374,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
                     const uint32_t x23lo = __byte_perm(w2, w3, 0x5140), x23hi = __byte_perm(w2, w3, 0x7362);
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
+                        if (nt >= nt_act) continue;
                         // m-tile 2*q4: rows g -> column 32q4+4g, g+8 -> 32q4+4g+1
                         mma_f16(oacc[nt][2 * q4], e4m3x2_to_f16x2(x01lo), e4m3x2_to_f16x2(x01lo >> 16),
                                 e4m3x2_to_f16x2(x23lo), e4m3x2_to_f16x2(x23lo >> 16), pb0[nt], pb1[nt]);
@@ -407,6 +433,11 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
                 uint32_t pb0[BPS][NT], pb1[BPS][NT];
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
+                    if (nt >= nt_act) {
+#pragma unroll
+                        for (int b = 0; b < BPS; ++b) pb0[b][nt] = pb1[b][nt] = 0u;
+                        continue;
+                    }
                     float x[BPS][4];
                     float b0 = -INFINITY, b1 = -INFINITY;
 #pragma unroll
@@ -517,20 +548,34 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
+                if (nt >= nt_act) continue;
 #pragma unroll
                 for (int o = 4; o < 32; o <<= 1) l[nt][c] += __shfl_xor_sync(0xffffffffu, l[nt][c], o);
             }
-        const bool split = p.nparts[s] > 1;
+        bool split = p.nparts[s] > 1;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-                const int hh = nt * 8 + 2 * t + c;
-                if (hh >= G) continue;
+                int hh = nt * 8 + 2 * t + c, so = s;
+                if constexpr (GROUPED) {
+                    const int col = hh;
+                    if (col >= ncols) continue;
+                    const int mi = col / G;
+                    hh = col - mi * G;
+                    if (mi > 0) {
+                        so = p.sub_members[mbase + mi];
+                        split = p.nparts[so] > 1;
+                    } else {
+                        split = p.nparts[s] > 1;
+                    }
+                } else {
+                    if (hh >= G) continue;
+                }
                 const int hq = hq0 + hh;
                 const float inv = l[nt][c] > 0.f ? p.out_scale / l[nt][c] : 0.f;
                 if (!split) {
-                    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + ((size_t)s * p.num_heads + hq) * D;
+                    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + ((size_t)so * p.num_heads + hq) * D;
                     if constexpr (!FP8) {
 #pragma unroll
                         for (int i = 0; i < KS; ++i) {
@@ -547,7 +592,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
                         }
                     }
                 } else {
-                    const size_t slot = ((size_t)s * p.num_heads + hq) * p.max_parts + part;
+                    const size_t slot = ((size_t)so * p.num_heads + hq) * p.max_parts + part;
                     float* o = p.part_o + slot * D;
                     if constexpr (!FP8) {
 #pragma unroll
@@ -585,12 +630,12 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
 #endif
 }
 
-template <bool FP8, int D, int NT, int WARPS, int STAGES, int BPS>
+template <bool FP8, int D, int NT, int WARPS, int STAGES, int BPS, bool GROUPED = false>
 static cudaError_t launch_tc(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeParams& p, int num_sms,
                              cudaStream_t stream) {
     using C = TileCfg<FP8, D>;
     const int smem = WARPS * STAGES * C::kStageBytes + 1024;
-    auto kern = decode_tc_kernel<FP8, D, NT, WARPS, STAGES, BPS>;
+    auto kern = decode_tc_kernel<FP8, D, NT, WARPS, STAGES, BPS, GROUPED>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3(num_sms), dim3(WARPS * 32), smem, stream, tmK, tmV, p);
@@ -631,14 +676,30 @@ extern "C" int pkv_debug_timeline(void* host, int rows) {
 #endif
 
 
-int decode_tc_warps(bool fp8, int head_dim) {
+// The shared-prefix variant (bf16, head_dim 128) holds 16 score columns.
+#ifndef PKV_TC_WARPS_GROUPED
+#define PKV_TC_WARPS_GROUPED 12
+#endif
+#ifndef PKV_TC_STAGES_GROUPED
+#define PKV_TC_STAGES_GROUPED 2
+#endif
+
+int decode_tc_warps(bool fp8, int head_dim, bool grouped) {
+    if (grouped) return PKV_TC_WARPS_GROUPED;
     if (fp8) return PKV_TC_WARPS_FP8;
     return head_dim == 128 ? PKV_TC_WARPS_BF16 : PKV_TC_WARPS_BF16_D64;
 }
 
+bool decode_tc_groupable(bool fp8, int head_dim, int group) { return !fp8 && head_dim == 128 && group <= 8; }
+
 cudaError_t launch_decode_tc(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeParams& p, bool fp8,
                              int num_sms, cudaStream_t stream) {
     const int nt = (p.group + 7) / 8;
+    if (p.num_groups > 0) {
+        if (!decode_tc_groupable(fp8, p.head_dim, p.group)) return cudaErrorInvalidValue;
+        return launch_tc<false, 128, 2, PKV_TC_WARPS_GROUPED, PKV_TC_STAGES_GROUPED, PKV_TC_BPS_BF16, true>(
+            tmK, tmV, p, num_sms, stream);
+    }
     if (fp8) {
         if (p.head_dim != 128) return cudaErrorInvalidValue;
         return nt == 1 ? launch_tc<true, 128, 1, PKV_TC_WARPS_FP8, PKV_TC_STAGES_FP8, PKV_TC_BPS_FP8>(tmK, tmV, p, num_sms, stream)

@@ -27,6 +27,11 @@ constexpr int kBlockSize = 16;
 //   items    int4  [num_seqs * max_parts]   (seq, partition, first block, blocks) work list
 //   part_ml  float2[num_seqs * num_heads * max_parts]   (m, l) per partition
 //   part_o   float [num_seqs * num_heads * max_parts * head_dim]
+// and, for the shared-prefix decode only (written by the plan):
+//   seq_sub     int32 [num_seqs]   subgroup of each sequence, -1 = none
+//   seq_k       int32 [num_seqs]   leading blocks the sequence shares with its subgroup
+//   sub_info    int4  [num_seqs]   (first member, members, shared blocks, 0) per subgroup
+//   sub_members int32 [num_seqs]   member sequences, subgroup by subgroup
 // Each region starts on a 256-byte boundary.
 struct WsHeader {
     int counter;        // next unit to hand out (zeroed by the plan kernel)
@@ -34,12 +39,14 @@ struct WsHeader {
     int num_units;      // num_items * num_kv_heads
     int partition;      // largest partition in tokens chosen for this call
     int timeout;        // set when a bounded wait ran out
-    int pad[59];
+    int num_subs;       // shared-prefix subgroups built by the plan
+    int num_members;    // sequences in those subgroups
+    int pad[57];
 };
 static_assert(sizeof(WsHeader) == 256, "header is one 256-byte line");
 
 struct WsLayout {
-    size_t nparts, items, part_ml, part_o, total;
+    size_t nparts, items, part_ml, part_o, seq_sub, seq_k, sub_info, sub_members, total;
     int max_parts;
 };
 
@@ -57,6 +64,24 @@ __host__ __device__ inline WsLayout ws_layout(int num_seqs, int num_heads, int h
     off = pkv_align256(off + sizeof(float2) * (size_t)num_seqs * num_heads * max_parts);
     L.part_o = off;
     off = pkv_align256(off + sizeof(float) * (size_t)num_seqs * num_heads * max_parts * head_dim);
+    L.seq_sub = L.seq_k = L.sub_info = L.sub_members = 0;
+    L.total = off;
+    return L;
+}
+
+// Layout of the shared-prefix decode: one more partition per sequence (its
+// shared and its own blocks are cut separately) and the subgroup arrays.
+__host__ __device__ inline WsLayout ws_layout_shared(int num_seqs, int num_heads, int head_dim, int max_parts) {
+    WsLayout L = ws_layout(num_seqs, num_heads, head_dim, max_parts + 1);
+    size_t off = L.total;
+    L.seq_sub = off;
+    off = pkv_align256(off + sizeof(int) * (size_t)num_seqs);
+    L.seq_k = off;
+    off = pkv_align256(off + sizeof(int) * (size_t)num_seqs);
+    L.sub_info = off;
+    off = pkv_align256(off + sizeof(int4) * (size_t)num_seqs);
+    L.sub_members = off;
+    off = pkv_align256(off + sizeof(int) * (size_t)num_seqs);
     L.total = off;
     return L;
 }
@@ -86,6 +111,19 @@ struct DecodeParams {
     float* part_o;
     int max_parts;
     int32_t* err;
+    // Shared-prefix groups (num_groups == 0: none).  Hints from the caller:
+    // group g lists sequences group_seqs[group_offsets[g] .. group_offsets[g+1])
+    // that claim to share their first group_shared_blocks[g] blocks.
+    const int32_t* group_offsets;
+    const int32_t* group_seqs;
+    const int32_t* group_shared_blocks;
+    int num_groups;
+    int num_group_seqs;  // entries of group_seqs (offsets are clamped to it)
+    int group_cap;       // members per subgroup: their query heads fill 16 score columns
+    int* seq_sub;        // the plan's checked subgroups (workspace)
+    int* seq_k;
+    int4* sub_info;
+    int* sub_members;
 };
 
 // ------------------------------------------------------------------ small helpers

@@ -63,9 +63,19 @@ def decode_workspace_bytes(num_seqs, num_heads, head_dim, max_context_len, parti
     return int(n)
 
 
-def decode_workspace(num_seqs, num_heads, head_dim, max_context_len, partition_tokens=0, device=None):
-    """Allocate (through torch) a decode workspace for these bounds."""
-    n = decode_workspace_bytes(num_seqs, num_heads, head_dim, max_context_len, partition_tokens)
+def decode_workspace_bytes_shared(num_seqs, num_heads, head_dim, max_context_len, partition_tokens=0):
+    n = L.lib().pkv_decode_workspace_bytes_shared(int(num_seqs), int(num_heads), int(head_dim),
+                                                  int(max_context_len), int(partition_tokens))
+    if n == 0:
+        raise ValueError("invalid workspace bounds")
+    return int(n)
+
+
+def decode_workspace(num_seqs, num_heads, head_dim, max_context_len, partition_tokens=0, device=None, shared=False):
+    """Allocate (through torch) a decode workspace for these bounds (shared=True:
+    for paged_attention_decode_shared)."""
+    f = decode_workspace_bytes_shared if shared else decode_workspace_bytes
+    n = f(num_seqs, num_heads, head_dim, max_context_len, partition_tokens)
     return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
 
 
@@ -85,6 +95,33 @@ def paged_attention_decode(out, q, k_pool, v_pool, block_tables, context_lens, s
         Hq, Hkv, D, float(scale), float(k_scale), float(v_scale), int(partition_tokens),
         _ptr(workspace), int(workspace.numel() * workspace.element_size()), _ptr(err_count), _stream(stream))
     L.check("pkv_paged_attention_decode", st)
+    return out
+
+
+def paged_attention_decode_shared(out, q, k_pool, v_pool, block_tables, context_lens, scale, max_context_len,
+                                  workspace, group_offsets, group_seqs, group_shared_blocks, k_scale=1.0,
+                                  v_scale=1.0, partition_tokens=0, err_count=None, stream=None):
+    """paged_attention_decode that reads blocks shared by a group of sequences
+    once for the group.  The groups (int32 device tensors, see
+    BlockManager.prefix_groups) are hints; the kernels check them."""
+    S, Hq, D = q.shape
+    NB, bs, Hkv, D2 = k_pool.shape
+    if D2 != D or out.shape != q.shape:
+        raise ValueError("shape mismatch")
+    for t in (block_tables, context_lens, group_offsets, group_seqs, group_shared_blocks):
+        if t.dtype != torch.int32:
+            raise TypeError("tables, lengths and groups must be int32")
+    ng = int(group_shared_blocks.numel())
+    if group_offsets.numel() != ng + 1:
+        raise ValueError("group_offsets must have num_groups + 1 entries")
+    st = L.lib().pkv_paged_attention_decode_shared(
+        _ptr(out), _ptr(q), _dtype_code(q), _ptr(k_pool), _ptr(v_pool), _dtype_code(k_pool),
+        _ptr(block_tables), int(block_tables.shape[1]), _ptr(context_lens), S, int(max_context_len), NB, bs,
+        Hq, Hkv, D, float(scale), float(k_scale), float(v_scale), int(partition_tokens),
+        _ptr(group_offsets) if ng else None, _ptr(group_seqs) if group_seqs.numel() else None,
+        int(group_seqs.numel()), _ptr(group_shared_blocks) if ng else None, ng,
+        _ptr(workspace), int(workspace.numel() * workspace.element_size()), _ptr(err_count), _stream(stream))
+    L.check("pkv_paged_attention_decode_shared", st)
     return out
 
 

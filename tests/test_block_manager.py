@@ -210,3 +210,31 @@ def test_swap_errors(BM):
     assert bm.num_free_host() == 4 and bm.num_free() == 8
     bm.set_host_pool(8)
     assert bm.num_free_host() == 8
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_prefix_groups_match_reference(BM, seed):
+    """Random families of forks with divergent continuations: the native hints
+    equal the reference manager's for random batches."""
+    rng = np.random.default_rng(300 + seed)
+    NB = 600
+    order = rng.permutation(NB)
+    bm, ref = BM(NB, 16, free_order=order), RefBlockManager(NB, 16, free_order=order)
+    live = []
+    for fam in range(12):
+        n = int(rng.integers(0, 120))
+        a, r = bm.alloc_seq(n), ref.alloc_seq(n)
+        assert a == r
+        live.append(a)
+        for _ in range(int(rng.integers(0, 4))):
+            src = live[int(rng.integers(len(live)))]
+            assert bm.fork(src) == ref.fork(src)
+            live.append(len(live))
+    for _ in range(400):
+        s = live[int(rng.integers(len(live)))]
+        assert bm.append_token(s) == ref.append_token(s)
+    for _ in range(20):
+        batch = [live[int(i)] for i in rng.choice(len(live), size=int(rng.integers(1, len(live))), replace=False)]
+        offs, mem, sh = bm.prefix_groups(batch)
+        r_offs, r_mem, r_sh = ref.prefix_groups(batch)
+        assert (offs.tolist(), mem.tolist(), sh.tolist()) == (r_offs, r_mem, r_sh)
