@@ -220,11 +220,13 @@ int pkv_paged_attention_decode_noalloc(void* out, const void* q, int q_dtype,
  *   group_offsets        [num_groups + 1]  group g is group_seqs[offsets[g] .. offsets[g+1])
  *   group_seqs           [num_group_seqs]  batch indices (0 .. num_seqs-1) of its members
  *   group_shared_blocks  [num_groups]      leading blocks the members are said to share
- * These are hints (pkv_bm_prefix_groups computes them): the kernels keep a
- * member only if it is in range and in no earlier-claimed group, and cut a
- * group's shared blocks to those every kept member holds in full (16 tokens
- * within its context) with the same physical id in every member's table.  A
- * wrong hint costs time, never correctness.  Up to 1024 members per group are
+ * These are hints (pkv_bm_prefix_groups computes them): the plan keeps a
+ * member only if it is in range and in no group claimed before (claim order
+ * between groups is unspecified), and cuts a group's shared blocks to those
+ * every kept member holds in full (16 tokens within its context); each work
+ * item over shared blocks checks that its members' tables name the same
+ * physical blocks and, where they do not, runs once per member.  A wrong hint
+ * costs time, never correctness.  Up to 512 members per group are
  * considered.  The result equals pkv_paged_attention_decode's up to rounding
  * (partitions are cut differently: each sequence's shared and own blocks
  * separately).  Grouping applies to bf16 caches with head_dim 128 and at most 8
@@ -337,6 +339,29 @@ int pkv_bm_tables(const pkv_block_manager* bm, const int32_t* seqs, int n, int32
                   int max_blocks, int32_t pad, int32_t* lens);
 /* Current free list, front first (n_out entries). */
 int pkv_bm_free_list(const pkv_block_manager* bm, int32_t* out, int cap, int* n_out);
+
+/* Prefix caching across requests (full-block hashing: the glossary entry's
+ * sharing section says hashing whole blocks extends sharing to separate
+ * requests, which is how prompt caching is implemented).  With the cache on,
+ * alloc_seq_tokens registers every full block of a prompt under the key
+ * (parent block's registration, its block_size token ids); a later prompt
+ * that begins with the same tokens gets the same physical blocks for its
+ * longest run of matching leading full blocks (reference counts + 1) and
+ * *num_cached_out = that run x block_size: the caller writes K/V only for
+ * tokens [num_cached, num_tokens).  Keys hold the exact tokens (a hash picks
+ * the bucket only), so different prefixes never collide.  A registered block
+ * whose count drops to 0 keeps its contents and its key and goes to the back
+ * of the free list; a hit takes it back out; when the free list hands it out
+ * for new data its key is dropped.  Only prompt blocks are registered (tokens
+ * appended later carry no ids here); registered blocks are always full, so
+ * copy-on-write never touches them.  PKV_ENOMEM (nothing changed) if the
+ * blocks that are not hits, plus the hits that must leave the free list, do
+ * not fit.  With the cache off, alloc_seq_tokens is alloc_seq; turning it off
+ * forgets every key. */
+int pkv_bm_set_prefix_cache(pkv_block_manager* bm, int enable);
+int pkv_bm_alloc_seq_tokens(pkv_block_manager* bm, const int32_t* tokens, int num_tokens, int32_t* seq_out,
+                            int* num_cached_out);
+int pkv_bm_num_cached_blocks(const pkv_block_manager* bm);
 
 /* Shared-prefix hints for pkv_paged_attention_decode_shared, for the batch
  * seqs[0..n) (in that order: members are given as batch indices 0..n-1).

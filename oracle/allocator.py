@@ -16,6 +16,8 @@ Written from the pages' description of the host side of PagedAttention:
   only the block that must split is copied; blocks with no references are freed.
 - same glossary page, "Tecnicas relacionadas" (continuous batching): a finished
   sequence's blocks return to the free pool at once.
+- same glossary page, end of the sharing section: hashing whole blocks extends
+  sharing across requests (prompt caching).
 - "Le cache KV et PagedAttention" (gyaansetu.com), fine-grained eviction: when
   memory runs out, a sequence's small pages can go to the CPU instead of the
   whole sequence being dropped, and come back later.
@@ -28,6 +30,11 @@ blocks raises MemoryError and leaves the state unchanged.  Swap moves all of a
 sequence's pages at once to a host pool with its own first-in first-out free
 list (ids 0..n-1); a page shared with another sequence is copied out and comes
 back as a private block; a swapped sequence can only be swapped in or freed.
+Prefix caching keys a full prompt block by its exact token ids and its parent
+block's registration (a number never reused), registers only prompt blocks,
+reuses the longest run of matching leading full blocks, keeps an unused
+registered block's key while it waits in the free list (a hit takes it back
+out of the list), and drops the key when the block is handed out for new data.
 """
 from collections import deque
 
@@ -50,6 +57,10 @@ class RefBlockManager:
         self._next = 0
         self.host_free = deque()
         self.swapped = set()
+        self.prefix_cache = False
+        self.cache = {}            # (parent serial, token tuple) -> (block, serial)
+        self.key_of = {}           # block -> its key
+        self._serial = 0
 
     # -- allocation ---------------------------------------------------------
     def _pop(self):
@@ -58,6 +69,8 @@ class RefBlockManager:
         b = self.free.popleft()
         assert self.ref[b] == 0
         self.ref[b] = 1
+        if b in self.key_of:              # new contents: forget the old key
+            del self.cache[self.key_of.pop(b)]
         return b
 
     def alloc_seq(self, num_tokens):
@@ -70,6 +83,50 @@ class RefBlockManager:
         self.tables[seq] = [self._pop() for _ in range(need)]
         self.lens[seq] = num_tokens
         return seq
+
+    def set_prefix_cache(self, enable=True):
+        self.prefix_cache = bool(enable)
+        if not enable:
+            self.cache.clear()
+            self.key_of.clear()
+
+    def alloc_seq_tokens(self, tokens):
+        """New sequence for a prompt given by token ids.
+
+        Returns (seq, number of leading tokens whose blocks came from the cache).
+        """
+        tokens = [int(t) for t in tokens]
+        if not self.prefix_cache:
+            return self.alloc_seq(len(tokens)), 0
+        bs = self.block_size
+        full = len(tokens) // bs
+        need = -(-len(tokens) // bs)
+        hits, parent = [], 0
+        for j in range(full):
+            key = (parent, tuple(tokens[j * bs:(j + 1) * bs]))
+            if key not in self.cache:
+                break
+            block, parent = self.cache[key]
+            hits.append(block)
+        waking = [b for b in hits if self.ref[b] == 0]
+        if need - len(hits) + len(waking) > len(self.free):
+            raise MemoryError("not enough free blocks")
+        for b in hits:
+            if self.ref[b] == 0:
+                self.free.remove(b)
+            self.ref[b] += 1
+        table = hits + [self._pop() for _ in range(need - len(hits))]
+        for j in range(len(hits), full):
+            self._serial += 1
+            key = (parent, tuple(tokens[j * bs:(j + 1) * bs]))
+            self.cache[key] = (table[j], self._serial)
+            self.key_of[table[j]] = key
+            parent = self._serial
+        seq = self._next
+        self._next += 1
+        self.tables[seq] = table
+        self.lens[seq] = len(tokens)
+        return seq, len(hits) * bs
 
     def fork(self, parent):
         """New sequence sharing every block of `parent` (reference counts + 1)."""

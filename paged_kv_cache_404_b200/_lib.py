@@ -42,6 +42,9 @@ SIGNATURES = {
     "pkv_bm_tables": (_i, [_p, _p, _i, _p, _i, C.c_int32, _p]),
     "pkv_bm_free_list": (_i, [_p, _p, _i, _p]),
     "pkv_bm_prefix_groups": (_i, [_p, _p, _i, _p, _p, _p, _p]),
+    "pkv_bm_set_prefix_cache": (_i, [_p, _i]),
+    "pkv_bm_alloc_seq_tokens": (_i, [_p, _p, _i, _p, _p]),
+    "pkv_bm_num_cached_blocks": (_i, [_p]),
     "pkv_bm_set_host_pool": (_i, [_p, _i]),
     "pkv_bm_swap_out": (_i, [_p, C.c_int32, _p, _i, _p]),
     "pkv_bm_swap_in": (_i, [_p, C.c_int32, _p, _i, _p]),

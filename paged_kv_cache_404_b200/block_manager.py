@@ -107,6 +107,22 @@ class BlockManager:
         L.check("pkv_bm_free_list", self._lib.pkv_bm_free_list(self._h, out.ctypes.data, out.size, C.byref(n)))
         return out[:n.value].copy()
 
+    # --- prefix caching across requests (full-block keys) ----------------------
+
+    def set_prefix_cache(self, enable=True):
+        L.check("pkv_bm_set_prefix_cache", self._lib.pkv_bm_set_prefix_cache(self._h, int(bool(enable))))
+
+    def alloc_seq_tokens(self, tokens):
+        """New sequence for a prompt given by token ids; returns (seq, tokens already cached)."""
+        t = np.ascontiguousarray(tokens, dtype=np.int32)
+        seq, cached = C.c_int32(), C.c_int()
+        L.check("pkv_bm_alloc_seq_tokens", self._lib.pkv_bm_alloc_seq_tokens(
+            self._h, t.ctypes.data if t.size else None, t.size, C.byref(seq), C.byref(cached)))
+        return seq.value, cached.value
+
+    def num_cached_blocks(self):
+        return self._lib.pkv_bm_num_cached_blocks(self._h)
+
     def prefix_groups(self, seqs):
         """Shared-prefix hints of a batch: (offsets int32 [g+1], members int32 [m], shared int32 [g])."""
         seqs = np.ascontiguousarray(seqs, dtype=np.int32)

@@ -19,21 +19,54 @@
 //  - swap: a sequence's pages can move to a host pool and back, page by page,
 //    instead of evicting whole sequences ("Le cache KV et PagedAttention",
 //    fine-grained eviction); the manager decides the block pairs, the copies
-//    run on the GPU (pkv_swap_blocks).
+//    run on the GPU (pkv_swap_blocks);
+//  - prefix caching: full prompt blocks are registered under a key made of
+//    their tokens and their parent block's key, so a later request whose
+//    prompt starts the same way reuses them (glossary entry, full-block
+//    hashing extends sharing across requests).  A registered block that no
+//    sequence uses stays in the free list with its contents; a hit takes it
+//    back out, and reusing it for new data drops its registration.
 // Plain C++ with host memory only; exported through the C ABI in pagedkv.h.
 #include <cstdint>
 #include <cstring>
 #include <deque>
+#include <functional>
 #include <new>
 #include <unordered_map>
 #include <vector>
 
 #include "pagedkv.h"
 
+// Key of a full prompt block: the registration serial of its parent block (0
+// for a prompt's first block), then its block_size token ids.  Exact content,
+// hashed only to find the bucket, so two different prefixes never share a key.
+struct KeyHash {
+    size_t operator()(const std::vector<int64_t>& k) const {
+        uint64_t h = 1469598103934665603ull;
+        for (int64_t x : k) {
+            h ^= (uint64_t)x;
+            h *= 1099511628211ull;
+            h ^= h >> 29;
+        }
+        return (size_t)h;
+    }
+};
+
+struct CachedBlock {
+    int32_t block;
+    uint64_t serial;  // unique per registration: children are keyed by it
+};
+
 struct pkv_block_manager {
     int num_blocks = 0;
     int block_size = 0;
-    std::deque<int32_t> free_list;
+    // Free list, first in first out.  An entry is live while its block is free
+    // and its generation matches; a cached block taken back out of the list
+    // leaves a dead entry behind (skipped when it reaches the front).
+    std::deque<std::pair<int32_t, uint32_t>> free_q;
+    std::vector<uint32_t> free_gen;
+    std::vector<uint8_t> is_free;
+    size_t free_count = 0;
     std::vector<int32_t> refs;                  // per physical block
     std::vector<std::vector<int32_t>> tables;   // per sequence id
     std::vector<int32_t> lens;                  // tokens per sequence
@@ -42,6 +75,10 @@ struct pkv_block_manager {
     int num_host_blocks = 0;
     std::deque<int32_t> host_free;
     std::vector<uint8_t> host_used;
+    bool prefix_cache = false;
+    uint64_t next_serial = 1;
+    std::unordered_map<std::vector<int64_t>, CachedBlock, KeyHash> cache;
+    std::vector<std::vector<int64_t>> key_of;  // per block: its key, empty if unregistered
 
     bool valid_seq(int32_t s) const { return s >= 0 && (size_t)s < tables.size() && alive[s]; }
     // resident (on the device) sequence: PKV_OK, else the error to return
@@ -50,11 +87,43 @@ struct pkv_block_manager {
         return swapped[s] ? PKV_ESWAPPED : PKV_OK;
     }
 
-    int32_t take_block() {
-        const int32_t b = free_list.front();
-        free_list.pop_front();
+    void push_free(int32_t b) {
+        is_free[b] = 1;
+        free_q.emplace_back(b, ++free_gen[b]);
+        ++free_count;
+    }
+
+    // a cached free block reused by a hit: its queue entry goes dead
+    void revive(int32_t b) {
+        is_free[b] = 0;
+        --free_count;
         refs[b] = 1;
-        return b;
+    }
+
+    void uncache(int32_t b) {
+        if (!key_of.empty() && !key_of[b].empty()) {
+            cache.erase(key_of[b]);
+            key_of[b].clear();
+        }
+    }
+
+    int32_t take_block() {
+        for (;;) {
+            const std::pair<int32_t, uint32_t> e = free_q.front();
+            free_q.pop_front();
+            if (is_free[e.first] && free_gen[e.first] == e.second) {
+                const int32_t b = e.first;
+                is_free[b] = 0;
+                --free_count;
+                uncache(b);  // new contents: the old key no longer describes it
+                refs[b] = 1;
+                return b;
+            }
+        }
+    }
+
+    void release(int32_t b) {
+        if (--refs[b] == 0) push_free(b);
     }
 
     int32_t new_seq(std::vector<int32_t>&& table, int32_t len) {
@@ -76,8 +145,10 @@ int pkv_bm_create(int num_blocks, int block_size, const int32_t* free_order, int
     bm->num_blocks = num_blocks;
     bm->block_size = block_size;
     bm->refs.assign(num_blocks, 0);
+    bm->free_gen.assign(num_blocks, 0);
+    bm->is_free.assign(num_blocks, 0);
     if (free_order == nullptr) {
-        for (int b = 0; b < num_blocks; ++b) bm->free_list.push_back(b);
+        for (int b = 0; b < num_blocks; ++b) bm->push_free(b);
     } else {
         std::vector<uint8_t> seen(num_blocks, 0);
         for (int i = 0; i < free_count; ++i) {
@@ -87,7 +158,7 @@ int pkv_bm_create(int num_blocks, int block_size, const int32_t* free_order, int
                 return PKV_EINVAL;
             }
             seen[b] = 1;
-            bm->free_list.push_back(b);
+            bm->push_free(b);
         }
     }
     *out = bm;
@@ -99,7 +170,7 @@ void pkv_bm_destroy(pkv_block_manager* bm) { delete bm; }
 int pkv_bm_alloc_seq(pkv_block_manager* bm, int num_tokens, int32_t* seq_out) {
     if (bm == nullptr || seq_out == nullptr || num_tokens < 0) return PKV_EINVAL;
     const size_t need = ((size_t)num_tokens + bm->block_size - 1) / bm->block_size;
-    if (need > bm->free_list.size()) return PKV_ENOMEM;
+    if (need > bm->free_count) return PKV_ENOMEM;
     std::vector<int32_t> table;
     table.reserve(need);
     for (size_t i = 0; i < need; ++i) table.push_back(bm->take_block());
@@ -134,14 +205,14 @@ int pkv_bm_append_tokens(pkv_block_manager* bm, const int32_t* seqs, int n, int6
         const int32_t off = len % bm->block_size;
         if (off == 0) {
             // last block full (or none yet): next free block, nothing to copy
-            if (bm->free_list.empty()) {
+            if (bm->free_count == 0) {
                 status = PKV_ENOMEM;
                 break;
             }
             table.push_back(bm->take_block());
         } else if (bm->refs[table.back()] > 1) {
             // partly filled block still shared: copy it, write into the copy
-            if (bm->free_list.empty()) {
+            if (bm->free_count == 0) {
                 status = PKV_ENOMEM;
                 break;
             }
@@ -171,7 +242,7 @@ int pkv_bm_free_seq(pkv_block_manager* bm, int32_t seq) {
         }
     } else {
         for (int32_t b : bm->tables[seq]) {
-            if (--bm->refs[b] == 0) bm->free_list.push_back(b);
+            bm->release(b);
         }
     }
     bm->tables[seq].clear();
@@ -182,7 +253,7 @@ int pkv_bm_free_seq(pkv_block_manager* bm, int32_t seq) {
     return PKV_OK;
 }
 
-int pkv_bm_num_free(const pkv_block_manager* bm) { return bm ? (int)bm->free_list.size() : -1; }
+int pkv_bm_num_free(const pkv_block_manager* bm) { return bm ? (int)bm->free_count : -1; }
 
 int pkv_bm_seq_len(const pkv_block_manager* bm, int32_t seq, int32_t* len_out) {
     if (bm == nullptr || len_out == nullptr) return PKV_EINVAL;
@@ -236,10 +307,11 @@ int pkv_bm_tables(const pkv_block_manager* bm, const int32_t* seqs, int n, int32
 
 int pkv_bm_free_list(const pkv_block_manager* bm, int32_t* out, int cap, int* n_out) {
     if (bm == nullptr || n_out == nullptr || cap < 0 || (cap > 0 && out == nullptr)) return PKV_EINVAL;
-    *n_out = (int)bm->free_list.size();
-    if ((int)bm->free_list.size() > cap) return PKV_EINVAL;
+    *n_out = (int)bm->free_count;
+    if ((int)bm->free_count > cap) return PKV_EINVAL;
     int i = 0;
-    for (int32_t b : bm->free_list) out[i++] = b;
+    for (const std::pair<int32_t, uint32_t>& e : bm->free_q)
+        if (bm->is_free[e.first] && bm->free_gen[e.first] == e.second) out[i++] = e.first;
     return PKV_OK;
 }
 
@@ -287,6 +359,74 @@ int pkv_bm_prefix_groups(const pkv_block_manager* bm, const int32_t* seqs, int n
     return PKV_OK;
 }
 
+int pkv_bm_set_prefix_cache(pkv_block_manager* bm, int enable) {
+    if (bm == nullptr) return PKV_EINVAL;
+    bm->prefix_cache = enable != 0;
+    if (!bm->prefix_cache) {
+        bm->cache.clear();
+        bm->key_of.clear();
+    } else if (bm->key_of.empty()) {
+        bm->key_of.assign(bm->num_blocks, {});
+    }
+    return PKV_OK;
+}
+
+int pkv_bm_alloc_seq_tokens(pkv_block_manager* bm, const int32_t* tokens, int num_tokens, int32_t* seq_out,
+                            int* num_cached_out) {
+    if (bm == nullptr || seq_out == nullptr || num_tokens < 0 || (num_tokens > 0 && tokens == nullptr))
+        return PKV_EINVAL;
+    if (!bm->prefix_cache) {
+        if (num_cached_out) *num_cached_out = 0;
+        return pkv_bm_alloc_seq(bm, num_tokens, seq_out);
+    }
+    const int bs = bm->block_size;
+    const int full = num_tokens / bs;
+    const size_t need = ((size_t)num_tokens + bs - 1) / bs;
+    auto key = [&](uint64_t parent, int j) {
+        std::vector<int64_t> k;
+        k.reserve(bs + 1);
+        k.push_back((int64_t)parent);
+        for (int i = 0; i < bs; ++i) k.push_back(tokens[(size_t)j * bs + i]);
+        return k;
+    };
+    // 1. longest run of leading full blocks already registered
+    std::vector<CachedBlock> hits;
+    uint64_t parent = 0;
+    for (int j = 0; j < full; ++j) {
+        auto it = bm->cache.find(key(parent, j));
+        if (it == bm->cache.end()) break;
+        hits.push_back(it->second);
+        parent = it->second.serial;
+    }
+    size_t revived = 0;
+    for (const CachedBlock& h : hits) revived += bm->refs[h.block] == 0;
+    if (need - hits.size() + revived > bm->free_count) return PKV_ENOMEM;
+    // 2. take the hits (shared, or back out of the free list), then new blocks
+    std::vector<int32_t> table;
+    table.reserve(need);
+    for (const CachedBlock& h : hits) {
+        if (bm->refs[h.block] == 0)
+            bm->revive(h.block);
+        else
+            ++bm->refs[h.block];
+        table.push_back(h.block);
+    }
+    while (table.size() < need) table.push_back(bm->take_block());
+    // 3. register the new full blocks, each keyed by its parent's serial
+    for (int j = (int)hits.size(); j < full; ++j) {
+        std::vector<int64_t> k = key(parent, j);
+        const CachedBlock c{table[j], bm->next_serial++};
+        bm->key_of[c.block] = k;
+        bm->cache.emplace(std::move(k), c);
+        parent = c.serial;
+    }
+    if (num_cached_out) *num_cached_out = (int)hits.size() * bs;
+    *seq_out = bm->new_seq(std::move(table), num_tokens);
+    return PKV_OK;
+}
+
+int pkv_bm_num_cached_blocks(const pkv_block_manager* bm) { return bm ? (int)bm->cache.size() : -1; }
+
 int pkv_bm_set_host_pool(pkv_block_manager* bm, int num_host_blocks) {
     if (bm == nullptr || num_host_blocks < 0) return PKV_EINVAL;
     for (uint8_t u : bm->host_used)
@@ -314,7 +454,7 @@ int pkv_bm_swap_out(pkv_block_manager* bm, int32_t seq, int64_t* pairs_out, int 
         pairs_out[2 * i] = d;
         pairs_out[2 * i + 1] = h;
         // a page another sequence still uses stays on the device
-        if (--bm->refs[d] == 0) bm->free_list.push_back(d);
+        bm->release(d);
         table[i] = h;
     }
     bm->swapped[seq] = 1;
@@ -330,7 +470,7 @@ int pkv_bm_swap_in(pkv_block_manager* bm, int32_t seq, int64_t* pairs_out, int c
     const int k = (int)table.size();
     *num_pairs_out = 0;
     if (k > cap || (k > 0 && pairs_out == nullptr)) return PKV_EINVAL;
-    if ((size_t)k > bm->free_list.size()) return PKV_ENOMEM;
+    if ((size_t)k > bm->free_count) return PKV_ENOMEM;
     for (int i = 0; i < k; ++i) {
         const int32_t h = table[i];
         const int32_t d = bm->take_block();

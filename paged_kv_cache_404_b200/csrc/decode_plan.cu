@@ -67,97 +67,84 @@ __device__ __forceinline__ int for_each_piece(int B, int nb, int mb, bool geomet
 // Shared-prefix groups.  Sequences that start with the same physical blocks
 // (parallel samples of one prompt, requests with a common system prompt: the
 // glossary entry "PagedAttention", "Compartir bloques entre secuencias") can
-// read those blocks once for all of them.  The caller's hints are checked
-// here, never trusted: a member is kept only if it is in range and not already
-// in another group; the shared count is cut to the leading blocks that every
-// kept member holds in full and that are the same physical block in all their
-// tables.  A kept group is split into subgroups of at most group_cap members
-// (balanced sizes).  A wrong hint costs speed, not correctness.
-constexpr int kMaxGroupChunks = 32;  // members per group considered: 32 * 32
+// read those blocks once for all of them.  The caller's hints are not trusted:
+// here a member is kept only if it is in range and in no group claimed before,
+// and the shared count is cut to the blocks every kept member holds in full
+// (16 tokens inside its context).  That the members' tables really agree on
+// those blocks is checked by the decode kernel, item by item (a subgroup item
+// whose members' tables differ is run once per member).  A kept group is split
+// into subgroups of at most group_cap members (balanced sizes).  A wrong hint
+// costs time, never correctness.
+constexpr int kMaxGroupChunks = 32;  // members per group considered: 16 * 32
 
+// One half-warp per group (two groups per warp at a time, so that the loads of
+// both groups' three dependent steps -- hint, members, claim -- overlap).
 __device__ void build_groups(const DecodeParams& p, int* n_subs, int* n_members) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int half = lane >> 4, hl = lane & 15;
+    const int hbase = lane & 16;  // first lane of this half
     for (int s = tid; s < p.num_seqs; s += kPlanThreads) {
         p.seq_sub[s] = -1;
         p.seq_k[s] = 0;
     }
     __syncthreads();
-    for (int gi = warp; gi < p.num_groups; gi += kPlanThreads / 32) {
-        const int beg = p.group_offsets[gi];
-        if (beg < 0 || beg >= p.num_group_seqs) continue;
-        const int end = min(min(p.group_offsets[gi + 1], p.num_group_seqs), beg + 32 * kMaxGroupChunks);
-        int k = min(p.group_shared_blocks[gi], p.max_blocks_per_seq);
-        if (end <= beg + 1 || k <= 0) continue;
-        const int nchunks = (end - beg + 31) >> 5;
+    constexpr int kGroupsPerPass = 2 * (kPlanThreads / 32);
+    for (int g0 = 0; g0 < p.num_groups; g0 += kGroupsPerPass) {
+        const int gi = g0 + 2 * warp + half;
+        int beg = 0, end = 0, k = 0;
+        if (gi < p.num_groups) {
+            beg = p.group_offsets[gi];
+            end = p.group_offsets[gi + 1];
+            k = min(p.group_shared_blocks[gi], p.max_blocks_per_seq);
+        }
+        if (beg < 0 || beg >= p.num_group_seqs) end = beg;  // no members
+        end = min(min(end, p.num_group_seqs), beg + 16 * kMaxGroupChunks);
+        const bool live = end > beg + 1 && k > 0;
+        const int nchunks = live ? (end - beg + 15) >> 4 : 0;
+        const int nchunks_warp = max(nchunks, __shfl_xor_sync(0xffffffffu, nchunks, 16));
 
-        // claim the members (bit c of `mine`: member beg + 32c + lane is ours)
+        // claim the members (bit c of `mine`: member beg + 16c + hl is ours);
+        // the length is loaded alongside the claim
         uint32_t mine = 0;
-        int count = 0, s0 = -1;
-        for (int c = 0; c < nchunks; ++c) {
-            const int i = beg + 32 * c + lane;
-            const int s = i < end ? p.group_seqs[i] : -1;
-            bool got = false;
-            if (s >= 0 && s < p.num_seqs && atomicCAS(&p.seq_sub[s], -1, -2) == -1) {
-                got = true;
-                k = min(k, clamped_len(p, s, false) / kBlockSize);
-            }
-            const unsigned b = __ballot_sync(0xffffffffu, got);
+        int count = 0, s_lane = -1;
+        for (int c = 0; c < nchunks_warp; ++c) {
+            const int i = beg + 16 * c + hl;
+            const int s = (c < nchunks && i < end) ? p.group_seqs[i] : -1;
+            const bool valid = s >= 0 && s < p.num_seqs;
+            const int len = valid ? clamped_len(p, s, false) : 0;
+            const bool got = valid && atomicCAS(&p.seq_sub[s], -1, -2) == -1;
+            if (got) k = min(k, len / kBlockSize);
+            const unsigned b = (__ballot_sync(0xffffffffu, got) >> hbase) & 0xFFFFu;
             if (got) mine |= 1u << c;
-            if (s0 < 0 && b) s0 = __shfl_sync(0xffffffffu, s, __ffs(b) - 1);
+            if (c == 0) s_lane = s;
             count += __popc(b);
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) k = min(k, __shfl_xor_sync(0xffffffffu, k, o));
+        for (int o = 8; o > 0; o >>= 1) k = min(k, __shfl_xor_sync(0xffffffffu, k, o));
 
-        // cut k at the first block where a member's table differs from s0's
-        if (count >= 2 && k > 0) {
-            const int32_t* ref = p.block_tables + (size_t)s0 * p.max_blocks_per_seq;
-            for (int j0 = 0; j0 < k; j0 += 32) {
-                const int j = j0 + lane;
-                const int r = j < k ? __ldg(ref + j) : 0;
-                bool diff = false;
-                for (int c = 0; c < nchunks; ++c) {
-                    const int i = beg + 32 * c + lane;
-                    const int sl = ((mine >> c) & 1u) ? p.group_seqs[i] : -1;
-                    unsigned b = __ballot_sync(0xffffffffu, sl >= 0);
-                    while (b) {
-                        const int src = __ffs(b) - 1;
-                        b &= b - 1;
-                        const int sm = __shfl_sync(0xffffffffu, sl, src);
-                        if (j < k && __ldg(p.block_tables + (size_t)sm * p.max_blocks_per_seq + j) != r) diff = true;
-                    }
-                }
-                const unsigned d = __ballot_sync(0xffffffffu, diff);
-                if (d) {
-                    k = j0 + __ffs(d) - 1;
-                    break;
-                }
-            }
-        }
-
-        const bool keep = count >= 2 && k > 0;
+        const bool keep = live && count >= 2 && k > 0;
         const int nsub = keep ? (count + p.group_cap - 1) / p.group_cap : 0;
         int mbase = 0, sbase = 0;
-        if (keep && lane == 0) {
+        if (keep && hl == 0) {
             mbase = atomicAdd(n_members, count);
             sbase = atomicAdd(n_subs, nsub);
         }
-        mbase = __shfl_sync(0xffffffffu, mbase, 0);
-        sbase = __shfl_sync(0xffffffffu, sbase, 0);
+        mbase = __shfl_sync(0xffffffffu, mbase, hbase);
+        sbase = __shfl_sync(0xffffffffu, sbase, hbase);
         if (keep)
-            for (int q = lane; q < nsub; q += 32) {
+            for (int q = hl; q < nsub; q += 16) {
                 const int a = (int)(((long long)q * count) / nsub), b = (int)(((long long)(q + 1) * count) / nsub);
                 p.sub_info[sbase + q] = make_int4(mbase + a, b - a, k, 0);
             }
         // members in claim order; member of rank r goes to subgroup ((r+1)*nsub - 1) / count
         int rank0 = 0;
-        for (int c = 0; c < nchunks; ++c) {
+        for (int c = 0; c < nchunks_warp; ++c) {
             const bool own = (mine >> c) & 1u;
-            const unsigned b = __ballot_sync(0xffffffffu, own);
+            const unsigned b = (__ballot_sync(0xffffffffu, own) >> hbase) & 0xFFFFu;
             if (own) {
-                const int s = p.group_seqs[beg + 32 * c + lane];
+                const int s = c == 0 ? s_lane : p.group_seqs[beg + 16 * c + hl];
                 if (keep) {
-                    const int r = rank0 + __popc(b & ((1u << lane) - 1u));
+                    const int r = rank0 + __popc(b & ((1u << hl) - 1u));
                     p.sub_members[mbase + r] = s;
                     p.seq_sub[s] = sbase + (int)(((long long)(r + 1) * nsub - 1) / count);
                     p.seq_k[s] = k;
@@ -171,10 +158,26 @@ __device__ void build_groups(const DecodeParams& p, int* n_subs, int* n_members)
     __syncthreads();
 }
 
+// Number of pieces for_each_piece cuts B blocks into (closed form of its loop).
+__device__ __noinline__ int count_pieces(int B, int nb, int mb, bool geometric) {
+    if (B <= 0) return 0;
+    if (!geometric) return (B + nb - 1) / nb;
+    const int body = (B - 1) / nb;
+    int T = B - body * nb, n = body + 1;
+    while (T > 2 * mb) {
+        T -= T / 2;
+        ++n;
+    }
+    return n;
+}
+
+constexpr int kSmemSeqs = 4096;  // per-sequence block counts kept in shared memory up to this many
+
 __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams p, int fixed_partition, int min_partition,
                                                                    int num_candidates, int target_units,
                                                                    int zero_out_dtype) {
     __shared__ int hist[kMaxBuckets];
+    __shared__ int own_blocks[kSmemSeqs];  // blocks of sequence s outside its shared prefix
     __shared__ unsigned long long units_of[kMaxCandidates];
     __shared__ int chosen;
     __shared__ int n_subs, n_members;
@@ -189,42 +192,31 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
     // 0. shared-prefix subgroups: sequence s then owns blocks [seq_k[s], B) and
     //    its subgroup computes blocks [0, seq_k[s]) once for all its members
     if (tid == 0) n_subs = n_members = 0;
+    if (tid < kMaxCandidates) units_of[tid] = 0;
     __syncthreads();
     const bool grouped = p.num_groups > 0;
     if (grouped) build_groups(p, &n_subs, &n_members);
     const int num_subs = n_subs;
-    auto own_k = [&](int s) { return grouped ? p.seq_k[s] : 0; };
+    // blocks of s after its shared prefix (the length is clamped and counted once, here)
+    auto own_of = [&](int s, bool count) {
+        return ceil_div(clamped_len(p, s, count), kBlockSize) - (grouped ? p.seq_k[s] : 0);
+    };
+    for (int s = tid; s < p.num_seqs && s < kSmemSeqs; s += kPlanThreads) own_blocks[s] = own_of(s, true);
+    for (int s = kSmemSeqs + tid; s < p.num_seqs; s += kPlanThreads) own_of(s, true);
+    __syncthreads();
+    auto own = [&](int s) { return s < kSmemSeqs ? own_blocks[s] : own_of(s, false); };
 
     // 1. largest partition: the largest candidate min_partition << c whose work
-    //    list still has target_units units (one pass over the lengths for all c)
-    if (tid < kMaxCandidates) units_of[tid] = 0;
-    __syncthreads();
+    //    list still has target_units units
     if (fixed_partition > 0) {
         if (tid == 0) chosen = fixed_partition;
     } else {
-        unsigned long long cnt[kMaxCandidates];
-#pragma unroll
-        for (int c = 0; c < kMaxCandidates; ++c) cnt[c] = 0;
-        for (int s = tid; s < p.num_seqs; s += kPlanThreads) {
-            const int B = ceil_div(clamped_len(p, s, false), kBlockSize) - own_k(s);
-#pragma unroll
-            for (int c = 0; c < kMaxCandidates; ++c)
-                if (c < num_candidates)
-                    cnt[c] += (unsigned long long)for_each_piece(B, (min_partition << c) / kBlockSize, mb, geometric,
-                                                                 [](int, int) {});
-        }
-        for (int q = tid; q < num_subs; q += kPlanThreads) {
-            const int k = p.sub_info[q].z;
-#pragma unroll
-            for (int c = 0; c < kMaxCandidates; ++c)
-                if (c < num_candidates)
-                    cnt[c] += (unsigned long long)for_each_piece(k, (min_partition << c) / kBlockSize, mb, geometric,
-                                                                 [](int, int) {});
-        }
-#pragma unroll
-        for (int c = 0; c < kMaxCandidates; ++c) {
-            if (c >= num_candidates) break;
-            unsigned long long v = cnt[c];
+#pragma unroll 1
+        for (int c = 0; c < num_candidates; ++c) {
+            const int nb = (min_partition << c) / kBlockSize;
+            unsigned long long v = 0;
+            for (int s = tid; s < p.num_seqs; s += kPlanThreads) v += count_pieces(own(s), nb, mb, geometric);
+            for (int q = tid; q < num_subs; q += kPlanThreads) v += count_pieces(p.sub_info[q].z, nb, mb, geometric);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
             if ((tid & 31) == 0 && v) atomicAdd(&units_of[c], v);
@@ -240,22 +232,20 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
             chosen = P;
         }
     }
+    for (int b = tid; b < kMaxBuckets; b += kPlanThreads) hist[b] = 0;
     __syncthreads();
     const int P = chosen;
     const int nb_top = P / kBlockSize;
     const int nbuckets = nb_top < kMaxBuckets ? nb_top : kMaxBuckets;
 
-    // 2. histogram of item sizes
-    for (int b = tid; b < kMaxBuckets; b += kPlanThreads) hist[b] = 0;
-    __syncthreads();
+    // 2. histogram of item sizes; partitions per sequence (shared ones first)
     for (int s = tid; s < p.num_seqs; s += kPlanThreads) {
-        const int L = clamped_len(p, s, true);
-        const int k = own_k(s);
-        const int B = ceil_div(L, kBlockSize) - k;
-        p.nparts[s] = for_each_piece(k, nb_top, mb, geometric, [](int, int) {}) +
+        const int k = grouped ? p.seq_k[s] : 0;
+        const int B = own(s);
+        p.nparts[s] = count_pieces(k, nb_top, mb, geometric) +
                       for_each_piece(B, nb_top, mb, geometric,
                                      [&](int, int n) { atomicAdd(&hist[bucket_of(n, nb_top, nbuckets)], 1); });
-        if (L == 0) {
+        if (B + k == 0) {
             // an empty context produces a zero output row (nothing else writes it)
             const size_t row = (size_t)s * p.num_heads * p.head_dim;
             const int n = p.num_heads * p.head_dim;
@@ -302,10 +292,9 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
     // 4. scatter the items (order inside a bucket does not affect results);
     //    a sequence's shared partitions come first, then its own
     for (int s = tid; s < p.num_seqs; s += kPlanThreads) {
-        const int k = own_k(s);
-        const int B = ceil_div(clamped_len(p, s, false), kBlockSize) - k;
-        int part = for_each_piece(k, nb_top, mb, geometric, [](int, int) {});
-        for_each_piece(B, nb_top, mb, geometric, [&](int first, int n) {
+        const int k = grouped ? p.seq_k[s] : 0;
+        int part = count_pieces(k, nb_top, mb, geometric);
+        for_each_piece(own(s), nb_top, mb, geometric, [&](int first, int n) {
             const int pos = atomicAdd(&hist[bucket_of(n, nb_top, nbuckets)], 1);
             p.items[pos] = make_int4(s, part++, k + first, n);
         });

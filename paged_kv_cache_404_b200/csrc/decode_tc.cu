@@ -131,20 +131,38 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
         if (u >= num_units) break;
         const int4 item = p.items[u / p.num_kv_heads];
         const int kvh = u - (u / p.num_kv_heads) * p.num_kv_heads;
-        int s = item.x;
+        int s_item = item.x;
         const int part = item.y;
         // A subgroup item (shared-prefix decode) serves M sequences that hold the
         // same physical blocks: one read of each K/V tile, M*G score columns
-        // (member i's query heads are columns i*G .. i*G+G-1).
-        int M = 1, mbase = 0;
+        // (member i's query heads are columns i*G .. i*G+G-1).  The claim that
+        // they hold the same blocks came from the caller: it is checked here for
+        // this item's blocks, and if any member's table differs the item runs
+        // once per member (M passes of one member each), as if ungrouped.
+        int M_item = 1, mbase_item = 0, npass = 1;
         if constexpr (GROUPED) {
-            if (s < 0) {
-                const int4 si = p.sub_info[-s - 1];
-                mbase = si.x;
-                M = si.y;
-                s = p.sub_members[mbase];
+            if (s_item < 0) {
+                const int4 si = p.sub_info[-s_item - 1];
+                mbase_item = si.x;
+                M_item = si.y;
+                s_item = p.sub_members[mbase_item];
+                const int32_t* t_first = p.block_tables + (size_t)s_item * p.max_blocks_per_seq + item.z;
+                bool same = true;
+                for (int j = lane; j < item.w; j += 32) {
+                    const int r = __ldg(t_first + j);
+#pragma unroll 4
+                    for (int mi = 1; mi < M_item; ++mi) {
+                        const int sm = p.sub_members[mbase_item + mi];
+                        same = (__ldg(p.block_tables + (size_t)sm * p.max_blocks_per_seq + item.z + j) == r) & same;
+                    }
+                }
+                if (!__all_sync(0xffffffffu, same)) npass = M_item;
             }
         }
+        for (int pass = 0; pass < npass; ++pass) {
+        const int M = npass > 1 ? 1 : M_item;
+        const int mbase = mbase_item + (npass > 1 ? pass : 0);
+        const int s = pass > 0 ? p.sub_members[mbase] : s_item;
         const int ncols = M * G;
         const int nt_act = GROUPED ? (ncols + 7) >> 3 : NT;  // n-tiles holding a column
         const int L = clamped_len(p, s, false);
@@ -610,6 +628,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
                     if (g == 0) p.part_ml[slot] = make_float2(m[nt][c], l[nt][c]);
                 }
             }
+        }  // pass
 #if PKV_DEBUG_TIMELINE
         ++dbg_units;
 #endif

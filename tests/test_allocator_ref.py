@@ -274,3 +274,154 @@ def test_prefix_groups_stop_at_first_different_block():
     bm.tables[b][2] = bm._pop()
     assert bm.prefix_groups([a, b, c]) == ([0, 3], [0, 1, 2], [2])
     assert bm.prefix_groups([a, c]) == ([0, 2], [0, 1], [4])
+
+
+# -- prefix caching across requests (full-block keys) --------------------------------
+
+def _cached_bm(nb=32):
+    bm = RefBlockManager(nb, 16)
+    bm.set_prefix_cache(True)
+    return bm
+
+
+SYS = list(range(1000, 1040))        # a 40-token system prompt: 2 full blocks + 8 tokens
+
+
+def test_same_system_prompt_reuses_full_blocks():
+    """Glossary entry: requests that start with the same system prompt share one
+    copy of it; hashing whole blocks extends sharing across requests."""
+    bm = _cached_bm()
+    a, ca = bm.alloc_seq_tokens(SYS + [1, 2, 3])
+    b, cb = bm.alloc_seq_tokens(SYS + [7, 8])
+    assert (ca, cb) == (0, 32)
+    assert bm.tables[a] == [0, 1, 2] and bm.tables[b] == [0, 1, 3]   # the 8-token tail is not shared
+    assert bm.ref[:4] == [2, 2, 1, 1]
+    c, cc = bm.alloc_seq_tokens(SYS[:16] + [5] * 30)                   # differs inside block 1
+    assert cc == 16 and bm.tables[c] == [0, 4, 5] and bm.ref[0] == 3
+    _check_invariants(bm)
+
+
+def test_a_block_is_keyed_by_its_whole_prefix():
+    """The same 16 tokens after a different first block are a different block."""
+    bm = _cached_bm()
+    x, y, z = [1] * 16, [2] * 16, [3] * 16
+    a, _ = bm.alloc_seq_tokens(x + y)
+    b, cb = bm.alloc_seq_tokens(z + y)
+    assert cb == 0 and set(bm.tables[a]).isdisjoint(bm.tables[b])
+    c, cc = bm.alloc_seq_tokens(x + y + z)
+    assert cc == 32 and bm.tables[c][:2] == bm.tables[a]
+
+
+def test_released_blocks_stay_cached_until_reused():
+    bm = _cached_bm(8)
+    a, _ = bm.alloc_seq_tokens(SYS)                      # blocks 0, 1, 2
+    bm.free_seq(a)
+    assert list(bm.free) == [3, 4, 5, 6, 7, 0, 1, 2]
+    b, cb = bm.alloc_seq_tokens(SYS[:32] + [9] * 4)      # hits 0, 1 out of the free list
+    assert cb == 32 and bm.tables[b] == [0, 1, 3]
+    assert list(bm.free) == [4, 5, 6, 7, 2]
+    bm.free_seq(b)
+    # a large request takes every free block, in order: the cached ones lose their keys
+    c = bm.alloc_seq(8 * 16)
+    assert bm.tables[c] == [4, 5, 6, 7, 2, 0, 1, 3] and not bm.cache
+    bm.free_seq(c)
+    d, cd = bm.alloc_seq_tokens(SYS)
+    assert cd == 0
+    _check_invariants(bm)
+
+
+def test_reused_parent_does_not_revive_stale_children():
+    """Block P held prompt A's first block, then was reused for prompt B's; a
+    prompt made of B's first block and A's second must not hit A's second block."""
+    bm = _cached_bm(4)
+    a0, a1, b0 = [1] * 16, [2] * 16, [3] * 16
+    a, _ = bm.alloc_seq_tokens(a0 + a1)                  # blocks 0 (a0), 1 (a1)
+    bm.free_seq(a)                                       # free list [2, 3, 0, 1], both cached
+    filler = bm.alloc_seq(32)                            # takes 2, 3
+    b, _ = bm.alloc_seq_tokens(b0)                       # takes 0: a0's key dropped, b0 registered
+    assert bm.tables[b] == [0]
+    c, cc = bm.alloc_seq_tokens(b0 + a1)
+    assert cc == 16 and bm.tables[c] == [0, 1]           # block 1 is not a hit ...
+    assert bm.ref[1] == 1                                # ... it was taken from the free list as new
+    bm.free_seq(filler)
+    _check_invariants(bm)
+
+
+def test_out_of_blocks_with_cache_changes_nothing():
+    bm = _cached_bm(4)
+    a, _ = bm.alloc_seq_tokens(SYS)                      # 0, 1, 2
+    bm.free_seq(a)
+    b = bm.alloc_seq(16)                                 # takes 3
+    state = (list(bm.free), list(bm.ref), dict(bm.cache))
+    with pytest.raises(MemoryError):
+        bm.alloc_seq_tokens(SYS + [0] * 9)               # 2 hits to wake + 2 new > 3 free
+    assert state == (list(bm.free), list(bm.ref), dict(bm.cache))
+    bm.free_seq(b)
+
+
+def test_prefix_cache_hits_hold_the_right_tokens():
+    """Requests over a few system prompts, released and reallocated at random;
+    each request writes only its uncached tokens, yet reading any live request
+    back through its table gives its whole logical token stream (content is a
+    function of (prefix, position), as a transformer's K/V is)."""
+    import oracle
+    rng = np.random.default_rng(8)
+    NB = 40
+    bm = _cached_bm(NB)
+    pool = np.full((NB, 16, 1, 4), -1.0, dtype=np.float32)
+    systems = [rng.integers(0, 9, size=n).tolist() for n in (37, 64, 20)]
+
+    def content(tokens):
+        # row of position i: (hash of the tokens up to i, i, token, 0)
+        h, rows = 0, []
+        for i, t in enumerate(tokens):
+            h = (h * 131 + t + 1) % 1000003
+            rows.append([h, i, t, 0])
+        return np.asarray(rows, dtype=np.float32).reshape(-1, 1, 4)
+
+    live = {}
+    for step in range(300):
+        if live and (rng.random() < 0.4 or bm.num_free() < 8):
+            s = list(live)[int(rng.integers(len(live)))]
+            bm.free_seq(s)
+            del live[s]
+            continue
+        toks = systems[int(rng.integers(3))] + rng.integers(0, 9, size=int(rng.integers(0, 30))).tolist()
+        try:
+            s, cached = bm.alloc_seq_tokens(toks)
+        except MemoryError:
+            continue
+        assert cached % 16 == 0 and cached <= len(toks)
+        rows = content(toks)
+        slots = bm.slots(s, cached, len(toks) - cached)
+        oracle.kv_write(rows[cached:], rows[cached:], oracle.F32, np.asarray(slots, np.int64), pool, pool.copy(),
+                        oracle.F32, 16)
+        live[s] = toks
+        for q, qt in live.items():
+            got = oracle.gather(pool, bm.tables[q], len(qt), 16)
+            assert np.array_equal(got, content(qt)), "request %d reads wrong tokens" % q
+    _check_invariants(bm)
+
+
+def test_evicted_prefix_is_not_served_from_overwritten_blocks():
+    """A cached prompt whose blocks were handed out for other data must miss:
+    reading it back gives its own tokens, written again."""
+    import oracle
+    bm = _cached_bm(6)
+    pool = np.zeros((6, 16, 1, 1), dtype=np.float32)
+
+    def put(tokens):
+        s, cached = bm.alloc_seq_tokens(tokens)
+        rows = np.asarray(tokens, dtype=np.float32).reshape(-1, 1, 1)
+        slots = np.asarray(bm.slots(s, cached, len(tokens) - cached), np.int64)
+        oracle.kv_write(rows[cached:], rows[cached:], oracle.F32, slots, pool, pool.copy(), oracle.F32, 16)
+        return s, cached
+
+    x = list(range(1, 49))                              # 3 full blocks
+    a, _ = put(x)
+    bm.free_seq(a)
+    other, _ = put([7] * 96)                            # takes all 6 blocks, x's included
+    bm.free_seq(other)
+    b, cached = put(x)
+    assert cached == 0
+    assert oracle.gather(pool, bm.tables[b], 48, 16).ravel().tolist() == x

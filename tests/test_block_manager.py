@@ -238,3 +238,53 @@ def test_prefix_groups_match_reference(BM, seed):
         offs, mem, sh = bm.prefix_groups(batch)
         r_offs, r_mem, r_sh = ref.prefix_groups(batch)
         assert (offs.tolist(), mem.tolist(), sh.tolist()) == (r_offs, r_mem, r_sh)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_prefix_cache_traces_match_reference(BM, seed):
+    """Prompts drawn from a few system prompts plus random user tokens, with
+    releases, forks and appends in between: same hits, tables, free list order
+    and cache size as the reference manager."""
+    from paged_kv_cache_404_b200 import PagedKVError
+    rng = np.random.default_rng(500 + seed)
+    NB = 220
+    order = rng.permutation(NB)
+    bm, ref = BM(NB, 16, free_order=order), RefBlockManager(NB, 16, free_order=order)
+    bm.set_prefix_cache(True)
+    ref.set_prefix_cache(True)
+    systems = [rng.integers(0, 50, size=int(rng.integers(10, 90))).tolist() for _ in range(4)]
+    live = []
+    for step in range(1500):
+        op = int(rng.integers(0, 10))
+        if op <= 3 or not live:
+            toks = systems[int(rng.integers(len(systems)))] + rng.integers(0, 3, size=int(rng.integers(0, 40))).tolist()
+            try:
+                exp = ref.alloc_seq_tokens(toks)
+            except MemoryError:
+                with pytest.raises(PagedKVError):
+                    bm.alloc_seq_tokens(toks)
+                continue
+            assert bm.alloc_seq_tokens(toks) == exp
+            live.append(exp[0])
+        elif op <= 5 and len(live) > 1:
+            s = live.pop(int(rng.integers(len(live))))
+            ref.free_seq(s)
+            bm.free_seq(s)
+        elif op == 6:
+            s = live[int(rng.integers(len(live)))]
+            r = ref.fork(s)
+            assert bm.fork(s) == r
+            live.append(r)
+        else:
+            s = live[int(rng.integers(len(live)))]
+            try:
+                exp = ref.append_token(s)
+            except MemoryError:
+                with pytest.raises(PagedKVError):
+                    bm.append_token(s)
+                continue
+            assert bm.append_token(s) == exp
+        if step % 100 == 0:
+            _same_state(bm, ref, live)
+            assert bm.num_cached_blocks() == len(ref.cache)
+    _same_state(bm, ref, live)

@@ -162,3 +162,71 @@ def test_fp8_cache_ignores_hints_and_equals_plain_decode():
     pkv.paged_attention_decode(plain, q, kp, vp, g_t, g_l, w.scale, max_len, ws2, ks, vs)
     torch.cuda.synchronize()
     assert torch.equal(out.view(torch.int16), plain.view(torch.int16))
+
+
+def test_prefix_cache_end_to_end():
+    """Requests over three system prompts: each request's prompt is allocated
+    through the prefix cache, only its uncached tokens are written, and the
+    grouped decode reads the shared blocks once.  Pools equal the oracle's
+    byte for byte (same managers' decisions on both sides), and the outputs
+    equal the oracle's attention over each request's whole logical stream."""
+    import paged_kv_cache_404_b200 as pkv
+    w = W.scaled(W.WORKLOADS["shared_prefix"], num_prompts=3)
+    rng = np.random.default_rng(77)
+    sys_lens = [300, 517, 64]
+    systems = [rng.integers(0, 30000, size=n).tolist() for n in sys_lens]
+    reqs = [(p, rng.integers(0, 30000, size=int(rng.integers(0, 200))).tolist()) for p in range(3) for _ in range(4)]
+    rng.shuffle(reqs)
+    NB = 400
+    order = W.free_order(w, NB)
+    bm, ref = pkv.BlockManager(NB, 16, free_order=order), oracle.RefBlockManager(NB, 16, free_order=order)
+    bm.set_prefix_cache(True)
+    ref.set_prefix_cache(True)
+    kp, vp = W.stale_fill(w, NB, "cuda")
+    hk, hv = to_np_bits(kp).copy(), to_np_bits(vp).copy()
+    # K/V of a system prompt's tokens are the same in every request that starts with it
+    sys_kv = [W.logical_kv(w, n, "cuda", stream=70 + p) for p, n in enumerate(sys_lens)]
+    ids, rids, logical = [], [], []
+    for r, (p, user) in enumerate(reqs):
+        toks = systems[p] + user
+        s, cached = bm.alloc_seq_tokens(toks)
+        rs, rcached = ref.alloc_seq_tokens(toks)
+        assert cached == rcached and bm.block_table(s).tolist() == ref.tables[rs]
+        uk, uv = W.logical_kv(w, len(user), "cuda", stream=100 + r)
+        k = torch.cat([sys_kv[p][0], uk]) if len(user) else sys_kv[p][0]
+        v = torch.cat([sys_kv[p][1], uv]) if len(user) else sys_kv[p][1]
+        n = len(toks)
+        if n > cached:
+            slots = bm.slots(s, cached, n - cached)
+            pkv.paged_kv_write(k[cached:].contiguous(), v[cached:].contiguous(), torch.from_numpy(slots).cuda(),
+                               kp, vp)
+            oracle.kv_write(to_np_bits(k[cached:]), to_np_bits(v[cached:]), oracle.BF16,
+                            np.asarray(ref.slots(rs, cached, n - cached), np.int64), hk, hv, oracle.BF16, 16)
+        ids.append(s)
+        rids.append(rs)
+        logical.append((to_np_bits(k), to_np_bits(v)))
+    torch.cuda.synchronize()
+    assert bm.num_cached_blocks() == len(ref.cache) > 0
+    assert np.array_equal(to_np_bits(kp), hk) and np.array_equal(to_np_bits(vp), hv)
+
+    lens = np.array([bm.seq_len(s) for s in ids], dtype=np.int32)
+    maxb = int(max(-(-int(L) // 16) for L in lens))
+    tabs, _ = bm.tables(ids, maxb, pad=-1)
+    offs, mem, sh = bm.prefix_groups(ids)
+    assert len(sh) == 3 and sorted(sh.tolist()) == sorted(n // 16 for n in sys_lens)
+    q = W.queries(w, len(ids), "cuda")
+    out, err, _ = _grouped(q, kp, vp, torch.from_numpy(tabs).cuda(), torch.from_numpy(lens).cuda(), w.scale,
+                           int(lens.max()), offs, mem, sh)
+    assert err == 0
+    # oracle: each request's whole logical K/V laid out contiguously in a pool of its own
+    for i, (k, v) in enumerate(logical):
+        n = k.shape[0]
+        nb = -(-n // 16)
+        ck = np.zeros((nb * 16,) + k.shape[1:], dtype=k.dtype)
+        cv = np.zeros_like(ck)
+        ck[:n], cv[:n] = k, v
+        ck, cv = ck.reshape((nb, 16) + k.shape[1:]), cv.reshape((nb, 16) + k.shape[1:])
+        ref_out, bad = oracle.paged_attention_decode(to_np_bits(q)[i:i + 1], oracle.BF16, ck, cv, oracle.BF16,
+                                                     np.arange(nb, dtype=np.int32)[None], lens[i:i + 1], w.scale)
+        assert bad == 0
+        assert_close(out_to_f64(out)[i:i + 1], ref_out, "bf16", "request %d" % i)

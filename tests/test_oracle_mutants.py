@@ -182,3 +182,41 @@ def test_pins_reject_swap_in_that_restores_old_block_ids(monkeypatch):
     monkeypatch.setattr(allocator.RefBlockManager, "swap_in", bad_swap_in)
     with pytest.raises(AssertionError):
         A.test_swap_round_trip_restores_every_token()
+
+
+def test_pins_reject_prefix_cache_keyed_by_tokens_only(monkeypatch):
+    """Planted mistake: a full block is keyed by its own 16 tokens only, not by
+    its prefix, so the same tokens after a different start alias one block."""
+    from oracle import allocator
+    real = allocator.RefBlockManager.alloc_seq_tokens
+
+    def bad(self, tokens):
+        saved = self._serial
+        seq, cached = real(self, tokens)
+        # re-key everything just registered without its parent
+        for b, key in list(self.key_of.items()):
+            if key[0] != 0:
+                blk, serial = self.cache.pop(key)
+                self.key_of[b] = (0, key[1])
+                self.cache[(0, key[1])] = (blk, serial)
+        return seq, cached
+
+    monkeypatch.setattr(allocator.RefBlockManager, "alloc_seq_tokens", bad)
+    with pytest.raises(AssertionError):
+        A.test_a_block_is_keyed_by_its_whole_prefix()
+
+
+def test_pins_reject_prefix_cache_that_keeps_keys_of_reused_blocks(monkeypatch):
+    """Planted mistake: a cached block handed out for new data keeps its key."""
+    from oracle import allocator
+
+    def bad_pop(self):
+        if not self.free:
+            raise MemoryError("no free block")
+        b = self.free.popleft()
+        self.ref[b] = 1
+        return b
+
+    monkeypatch.setattr(allocator.RefBlockManager, "_pop", bad_pop)
+    with pytest.raises(AssertionError):
+        A.test_evicted_prefix_is_not_served_from_overwritten_blocks()
