@@ -57,6 +57,10 @@ def lib():
         L.orc_paged_attention_decode.argtypes = [p, p, C.c_int, p, p, C.c_int, p, C.c_int, p, C.c_int,
                                                  C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
                                                  C.c_double, C.c_double, C.c_double, C.c_int, C.c_int]
+        L.orc_paged_attention_prefill.restype = C.c_int
+        L.orc_paged_attention_prefill.argtypes = [p, p, C.c_int, p, p, C.c_int, p, C.c_int, p, p, C.c_int,
+                                                  C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_double,
+                                                  C.c_double, C.c_double, p, C.c_int]
         L.orc_kv_cache_bytes.restype = C.c_double
         L.orc_kv_cache_bytes.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.c_double]
         L.orc_max_threads.restype = C.c_int
@@ -178,6 +182,39 @@ def paged_attention_decode(q, q_dtype, k_pool, v_pool, cache_dtype, block_tables
                                          int(partition_tokens), int(num_threads))
     if r < 0:
         raise ValueError("bad arguments to the oracle decode")
+    return out, r
+
+
+def paged_attention_prefill(q, q_dtype, k_pool, v_pool, cache_dtype, block_tables, context_lens, query_start,
+                            scale, k_scale=1.0, v_scale=1.0, rows=None, num_threads=0):
+    """fp64 causal multi-token attention through block tables.
+
+    q: [total_q, Hq, D]; query_start int32 [S + 1]; sequence s's queries are the
+    last (query_start[s+1] - query_start[s]) of its context_lens[s] tokens.
+    rows: optional iterable of query rows to compute (others stay 0).
+    Returns (out float64 [total_q, Hq, D], bad_entries).
+    """
+    q = _c(q)
+    kp = _c(k_pool)
+    vp = _c(v_pool)
+    bt = _c(block_tables, np.int32)
+    cl = _c(context_lens, np.int32)
+    qs = _c(query_start, np.int32)
+    T, Hq, D = q.shape
+    NB, bs, Hkv, D2 = kp.shape
+    S = cl.shape[0]
+    assert D2 == D and bt.shape[0] == S and qs.shape[0] == S + 1 and qs[-1] == T
+    mask = None
+    if rows is not None:
+        mask = np.zeros(T, dtype=np.uint8)
+        mask[np.asarray(list(rows), dtype=np.int64)] = 1
+    out = np.zeros((T, Hq, D), dtype=np.float64)
+    r = lib().orc_paged_attention_prefill(_ptr(out), _ptr(q), q_dtype, _ptr(kp), _ptr(vp), cache_dtype, _ptr(bt),
+                                          bt.shape[1], _ptr(cl), _ptr(qs), S, NB, bs, Hq, Hkv, D, float(scale),
+                                          float(k_scale), float(v_scale), _ptr(mask) if mask is not None else None,
+                                          int(num_threads))
+    if r < 0:
+        raise ValueError("bad arguments to the oracle prefill")
     return out, r
 
 

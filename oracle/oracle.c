@@ -411,6 +411,68 @@ int orc_paged_attention_decode(double* out, const void* q, int q_dtype, const vo
     return bad;
 }
 
+/* Causal multi-token attention through block tables (the prompt pass: the
+ * prompt's blocks are allocated first and then filled, and attention reads
+ * them through the table in logical order, iplexlaw.co.kr, section on logical
+ * vs physical order; every token attends to all the tokens before it,
+ * gyaansetu.com, KV-cache definition).
+ * Sequence s has nq = query_start[s+1] - query_start[s] new tokens: the last
+ * nq of its context_lens[s] tokens, whose K/V are already in the pools.  Query
+ * row r = query_start[s] + i is at position p = context_lens[s] - nq + i and
+ * attends to tokens t <= p, exactly as a single-query decode over p + 1
+ * tokens would.
+ *   out [total_q][num_heads][head_dim] (double); q [total_q][num_heads][head_dim]
+ *   row_mask: NULL, or uint8 [total_q]: rows with 0 are skipped (left 0)
+ * Returns the number of out-of-range table entries among each sequence's
+ * first context_lens[s] tokens, or -1 for bad arguments (nq > context). */
+int orc_paged_attention_prefill(double* out, const void* q, int q_dtype, const void* k_pool,
+                                const void* v_pool, int cache_dtype, const int32_t* block_tables,
+                                int max_blocks_per_seq, const int32_t* context_lens,
+                                const int32_t* query_start, int num_seqs, int num_blocks, int block_size,
+                                int num_heads, int num_kv_heads, int head_dim, double scale,
+                                double k_scale, double v_scale, const uint8_t* row_mask, int num_threads) {
+    int bad = 0, s, group, total;
+    long long pair;
+    if (num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0 || head_dim <= 0 ||
+        block_size <= 0 || num_seqs < 0 || query_start[0] != 0)
+        return -1;
+    group = num_heads / num_kv_heads;
+    for (s = 0; s < num_seqs; s++) {
+        int L = context_lens[s], nq = query_start[s + 1] - query_start[s], j;
+        if (nq < 0 || nq > L || L > max_blocks_per_seq * block_size) return -1;
+        for (j = 0; j < (L + block_size - 1) / block_size; j++) {
+            int32_t b = block_tables[(size_t)s * max_blocks_per_seq + j];
+            if (b < 0 || b >= num_blocks) bad++;
+        }
+    }
+    total = query_start[num_seqs];
+#ifdef _OPENMP
+    if (num_threads > 0) omp_set_num_threads(num_threads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (pair = 0; pair < (long long)total * num_heads; pair++) {
+        int r = (int)(pair / num_heads), h = (int)(pair % num_heads);
+        int s2 = 0, d, pos;
+        double m, l;
+        double* o = out + ((size_t)r * num_heads + h) * head_dim;
+        double* qv;
+        double* scores;
+        if (row_mask != NULL && !row_mask[r]) continue;
+        while (query_start[s2 + 1] <= r) s2++;  /* the sequence holding row r */
+        pos = context_lens[s2] - (query_start[s2 + 1] - query_start[s2]) + (r - query_start[s2]);
+        qv = (double*)malloc(sizeof(double) * head_dim);
+        scores = (double*)malloc(sizeof(double) * (pos + 1));
+        for (d = 0; d < head_dim; d++) qv[d] = load_elem(q, q_dtype, ((size_t)r * num_heads + h) * head_dim + d);
+        if (attend_range(qv, k_pool, v_pool, cache_dtype, block_tables + (size_t)s2 * max_blocks_per_seq, 0,
+                         pos + 1, block_size, num_blocks, num_kv_heads, h / group, head_dim, scale, k_scale,
+                         v_scale, scores, &m, &l, o) == 0)
+            for (d = 0; d < head_dim; d++) o[d] = 0.0;
+        free(qv);
+        free(scores);
+    }
+    return bad;
+}
+
 /* Size in bytes of a KV cache: 2 (K and V) * layers * kv heads * head_dim *
  * element bytes per token, times the number of tokens. */
 double orc_kv_cache_bytes(int layers, int num_kv_heads, int head_dim, int elem_bytes, double tokens) {

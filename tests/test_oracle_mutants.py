@@ -40,6 +40,16 @@ MUTANTS = {
     "swap_accepts_repeated_dst": ("for (j = i + 1; j < num_pairs; j++)", "for (j = num_pairs; j < num_pairs; j++)"),
     "swap_half_block": ("(const char*)src_k + (size_t)s * block_bytes, block_bytes);",
                         "(const char*)src_k + (size_t)s * block_bytes, block_bytes / 2);"),
+    "prefill_excludes_itself": ("pos + 1, block_size, num_blocks, num_kv_heads, h / group,",
+                                "pos, block_size, num_blocks, num_kv_heads, h / group,"),
+    "prefill_position_ignores_prefix": ("pos = context_lens[s2] - (query_start[s2 + 1] - query_start[s2]) + (r - query_start[s2]);",
+                                        "pos = (r - query_start[s2]);"),
+    "prefill_attends_past_itself": [
+        ("scores = (double*)malloc(sizeof(double) * (pos + 1));", "scores = (double*)malloc(sizeof(double) * (pos + 2));"),
+        ("pos + 1, block_size, num_blocks, num_kv_heads, h / group,",
+         "(pos + 2 <= context_lens[s2] ? pos + 2 : pos + 1), block_size, num_blocks, num_kv_heads, h / group,")],
+    "prefill_head_mapping": ("pos + 1, block_size, num_blocks, num_kv_heads, h / group,",
+                             "pos + 1, block_size, num_blocks, num_kv_heads, h % num_kv_heads,"),
     "gather_wrong_slot": ("((size_t)blk * block_size + (size_t)(t % block_size)) * row_bytes, row_bytes);",
                           "((size_t)blk * block_size + (size_t)(t / block_size)) * row_bytes, row_bytes);"),
 }
@@ -62,16 +72,21 @@ def _pins(golden):
         P.test_kv_write_bf16_is_raw_copy_and_touches_nothing_else,
         P.test_kv_write_fp8_matches_library_cast, P.test_copy_blocks_semantics,
         P.test_swap_blocks_between_pools_of_different_sizes,
+        lambda: [P.test_prefill_equals_numpy_causal_attention(*a) for a in [(2, 2), (8, 2)]],
+        P.test_prefill_first_position_returns_v0, P.test_prefill_bf16_and_row_subset,
     ]
     return fns
 
 
-def _build_mutant(tmp, name, old, new):
+def _build_mutant(tmp, name, edits):
+    """edits: one (old, new) pair or a list of them, applied to the oracle's source."""
     src = open(SRC).read()
-    assert src.count(old) >= 1, "mutation anchor not found: %s" % name
+    for old, new in ([edits] if isinstance(edits, tuple) else edits):
+        assert src.count(old) >= 1, "mutation anchor not found: %s" % name
+        src = src.replace(old, new)
     path_c = os.path.join(tmp, name + ".c")
     path_so = os.path.join(tmp, name + ".so")
-    open(path_c, "w").write(src.replace(old, new))
+    open(path_c, "w").write(src)
     subprocess.run(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
                     path_c, "-o", path_so, "-lm"], check=True)
     return path_so
@@ -92,8 +107,7 @@ def _load_like_oracle(path):
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_pins_reject_planted_mistake(name, golden_dir, tmp_path):
-    old, new = MUTANTS[name]
-    path = _build_mutant(str(tmp_path), name, old, new)
+    path = _build_mutant(str(tmp_path), name, MUTANTS[name])
     mutant = _load_like_oracle(path)
     saved = oracle._lib
     oracle._lib = mutant

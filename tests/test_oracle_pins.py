@@ -468,3 +468,84 @@ def test_swap_blocks_between_pools_of_different_sizes():
     # the same src twice is fine (two copies of one page)
     assert oracle.swap_blocks(hk, hv, dk, dv, [[2, 4], [2, 5]]) == 0
     assert np.array_equal(hk[4], dk[2]) and np.array_equal(hk[5], dk[2])
+
+
+# ------------------------------------------------------------------ causal prefill
+
+def _prefill_case(seed, lens, nqs, Hq, Hkv, D, dtype=np.float32):
+    """Scattered pools and tables from the reference manager; q rows per sequence."""
+    rng = np.random.default_rng(seed)
+    NB = sum(-(-L // 16) for L in lens) + 7
+    bm = RefBlockManager(NB, 16, free_order=rng.permutation(NB))
+    ids = [bm.alloc_seq(L) for L in lens]
+    maxb = max(-(-L // 16) for L in lens)
+    tabs = np.full((len(lens), maxb), -1, np.int32)
+    for i, s in enumerate(ids):
+        tabs[i, :len(bm.tables[s])] = bm.tables[s]
+    kp = rng.standard_normal((NB, 16, Hkv, D)).astype(dtype)
+    vp = rng.standard_normal((NB, 16, Hkv, D)).astype(dtype)
+    qs = np.concatenate([[0], np.cumsum(nqs)]).astype(np.int32)
+    q = rng.standard_normal((int(qs[-1]), Hq, D)).astype(dtype)
+    return q, kp, vp, tabs, np.asarray(lens, np.int32), qs
+
+
+def _numpy_causal(q, kp, vp, tabs, lens, qs, scale):
+    """Brute force: gather each sequence's logical K/V with numpy indexing, mask
+    keys after the query's position, library softmax."""
+    T, Hq, D = q.shape
+    Hkv = kp.shape[2]
+    G = Hq // Hkv
+    out = np.zeros((T, Hq, D))
+    for s in range(len(lens)):
+        L = int(lens[s])
+        t = np.arange(L)
+        K = kp[tabs[s][t // 16], t % 16].astype(np.float64)       # [L, Hkv, D]
+        V = vp[tabs[s][t // 16], t % 16].astype(np.float64)
+        nq = int(qs[s + 1] - qs[s])
+        for i in range(nq):
+            r = int(qs[s]) + i
+            pos = L - nq + i
+            for h in range(Hq):
+                sc = scale * (K[:pos + 1, h // G] @ q[r, h].astype(np.float64))
+                out[r, h] = sp_softmax(sc) @ V[:pos + 1, h // G]
+    return out
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(2, 2), (8, 2)])
+def test_prefill_equals_numpy_causal_attention(Hq, Hkv):
+    # a whole prompt (37 tokens), a prompt after a 15-token cached prefix, a 1-token step
+    q, kp, vp, tabs, lens, qs = _prefill_case(31, [37, 20, 16], [37, 5, 1], Hq, Hkv, 32)
+    got, bad = oracle.paged_attention_prefill(q, oracle.F32, kp, vp, oracle.F32, tabs, lens, qs, 0.3)
+    assert bad == 0
+    np.testing.assert_allclose(got, _numpy_causal(q, kp, vp, tabs, lens, qs, 0.3), rtol=1e-12, atol=1e-12)
+
+
+def test_prefill_first_position_returns_v0():
+    q, kp, vp, tabs, lens, qs = _prefill_case(32, [40], [40], 4, 2, 16)
+    got, _ = oracle.paged_attention_prefill(q, oracle.F32, kp, vp, oracle.F32, tabs, lens, qs, 0.5)
+    b0 = tabs[0][0]
+    for h in range(4):
+        assert np.array_equal(got[0, h], kp.dtype.type(1) * vp[b0, 0, h // 2].astype(np.float64))
+
+
+def test_prefill_row_equals_decode_of_its_prefix():
+    """Row i of a prompt is the decode of the first pos + 1 tokens."""
+    q, kp, vp, tabs, lens, qs = _prefill_case(33, [50], [12], 4, 4, 16)
+    got, _ = oracle.paged_attention_prefill(q, oracle.F32, kp, vp, oracle.F32, tabs, lens, qs, 0.25)
+    for i in range(12):
+        pos = 50 - 12 + i
+        dec, _ = oracle.paged_attention_decode(q[i:i + 1], oracle.F32, kp, vp, oracle.F32, tabs,
+                                               np.array([pos + 1], np.int32), 0.25)
+        np.testing.assert_allclose(got[i], dec[0], rtol=1e-13, atol=1e-13)
+
+
+def test_prefill_bf16_and_row_subset():
+    q, kp, vp, tabs, lens, qs = _prefill_case(34, [33, 70], [33, 40], 4, 2, 32)
+    bits = lambda a: torch.from_numpy(a).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)  # noqa: E731
+    qb, kb, vb = bits(q), bits(kp), bits(vp)
+    full, _ = oracle.paged_attention_prefill(qb, oracle.BF16, kb, vb, oracle.BF16, tabs, lens, qs, 0.2)
+    ref = _numpy_causal(oracle.bf16_to_f64(qb), oracle.bf16_to_f64(kb), oracle.bf16_to_f64(vb), tabs, lens, qs, 0.2)
+    np.testing.assert_allclose(full, ref, rtol=1e-12, atol=1e-12)
+    part, _ = oracle.paged_attention_prefill(qb, oracle.BF16, kb, vb, oracle.BF16, tabs, lens, qs, 0.2,
+                                             rows=[0, 32, 50])
+    assert np.array_equal(part[[0, 32, 50]], full[[0, 32, 50]]) and not part[1].any()
