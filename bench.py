@@ -21,6 +21,12 @@ the max over ranks and the value the sum over ranks (weak scaling).
 --impl reference times the CPU oracle (the plain fp64 reference) on a bounded
 sample of the same workload, on this host's cores.
 
+--workload prefill70b measures the prompt pass instead (a separate line): 16
+prompts of 512..4,096 tokens (Llama-3.1-70B shape) written into blocks with the
+multi-token KV write, then causal paged attention over them; metric TFLOP/s of
+the causal attention (4 * Hq * D * sum over query rows of keys attended),
+roofline against the measured dense bf16 tensor peak.
+
 --swap measures block swap instead (a separate line, not the headline): a
 quarter of the gqa70b batch (64 sequences x 4,096 tokens, 1 GiB of K+V) moves
 from scattered device blocks to a page-locked host pool and back through
@@ -56,6 +62,8 @@ DESCR = {
     "shared_prefix": "shared-prefix parallel sampling: 64 prompts x n=3, 1000-token prefix + U{0..512}, GQA 32/8, "
                      "head_dim 128, bf16, copy-on-write + write + decode per step",
     "fp8_long": "FP8 E4M3 cache, GQA 32/8, head_dim 128, 128 seqs, lengths log-U[256, 32768], write + split decode",
+    "prefill70b": "prompt pass, Llama-3.1-70B shape: 64 q / 8 kv heads, head_dim 128, bf16, 16 prompts of "
+                  "U[512, 4096] tokens: multi-token KV write + causal paged attention",
 }
 
 
@@ -454,6 +462,20 @@ def run_reference(args, w, rank, world):
     if rank != 0:
         return
     import oracle
+    if w.name == "prefill70b":
+        t0 = time.perf_counter()
+        samples = [prefill_cpu_baseline(w, target_s=2.0) for _ in range(args.steps)]
+        total = time.perf_counter() - t0
+        value = statistics.mean(x["value"] for x in samples)
+        line = {"metric": "causal paged prefill attention TFLOP/s (4*Hq*D*keys attended per query row)",
+                "value": value, "unit": "TFLOP/s", "impl": "reference", "n_gpus": world, "steps": args.steps,
+                "warmup": 0, "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": "prefill70b: " + DESCR["prefill70b"], "parallelism": "cpu (OpenMP)"},
+                "cpu_baseline": dict(samples[-1], value=value),
+                "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
     elem = 1 if w.cache_dtype == "fp8" else 2
     per_tok = w.num_kv_heads * w.head_dim * 2 * elem
     # size one step's sample to about 3 s of CPU work
@@ -488,6 +510,174 @@ def run_reference(args, w, rank, world):
 
 
 # ------------------------------------------------------------------ main
+
+def measured_peak_tensor():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (cuBLAS bf16 burst)"
+    except Exception:  # noqa: BLE001
+        return 1590.0, "fallback"
+
+
+class PrefillStep:
+    """Device-resident inputs of one prompt pass: every prompt token's K/V written
+    at its slot, then causal attention of every prompt token."""
+
+    def __init__(self, w, device):
+        import paged_kv_cache_404_b200 as pkv
+        self.pkv, self.w, self.device = pkv, w, device
+        lens = W.context_lens(w)
+        self.S = len(lens)
+        need = int(sum(-(-int(L) // 16) for L in lens))
+        NB = W.pool_blocks(w, need)
+        bm = pkv.BlockManager(NB, 16, free_order=W.free_order(w, NB))
+        ids = [bm.alloc_seq(int(L)) for L in lens]
+        self.total = int(lens.astype(np.int64).sum())
+        slots = np.concatenate([bm.slots(s, 0, int(L)) for s, L in zip(ids, lens)])
+        tables, self.lens = bm.tables(ids, max(-(-int(L) // 16) for L in lens), pad=-1)
+        self.k_pool, self.v_pool = W.stale_fill(w, NB, device)
+        self.k_new, self.v_new = W.logical_kv(w, self.total, device, stream=80)
+        self.q = W.queries(W.scaled(w, num_seqs=self.total), self.total, device)
+        self.out = torch.empty_like(self.q)
+        self.g_slots = torch.from_numpy(slots.astype(np.int64)).to(device)
+        self.g_tables = torch.from_numpy(tables).to(device)
+        self.g_lens = torch.from_numpy(self.lens).to(device)
+        self.g_qs = torch.from_numpy(np.concatenate([[0], np.cumsum(self.lens)]).astype(np.int32)).to(device)
+        self.max_q = int(self.lens.max())
+        self.err = torch.zeros(1, dtype=torch.int32, device=device)
+        L64 = self.lens.astype(np.float64)
+        self.flops = 4.0 * w.num_heads * w.head_dim * float((L64 * (L64 + 1) / 2).sum())
+        self.kv_bytes = self.total * w.num_kv_heads * w.head_dim * 2 * 2
+
+    def write(self):
+        self.pkv.paged_kv_write(self.k_new, self.v_new, self.g_slots, self.k_pool, self.v_pool, err_count=self.err)
+
+    def attend(self):
+        self.pkv.paged_attention_prefill(self.out, self.q, self.k_pool, self.v_pool, self.g_tables, self.g_lens,
+                                         self.g_qs, self.w.scale, self.max_q, err_count=self.err)
+
+
+def prefill_cpu_baseline(w, target_s=12.0):
+    """The oracle's causal attention on a bounded sample of query rows."""
+    import oracle
+    rng = np.random.default_rng(7)
+    lens = W.context_lens(w)
+    L = int(lens[0])
+    NB = -(-L // 16)
+    tabs = np.arange(NB, dtype=np.int32)[None]
+    g = torch.Generator().manual_seed(1234)
+    kp = torch.randn((NB, 16, w.num_kv_heads, w.head_dim), generator=g).to(torch.bfloat16)
+    vp = torch.randn((NB, 16, w.num_kv_heads, w.head_dim), generator=g).to(torch.bfloat16)
+    q = torch.randn((L, w.num_heads, w.head_dim), generator=g).to(torch.bfloat16)
+    bits = lambda t: t.view(torch.int16).numpy().view(np.uint16)  # noqa: E731
+    qs = np.array([0, L], np.int32)
+
+    def run(rows):
+        t0 = time.perf_counter()
+        oracle.paged_attention_prefill(bits(q), oracle.BF16, bits(kp), bits(vp), oracle.BF16, tabs,
+                                       np.array([L], np.int32), qs, w.scale, rows=rows)
+        return time.perf_counter() - t0
+
+    rows = np.sort(rng.choice(L, 4, replace=False))
+    dt = run(rows)
+    n = int(max(4, min(L, 4 * target_s / max(dt, 1e-3))))
+    rows = np.sort(rng.choice(L, n, replace=False))
+    dt = run(rows)
+    flops = 4.0 * w.num_heads * w.head_dim * float((rows + 1).sum())
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": "%d query rows of a %d-token prompt (all 64 heads), fp64, %.2f s" % (n, L, dt)}
+
+
+def run_prefill(args, device, rank, world):
+    w = rank_workload(W.WORKLOADS["prefill70b"], rank)
+    step = PrefillStep(w, device)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        step.write()
+        step.attend()
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    with ClockSampler(device) as clk:
+        a0 = torch.cuda.Event(enable_timing=True)
+        z0 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for a, b, c in ev:
+            a.record(stream)
+            step.write()
+            b.record(stream)
+            step.attend()
+            c.record(stream)
+        z0.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    total_ms = reduce_max(a0.elapsed_time(z0), world, device)
+    att_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
+    wr_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
+    value = step.flops * world * args.steps / (total_ms / 1e3) / 1e12
+
+    e2e = None
+    if not args.no_e2e:
+        # through the public API from pinned host buffers: inputs up, output down, every step
+        names = ["q", "k_new", "v_new", "g_slots", "g_tables", "g_lens", "g_qs"]
+        host = {n: getattr(step, n).cpu().pin_memory() for n in names}
+        out_host = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = out_host.numel() * out_host.element_size()
+        n_e = max(3, args.steps // 4)
+
+        def e2e_step():
+            for n in names:
+                getattr(step, n).copy_(host[n], non_blocking=True)
+            step.write()
+            step.attend()
+            out_host.copy_(step.out, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e):
+            e2e_step()
+        z.record(stream)
+        torch.cuda.synchronize()
+        e_ms = reduce_max(a.elapsed_time(z), world, device)
+        e2e = {"value": round(step.flops * world * n_e / (e_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms / n_e, 4)}
+
+    peak, peak_kind = measured_peak_tensor()
+    achieved = step.flops / (att_ms / 1e3) / 1e12
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = prefill_cpu_baseline(w)
+        line = {
+            "metric": "causal paged prefill attention TFLOP/s (4*Hq*D*keys attended per query row)",
+            "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16 (fp32 accumulate)",
+            "data": "synthetic (seeded N(0,1) q/K/V, seeded block placement)",
+            "config": {"workload": "prefill70b: " + DESCR["prefill70b"], "global_batch": step.S * world,
+                       "seq_len": step.max_q, "prompt_tokens": step.total,
+                       "parallelism": "replicas: prompts sharded by rank, no collective",
+                       "l2": "inputs larger than L2 (q %.0f MB + K/V %.0f MB per GPU vs 126 MB L2)" % (
+                           step.q.numel() * 2 / 1e6, 2 * step.k_pool.numel() * 2 / 1e6)},
+            "prompt_tokens_per_s": round(step.total * world * args.steps / (total_ms / 1e3), 1),
+            "us_attention": round(1e3 * att_ms, 2), "us_write": round(1e3 * wr_ms, 2),
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(achieved / peak, 4), "traffic": None,
+                         "kernel": "prefill_kernel (mma.sync m16n8k16 bf16)", "peak_source": peak_kind},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps, "device_errors": int(step.err.item()),
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+
 
 def run_swap(args, device):
     """Swap-out and swap-in throughput of pkv_swap_blocks over the host link."""
@@ -599,6 +789,20 @@ def main(argv=None):
     torch.cuda.set_device(local)
     if args.swap:
         run_swap(args, torch.device("cuda", local))
+        return
+    if args.workload == "prefill70b":
+        if world > 1:
+            import datetime
+            import torch.distributed as dist
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+            dist.barrier()
+            pkv_build.build()
+        run_prefill(args, torch.device("cuda", local), rank, world)
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
         return
     device = torch.device("cuda", local)
     if world > 1:

@@ -252,6 +252,36 @@ int pkv_paged_attention_decode_shared(void* out, const void* q, int q_dtype,
                                       int32_t* err_count, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Causal multi-token attention (the prompt pass) through block tables.
+ * Source: a prompt's blocks are allocated first and its last block then
+ * filled; attention reads the blocks through the table in logical order
+ * (iplexlaw.co.kr, section on logical vs physical order); each token attends
+ * to all the tokens before it (gyaansetu.com, what the KV cache holds).
+ *
+ * Sequence s has nq_s = query_start[s+1] - query_start[s] new query tokens:
+ * the last nq_s of its context_lens[s] tokens, whose K/V are already in the
+ * pools (pkv_paged_kv_write with the prompt's slots).  Query row
+ * r = query_start[s] + i sits at position context_lens[s] - nq_s + i and
+ * attends to tokens 0 .. that position.  A whole prompt, a prompt after a
+ * cached prefix and a chunk of a long prompt are all this call.
+ *   out, q          [total_q][num_heads][head_dim], total_q = query_start[num_seqs]
+ *   block_tables    int32 [num_seqs][max_blocks_per_seq]
+ *   context_lens    int32 [num_seqs]; query_start int32 [num_seqs + 1], query_start[0] = 0
+ *   max_query_len   >= every nq_s (sizes the launch; rows past it are not computed)
+ * Supported: bf16 q, bf16 cache, head_dim 128, block_size 16, any GQA group.
+ * Device-data errors (a table entry out of range among the blocks a sequence
+ * reads: its tokens are left out; nq_s > context_lens[s] or a context longer
+ * than the table: the sequence's rows are zeroed) are counted into err_count.
+ * ---------------------------------------------------------------------- */
+int pkv_paged_attention_prefill(void* out, const void* q, int q_dtype,
+                                const void* k_pool, const void* v_pool, int cache_dtype,
+                                const int32_t* block_tables, int max_blocks_per_seq,
+                                const int32_t* context_lens, const int32_t* query_start, int num_seqs,
+                                int max_query_len, int num_blocks, int block_size, int num_heads,
+                                int num_kv_heads, int head_dim, float scale,
+                                int32_t* err_count, void* stream);
+
+/* ------------------------------------------------------------------------
  * Copy-on-write block copy: for every pair (src, dst) copy the whole physical
  * block src over block dst, in both pools.
  * Source: before a sequence writes into a block that other sequences still

@@ -15,6 +15,7 @@ from .ops import (  # noqa: F401
     decode_workspace_bytes_shared,
     paged_attention_decode,
     paged_attention_decode_shared,
+    paged_attention_prefill,
     paged_attention_decode_noalloc,
     paged_kv_write,
     swap_blocks,

@@ -21,6 +21,8 @@ cudaError_t launch_decode_f32(const DecodeParams& p, int num_sms, cudaStream_t s
 int decode_tc_warps(bool fp8, int head_dim, bool grouped);
 bool decode_tc_groupable(bool fp8, int head_dim, int group);
 cudaError_t launch_decode_merge(const DecodeParams& p, int out_dtype, cudaStream_t stream);
+cudaError_t launch_prefill(const CUtensorMap& tmK, const CUtensorMap& tmV, const PrefillParams& p, int max_query_len,
+                           cudaStream_t stream);
 }  // namespace pkv
 
 using namespace pkv;
@@ -315,6 +317,45 @@ int decode_impl(void* out, const void* q, int q_dtype, const void* k_pool, const
 }  // namespace
 
 extern "C" {
+
+int pkv_paged_attention_prefill(void* out, const void* q, int q_dtype, const void* k_pool, const void* v_pool,
+                                int cache_dtype, const int32_t* block_tables, int max_blocks_per_seq,
+                                const int32_t* context_lens, const int32_t* query_start, int num_seqs,
+                                int max_query_len, int num_blocks, int block_size, int num_heads, int num_kv_heads,
+                                int head_dim, float scale, int32_t* err_count, void* stream) {
+    if (num_seqs < 0 || max_blocks_per_seq <= 0 || max_query_len < 0 || num_blocks <= 0 || block_size <= 0 ||
+        num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0)
+        return PKV_EINVAL;
+    if (num_heads % num_kv_heads != 0) return PKV_EINVAL;
+    if (block_size != kBlockSize) return PKV_EUNSUPPORTED;
+    if (q_dtype != PKV_BF16 || cache_dtype != PKV_BF16 || head_dim != 128) return PKV_EUNSUPPORTED;
+    if (num_seqs == 0 || max_query_len == 0) return PKV_OK;
+    if (num_seqs > 65535 || num_heads > 65535) return PKV_EUNSUPPORTED;
+    if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens || !query_start) return PKV_EINVAL;
+    if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) ||
+        !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(query_start, 4) || !aligned(err_count, 4))
+        return PKV_EINVAL;
+    PrefillParams p;
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.query_start = query_start;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_seqs = num_seqs;
+    p.num_blocks = num_blocks;
+    p.num_heads = num_heads;
+    p.group = num_heads / num_kv_heads;
+    p.score_scale = scale * 1.4426950408889634f;
+    p.err = err_count;
+    CUtensorMap tmK, tmV;
+    const long long slots = (long long)num_blocks * block_size;
+    if (!pool_tensor_map(&tmK, k_pool, cache_dtype, head_dim, num_kv_heads, slots) ||
+        !pool_tensor_map(&tmV, v_pool, cache_dtype, head_dim, num_kv_heads, slots))
+        return PKV_ECUDA;
+    cudaError_t e = launch_prefill(tmK, tmV, p, max_query_len, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PKV_OK : PKV_ECUDA;
+}
 
 int pkv_copy_blocks(void* k_pool, void* v_pool, size_t block_bytes, const int64_t* src_dst_pairs, int num_pairs,
                     int num_blocks, int32_t* err_count, void* stream) {

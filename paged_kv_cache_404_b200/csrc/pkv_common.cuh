@@ -126,6 +126,22 @@ struct DecodeParams {
     int* sub_members;
 };
 
+// Everything the prefill kernel needs besides the tensor maps.
+struct PrefillParams {
+    __nv_bfloat16* out;
+    const __nv_bfloat16* q;
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    const int32_t* query_start;
+    int max_blocks_per_seq;
+    int num_seqs;
+    int num_blocks;
+    int num_heads;
+    int group;
+    float score_scale;  // scale * log2(e)
+    int32_t* err;
+};
+
 // ------------------------------------------------------------------ small helpers
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -183,6 +199,10 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {

@@ -125,6 +125,28 @@ def paged_attention_decode_shared(out, q, k_pool, v_pool, block_tables, context_
     return out
 
 
+def paged_attention_prefill(out, q, k_pool, v_pool, block_tables, context_lens, query_start, scale, max_query_len,
+                            err_count=None, stream=None):
+    """Causal attention of each sequence's new tokens (the last nq of its context)
+    over its whole context; q/out [total_q, Hq, D], query_start int32 [S + 1]."""
+    T, Hq, D = q.shape
+    NB, bs, Hkv, D2 = k_pool.shape
+    S = int(context_lens.numel())
+    if D2 != D or out.shape != q.shape:
+        raise ValueError("shape mismatch")
+    for t in (block_tables, context_lens, query_start):
+        if t.dtype != torch.int32:
+            raise TypeError("tables, lengths and query_start must be int32")
+    if query_start.numel() != S + 1:
+        raise ValueError("query_start must have num_seqs + 1 entries")
+    st = L.lib().pkv_paged_attention_prefill(
+        _ptr(out), _ptr(q), _dtype_code(q), _ptr(k_pool), _ptr(v_pool), _dtype_code(k_pool), _ptr(block_tables),
+        int(block_tables.shape[1]), _ptr(context_lens), _ptr(query_start), S, int(max_query_len), NB, bs, Hq, Hkv,
+        D, float(scale), _ptr(err_count), _stream(stream))
+    L.check("pkv_paged_attention_prefill", st)
+    return out
+
+
 def paged_attention_decode_noalloc(out, q, k_pool, v_pool, block_tables, context_lens, scale, max_context_len,
                                    k_scale=1.0, v_scale=1.0, partition_tokens=0, err_count=None, stream=None):
     """paged_attention_decode for callers that cannot allocate: no workspace argument;

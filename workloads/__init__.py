@@ -15,6 +15,8 @@ Workloads are shaped like the PagedAttention pages' examples:
 - "shared_prefix": parallel sampling n=3 over 64 prompts sharing a 1,000-token
   prefix, continuations of 0..512 tokens.
 - "fp8_long": FP8 E4M3 cache, log-uniform context lengths 256..32,768.
+- "prefill70b": the prompt pass of the Llama-3.1-70B shape: 16 prompts of
+  512..4,096 tokens written into blocks and attended causally.
 """
 from dataclasses import dataclass, replace
 import math
@@ -61,6 +63,7 @@ WORKLOADS = {
     "shared_prefix": Workload("shared_prefix", 32, 8, 128, "bf16", "bf16", 192, "shared", 0, 512, seed=4,
                               num_prompts=64, samples=3, prefix_len=1000),
     "fp8_long": Workload("fp8_long", 32, 8, 128, "fp8", "bf16", 128, "loguniform", 256, 32768, seed=5),
+    "prefill70b": Workload("prefill70b", 64, 8, 128, "bf16", "bf16", 16, "uniform", 512, 4096, seed=6),
 }
 
 TINY_LENS = (1, 15, 16, 40)
