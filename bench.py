@@ -672,7 +672,7 @@ def run_prefill(args, device, rank, world):
             "us_attention": round(1e3 * att_ms, 2), "us_write": round(1e3 * wr_ms, 2),
             "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(achieved / peak, 4), "traffic": None,
-                         "kernel": "prefill_kernel (mma.sync m16n8k16 bf16)", "peak_source": peak_kind},
+                         "kernel": "prefill_tc_kernel (tcgen05.mma, TMEM accumulators)" if os.environ.get("PKV_PREFILL_KERNEL", "")[:1] != "m" else "prefill_kernel (mma.sync m16n8k16)", "peak_source": peak_kind},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps, "device_errors": int(step.err.item()),
             "clocks": clk.summary(),
         }

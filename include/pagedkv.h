@@ -264,11 +264,16 @@ int pkv_paged_attention_decode_shared(void* out, const void* q, int q_dtype,
  * r = query_start[s] + i sits at position context_lens[s] - nq_s + i and
  * attends to tokens 0 .. that position.  A whole prompt, a prompt after a
  * cached prefix and a chunk of a long prompt are all this call.
- *   out, q          [total_q][num_heads][head_dim], total_q = query_start[num_seqs]
+ *   out, q          [total_query_tokens][num_heads][head_dim]
  *   block_tables    int32 [num_seqs][max_blocks_per_seq]
- *   context_lens    int32 [num_seqs]; query_start int32 [num_seqs + 1], query_start[0] = 0
+ *   context_lens    int32 [num_seqs]; query_start int32 [num_seqs + 1], query_start[0] = 0,
+ *                   query_start[num_seqs] = total_query_tokens
  *   max_query_len   >= every nq_s (sizes the launch; rows past it are not computed)
  * Supported: bf16 q, bf16 cache, head_dim 128, block_size 16, any GQA group.
+ * The product runs on the tcgen05 tensor cores (TMEM accumulators); setting
+ * the environment variable PKV_PREFILL_KERNEL=mma before the first call
+ * selects the warp-level mma.sync kernel instead (same results, for
+ * comparison).
  * Device-data errors (a table entry out of range among the blocks a sequence
  * reads: its tokens are left out; nq_s > context_lens[s] or a context longer
  * than the table: the sequence's rows are zeroed) are counted into err_count.
@@ -277,8 +282,8 @@ int pkv_paged_attention_prefill(void* out, const void* q, int q_dtype,
                                 const void* k_pool, const void* v_pool, int cache_dtype,
                                 const int32_t* block_tables, int max_blocks_per_seq,
                                 const int32_t* context_lens, const int32_t* query_start, int num_seqs,
-                                int max_query_len, int num_blocks, int block_size, int num_heads,
-                                int num_kv_heads, int head_dim, float scale,
+                                int total_query_tokens, int max_query_len, int num_blocks, int block_size,
+                                int num_heads, int num_kv_heads, int head_dim, float scale,
                                 int32_t* err_count, void* stream);
 
 /* ------------------------------------------------------------------------

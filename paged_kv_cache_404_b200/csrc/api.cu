@@ -3,6 +3,8 @@
 // every buffer belongs to the caller.
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
+
 #include "pagedkv.h"
 #include "pkv_common.cuh"
 
@@ -23,6 +25,8 @@ bool decode_tc_groupable(bool fp8, int head_dim, int group);
 cudaError_t launch_decode_merge(const DecodeParams& p, int out_dtype, cudaStream_t stream);
 cudaError_t launch_prefill(const CUtensorMap& tmK, const CUtensorMap& tmV, const PrefillParams& p, int max_query_len,
                            cudaStream_t stream);
+cudaError_t launch_prefill_tc(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                              const PrefillParams& p, int max_query_len, cudaStream_t stream);
 }  // namespace pkv
 
 using namespace pkv;
@@ -78,6 +82,31 @@ bool pool_tensor_map(CUtensorMap* map, const void* pool, int cache_dtype, int he
                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// bf16 tensor [rows][heads][head_dim]: box of box_rows rows x 1 head x 128 bytes,
+// 128-byte swizzle; rows past the end read zeros.
+bool rows_tensor_map(CUtensorMap* map, const void* base, int head_dim, int heads, long long rows, int box_rows) {
+    auto enc = encode_fn();
+    if (enc == nullptr) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)heads, (cuuint64_t)rows};
+    const cuuint64_t strides[2] = {(cuuint64_t)head_dim * 2, (cuuint64_t)head_dim * heads * 2};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Prefill kernel: 0 = tcgen05 (default), 1 = mma.sync (PKV_PREFILL_KERNEL=mma, for comparison).
+int prefill_kernel_choice() {
+    static int choice = -1;
+    if (choice < 0) {
+        const char* v = getenv("PKV_PREFILL_KERNEL");
+        choice = (v != nullptr && v[0] == 'm') ? 1 : 0;
+    }
+    return choice;
 }
 
 int min_partition_of(int partition_tokens) {
@@ -321,15 +350,16 @@ extern "C" {
 int pkv_paged_attention_prefill(void* out, const void* q, int q_dtype, const void* k_pool, const void* v_pool,
                                 int cache_dtype, const int32_t* block_tables, int max_blocks_per_seq,
                                 const int32_t* context_lens, const int32_t* query_start, int num_seqs,
-                                int max_query_len, int num_blocks, int block_size, int num_heads, int num_kv_heads,
-                                int head_dim, float scale, int32_t* err_count, void* stream) {
-    if (num_seqs < 0 || max_blocks_per_seq <= 0 || max_query_len < 0 || num_blocks <= 0 || block_size <= 0 ||
-        num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0)
+                                int total_query_tokens, int max_query_len, int num_blocks, int block_size,
+                                int num_heads, int num_kv_heads, int head_dim, float scale, int32_t* err_count,
+                                void* stream) {
+    if (num_seqs < 0 || max_blocks_per_seq <= 0 || max_query_len < 0 || total_query_tokens < 0 || num_blocks <= 0 ||
+        block_size <= 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0)
         return PKV_EINVAL;
     if (num_heads % num_kv_heads != 0) return PKV_EINVAL;
     if (block_size != kBlockSize) return PKV_EUNSUPPORTED;
     if (q_dtype != PKV_BF16 || cache_dtype != PKV_BF16 || head_dim != 128) return PKV_EUNSUPPORTED;
-    if (num_seqs == 0 || max_query_len == 0) return PKV_OK;
+    if (num_seqs == 0 || max_query_len == 0 || total_query_tokens == 0) return PKV_OK;
     if (num_seqs > 65535 || num_heads > 65535) return PKV_EUNSUPPORTED;
     if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens || !query_start) return PKV_EINVAL;
     if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) ||
@@ -353,7 +383,15 @@ int pkv_paged_attention_prefill(void* out, const void* q, int q_dtype, const voi
     if (!pool_tensor_map(&tmK, k_pool, cache_dtype, head_dim, num_kv_heads, slots) ||
         !pool_tensor_map(&tmV, v_pool, cache_dtype, head_dim, num_kv_heads, slots))
         return PKV_ECUDA;
-    cudaError_t e = launch_prefill(tmK, tmV, p, max_query_len, static_cast<cudaStream_t>(stream));
+    cudaError_t e;
+    if (prefill_kernel_choice() == 1) {
+        e = launch_prefill(tmK, tmV, p, max_query_len, static_cast<cudaStream_t>(stream));
+    } else {
+        // q viewed as [total_q][heads][head_dim]; boxes of 128 rows x 1 head x 128 bytes
+        CUtensorMap tmQ;
+        if (!rows_tensor_map(&tmQ, q, head_dim, num_heads, total_query_tokens, 128)) return PKV_ECUDA;
+        e = launch_prefill_tc(tmQ, tmK, tmV, p, max_query_len, static_cast<cudaStream_t>(stream));
+    }
     return e == cudaSuccess ? PKV_OK : PKV_ECUDA;
 }
 

@@ -141,8 +141,8 @@ def paged_attention_prefill(out, q, k_pool, v_pool, block_tables, context_lens, 
         raise ValueError("query_start must have num_seqs + 1 entries")
     st = L.lib().pkv_paged_attention_prefill(
         _ptr(out), _ptr(q), _dtype_code(q), _ptr(k_pool), _ptr(v_pool), _dtype_code(k_pool), _ptr(block_tables),
-        int(block_tables.shape[1]), _ptr(context_lens), _ptr(query_start), S, int(max_query_len), NB, bs, Hq, Hkv,
-        D, float(scale), _ptr(err_count), _stream(stream))
+        int(block_tables.shape[1]), _ptr(context_lens), _ptr(query_start), S, T, int(max_query_len), NB, bs, Hq,
+        Hkv, D, float(scale), _ptr(err_count), _stream(stream))
     L.check("pkv_paged_attention_prefill", st)
     return out
 

@@ -131,3 +131,23 @@ def test_full_size_prefill_sampled_rows():
     rows = np.unique(np.concatenate([rows, c.qs[1:] - 1, c.qs[:-1]]))   # first and last row of every prompt
     ref, _ = c.oracle(rows=rows)
     assert_close(got[rows], ref[rows], "bf16", "prefill70b")
+
+
+def test_warp_mma_kernel_agrees(tmp_path):
+    """The mma.sync prefill kernel (PKV_PREFILL_KERNEL=mma, a separate process)
+    gives the oracle's result on the ragged case too."""
+    import os
+    import subprocess
+    import sys
+    code = (
+        "import numpy as np, sys; sys.path.insert(0, %r)\n"
+        "from tests.test_gpu_prefill import PrefillCase, RAGGED\n"
+        "from tests.helpers import assert_close, out_to_f64\n"
+        "c = PrefillCase(16, 4, *RAGGED, seed=44)\n"
+        "got = out_to_f64(c.run()); ref, bad = c.oracle()\n"
+        "assert bad == 0 and int(c.err.item()) == 0\n"
+        "assert_close(got, ref, 'bf16', 'mma.sync prefill')\n"
+        "print('ok')\n" % os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    env = dict(os.environ, PKV_PREFILL_KERNEL="mma")
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout[-2000:] + r.stderr[-2000:]
