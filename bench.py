@@ -589,8 +589,8 @@ def prefill_cpu_baseline(w, target_s=12.0):
             "sample": "%d query rows of a %d-token prompt (all 64 heads), fp64, %.2f s" % (n, L, dt)}
 
 
-def run_prefill(args, device, rank, world):
-    w = rank_workload(W.WORKLOADS["prefill70b"], rank)
+def run_prefill(args, w0, device, rank, world):
+    w = rank_workload(w0, rank)
     step = PrefillStep(w, device)
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
@@ -798,7 +798,7 @@ def main(argv=None):
                                     device_id=torch.device("cuda", local))
             dist.barrier()
             pkv_build.build()
-        run_prefill(args, torch.device("cuda", local), rank, world)
+        run_prefill(args, w0, torch.device("cuda", local), rank, world)
         if world > 1:
             import torch.distributed as dist
             dist.barrier()

@@ -7,40 +7,50 @@
 // (iplexlaw.co.kr, logical vs physical order; gyaansetu.com, what the KV cache
 // holds).
 //
-// One CTA per (sequence, 128 query rows, query head); six warps:
-//  - warp 4 (producer): TMA-loads the Q tile once and, per 128-key tile, the K
-//    and V of 8 blocks of the table (16-slot x 1-head x 128-byte boxes, 128-byte
-//    swizzle) into a 2-stage ring; V rows that hold no token of the context
+// One CTA per (sequence, 256 query rows = two Q tiles of 128, query head); ten
+// warps:
+//  - warp 8 (producer): TMA-loads the two Q tiles once and, per 64-key tile, the
+//    K and V of 4 blocks of the table (16-slot x 1-head x 128-byte boxes,
+//    128-byte swizzle) into a 3-stage ring; V rows that hold no token of the context
 //    (past its end, or a block past the table or with a bad id) are zeroed in
 //    shared memory, so that a zero probability never meets a NaN there;
-//  - warp 5 (MMA): one thread issues tcgen05.mma: S = Q K^T (M=128, N=128,
-//    K=128, bf16 -> fp32) into one of two TMEM buffers, then O += P V (P from
+//  - warp 9 (MMA): one thread issues tcgen05.mma: per Q tile t, S_t = Q_t K^T
+//    (M=128, N=64, K=128, bf16 -> fp32) into TMEM, then O_t += P_t V (P from
 //    shared memory, V MN-major) into a TMEM accumulator; tcgen05.commit signals
 //    mbarriers; the warp allocates and frees the 512 TMEM columns;
-//  - warps 0-3 (softmax): thread r owns query row r (TMEM lane r): loads its
-//    128 scores with tcgen05.ld, applies the causal mask, runs the online
+//  - warps 0-3 and 4-7 (softmax, one warpgroup per Q tile): thread r owns
+//    query row r of its tile (TMEM lane r): loads its 64 scores with
+//    tcgen05.ld, applies the causal mask, runs the online
 //    softmax in base 2 (the reference max moves only when a score exceeds it by
 //    more than 2^8, then O is rescaled in TMEM), writes P as bf16 into the
 //    swizzled K-major layout the PV MMA reads, and finally normalises O and
 //    stores the rows.
-// S for tile j+1 is computed while the softmax works on tile j.
+// The products are issued PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), ..., so that
+// each warpgroup's softmax runs while the tensor core works for the other.
 #include "pkv_common.cuh"
 
 namespace pkv {
 
 namespace {
 
-constexpr int kTcRows = 128;                   // query rows per CTA (MMA M)
-constexpr int kTcKeys = 128;                   // keys per tile (MMA N of S, K of PV)
+constexpr int kTcRows = 128;                   // query rows per Q tile (MMA M)
+constexpr int kTcQT = 2;                       // Q tiles per CTA (two softmax warpgroups, ping-pong)
+constexpr int kTcKeys = 64;                    // keys per KV tile (MMA N of S, K of PV)
 constexpr int kTcD = 128;                      // head_dim
-constexpr int kTcChunk = kTcRows * 128;        // one 64-element column chunk of a 128-row operand: 16 KB
-constexpr int kTcOperand = 2 * kTcChunk;       // 128 rows x 128 bf16: 32 KB
-constexpr int kTcStages = 2;
+constexpr int kTcQChunk = kTcRows * 128;       // one 64-element column chunk of a 128-row operand: 16 KB
+constexpr int kTcQBytes = 2 * kTcQChunk;       // Q tile: 128 rows x 128 bf16
+constexpr int kTcPBytes = kTcRows * 128;       // P tile: 128 rows x 64 keys (one chunk)
+constexpr int kTcKVChunk = kTcKeys * 128;      // one 64-element column chunk of a 64-row operand: 8 KB
+constexpr int kTcKVBytes = 2 * kTcKVChunk;     // K (or V) tile: 64 keys x 128 bf16
+constexpr int kTcStages = 3;
+constexpr int kTcBlocks = kTcKeys / kBlockSize;  // table blocks per KV tile
 // shared memory layout (offsets from a 1024-aligned base)
-constexpr int kTcQ = 0;
-constexpr int kTcP = kTcQ + kTcOperand;
-constexpr int kTcKV = kTcP + kTcOperand;       // stage st: K at kTcKV + st*2*kTcOperand, V after it
-constexpr int kTcSmem = kTcKV + kTcStages * 2 * kTcOperand;  // 192 KB
+constexpr int kTcQ = 0;                                    // Q tile t at kTcQ + t * kTcQBytes
+constexpr int kTcP = kTcQ + kTcQT * kTcQBytes;             // P tile t at kTcP + t * kTcPBytes
+constexpr int kTcKV = kTcP + kTcQT * kTcPBytes;            // stage st: K, then V
+constexpr int kTcSmem = kTcKV + kTcStages * 2 * kTcKVBytes;  // 192 KB
+// TMEM columns: S of Q tile t at t*64, O of Q tile t at 128 + t*128
+constexpr int kTcSCol = 0, kTcOCol = 128;
 constexpr float kRescaleThreshold = 8.f;       // log2 of the largest factor p may exceed 1 by
 
 // ---- tcgen05 wrappers -----------------------------------------------------------
@@ -119,39 +129,40 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 
 }  // namespace
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
-    // barriers: kv_full[2], kv_empty[2], q_full, s_full[2], p_full, pv_done, v_ready[2]
-    __shared__ __align__(8) uint64_t bars[12];
+    // kv_full[3], kv_empty[3], v_ready[3], q_full, s_full[2], p_full[2], pv_done[2]
+    __shared__ __align__(8) uint64_t bars[16];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
     volatile int* abort_flag = &abort_sh;
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
     const uint32_t b0 = smem_u32(&bars[0]);
-    const uint32_t kv_full = b0, kv_empty = b0 + 16, q_full = b0 + 32, s_full = b0 + 40, p_full = b0 + 56,
-                   pv_done = b0 + 64, v_ready = b0 + 72;
+    const uint32_t kv_full = b0, kv_empty = b0 + 24, v_ready = b0 + 48, q_full = b0 + 72, s_full = b0 + 80,
+                   p_full = b0 + 96, pv_done = b0 + 112;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int kProducer = 8, kMma = 9;
 
     const int s = blockIdx.y, h = blockIdx.z, kvh = h / p.group;
     const int tile = gridDim.x - 1 - blockIdx.x;
     if (threadIdx.x == 0) {
-        mbar_init(kv_full, 1);
-        mbar_init(kv_full + 8, 1);
-        mbar_init(kv_empty, 1);
-        mbar_init(kv_empty + 8, 1);
+        for (int i = 0; i < kTcStages; ++i) {
+            mbar_init(kv_full + 8 * i, 1);
+            mbar_init(kv_empty + 8 * i, 1);
+            mbar_init(v_ready + 8 * i, 1);
+        }
         mbar_init(q_full, 1);
-        mbar_init(s_full, 1);
-        mbar_init(s_full + 8, 1);
-        mbar_init(p_full, 4);
-        mbar_init(pv_done, 1);
-        mbar_init(v_ready, 1);
-        mbar_init(v_ready + 8, 1);
+        for (int t = 0; t < kTcQT; ++t) {
+            mbar_init(s_full + 8 * t, 1);
+            mbar_init(p_full + 8 * t, 4);
+            mbar_init(pv_done + 8 * t, 1);
+        }
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 4 && lane == 0) {
+    if (warp == kProducer && lane == 0) {
         prefetch_tensormap(&tmQ);
         prefetch_tensormap(&tmK);
         prefetch_tensormap(&tmV);
@@ -163,11 +174,11 @@ __global__ void __launch_bounds__(192, 1)
     const int qs0 = p.query_start[s];
     const int nq = p.query_start[s + 1] - qs0;
     const int ctx = p.context_lens[s];
-    const int row0 = tile * kTcRows;
+    const int row0 = tile * (kTcQT * kTcRows);
     if (row0 >= nq) return;  // the whole CTA leaves together, before TMEM allocation
     if (nq > ctx || ctx > p.max_blocks_per_seq * kBlockSize) {
         if (tile == 0 && h == 0 && threadIdx.x == 0) count_error(p.err);
-        const int rows = min(kTcRows, nq - row0);
+        const int rows = min(kTcQT * kTcRows, nq - row0);
         for (int e = threadIdx.x; e < rows * kTcD; e += blockDim.x) {
             const int r = e / kTcD, d = e - r * kTcD;
             p.out[((size_t)(qs0 + row0 + r) * p.num_heads + h) * kTcD + d] = __float2bfloat16(0.f);
@@ -175,15 +186,21 @@ __global__ void __launch_bounds__(192, 1)
         return;
     }
     const int pos0 = ctx - nq;
-    const int last_row = min(row0 + kTcRows, nq) - 1;
-    const int last_pos = pos0 + last_row;
-    const int ntiles = last_pos / kTcKeys + 1;
+    // KV tiles each Q tile reads (0 for a Q tile past the last query row)
+    int ntq[kTcQT];
+#pragma unroll
+    for (int t = 0; t < kTcQT; ++t) {
+        const int first = row0 + t * kTcRows;
+        ntq[t] = first < nq ? (pos0 + min(first + kTcRows, nq) - 1) / kTcKeys + 1 : 0;
+    }
+    const int ntiles = ntq[kTcQT - 1] > ntq[0] ? ntq[kTcQT - 1] : ntq[0];
+    const int last_pos = pos0 + min(row0 + kTcQT * kTcRows, nq) - 1;
     const int count_from = tile == 0 ? 0 : (pos0 + row0 - 1) / kBlockSize + 1;  // blocks first read here
     const int32_t* tab = p.block_tables + (size_t)s * p.max_blocks_per_seq;
     const int nblk_seq = (ctx + kBlockSize - 1) / kBlockSize;
 
-    // ---- TMEM: 512 columns (S buffers at 0 and 128, O at 256)
-    if (warp == 5) {
+    // ---- TMEM: 512 columns
+    if (warp == kMma) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_sh)),
                      "r"(512));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -193,23 +210,26 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
 
-    if (warp == 4) {
+    if (warp == kProducer) {
         // ================= producer =================
         if (lane == 0) {
-            mbar_arrive_expect_tx(q_full, kTcOperand);
             // rows past total_q read zeros (the tensor map ends there)
-            tma_load_3d(base + kTcQ, &tmQ, 0, h, qs0 + row0, q_full);
-            tma_load_3d(base + kTcQ + kTcChunk, &tmQ, 64, h, qs0 + row0, q_full);
+            mbar_arrive_expect_tx(q_full, kTcQT * kTcQBytes);
+            for (int t = 0; t < kTcQT; ++t) {
+                tma_load_3d(base + kTcQ + t * kTcQBytes, &tmQ, 0, h, qs0 + row0 + t * kTcRows, q_full);
+                tma_load_3d(base + kTcQ + t * kTcQBytes + kTcQChunk, &tmQ, 64, h, qs0 + row0 + t * kTcRows, q_full);
+            }
         }
         for (int j = 0; j < ntiles && !*abort_flag; ++j) {
             const int st = j % kTcStages, round = j / kTcStages;
-            // block ids of this tile: lanes 0..7; a block is loaded if it is in the table
+            // block ids of this tile: lanes 0..3; a block is loaded if it is in the table
             // and its id is in range
-            const int jb = j * 8 + (lane & 7);
+            const int jb = j * kTcBlocks + (lane & (kTcBlocks - 1));
             int id = -1;
-            if (lane < 8 && jb < nblk_seq) id = __ldg(tab + jb);
-            const bool load = lane < 8 && jb < nblk_seq && id >= 0 && id < p.num_blocks;
-            if (lane < 8 && jb < nblk_seq && !load && h == 0 && jb >= count_from && jb <= last_pos / kBlockSize)
+            if (lane < kTcBlocks && jb < nblk_seq) id = __ldg(tab + jb);
+            const bool load = lane < kTcBlocks && jb < nblk_seq && id >= 0 && id < p.num_blocks;
+            if (lane < kTcBlocks && jb < nblk_seq && !load && h == 0 && jb >= count_from &&
+                jb <= last_pos / kBlockSize)
                 count_error(p.err);
             const unsigned loaded = __ballot_sync(0xffffffffu, load);
             bool go = true;
@@ -222,30 +242,30 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 break;
             }
-            const uint32_t kdst = base + kTcKV + st * 2 * kTcOperand, vdst = kdst + kTcOperand;
+            const uint32_t kdst = base + kTcKV + st * 2 * kTcKVBytes, vdst = kdst + kTcKVBytes;
             if (lane == 0) mbar_arrive_expect_tx(kv_full + 8 * st, __popc(loaded) * 4 * (kBlockSize * 128));
             __syncwarp();
             if (load) {
                 const int row = id * kBlockSize;
                 const uint32_t off = lane * kBlockSize * 128;
                 tma_load_3d(kdst + off, &tmK, 0, kvh, row, kv_full + 8 * st);
-                tma_load_3d(kdst + kTcChunk + off, &tmK, 64, kvh, row, kv_full + 8 * st);
+                tma_load_3d(kdst + kTcKVChunk + off, &tmK, 64, kvh, row, kv_full + 8 * st);
                 tma_load_3d(vdst + off, &tmV, 0, kvh, row, kv_full + 8 * st);
-                tma_load_3d(vdst + kTcChunk + off, &tmV, 64, kvh, row, kv_full + 8 * st);
+                tma_load_3d(vdst + kTcKVChunk + off, &tmV, 64, kvh, row, kv_full + 8 * st);
             }
             // V rows with no token: whole blocks not loaded, and the slots past the context
             // in the sequence's last block (once it has landed)
-            for (int b = 0; b < 8; ++b) {
+            for (int b = 0; b < kTcBlocks; ++b) {
                 if ((loaded >> b) & 1u) continue;
                 for (int i = lane; i < kBlockSize * 16; i += 32) {
                     const int r = b * kBlockSize + (i >> 4), c = i & 15;
-                    const uint32_t a = vdst + (c >> 3) * kTcChunk + r * 128 + ((c & 7) << 4);
+                    const uint32_t a = vdst + (c >> 3) * kTcKVChunk + r * 128 + ((c & 7) << 4);
                     asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0) : "memory");
                 }
             }
             const int jt = (ctx % kBlockSize) ? nblk_seq - 1 : -1;
-            const int bt = jt - j * 8;
-            if (bt >= 0 && bt < 8 && ((loaded >> bt) & 1u)) {
+            const int bt = jt - j * kTcBlocks;
+            if (bt >= 0 && bt < kTcBlocks && ((loaded >> bt) & 1u)) {
                 bool landed = true;
                 if (lane == 0) landed = mbar_wait_bounded(kv_full + 8 * st, round & 1);
                 if (!__shfl_sync(0xffffffffu, landed, 0)) {
@@ -258,7 +278,7 @@ __global__ void __launch_bounds__(192, 1)
                 const int r0 = ctx % kBlockSize;
                 for (int i = lane; i < (kBlockSize - r0) * 16; i += 32) {
                     const int r = bt * kBlockSize + r0 + (i >> 4), c = i & 15;
-                    const uint32_t a = vdst + (c >> 3) * kTcChunk + r * 128 + ((c & 7) << 4);
+                    const uint32_t a = vdst + (c >> 3) * kTcKVChunk + r * 128 + ((c & 7) << 4);
                     asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0) : "memory");
                 }
             }
@@ -266,96 +286,117 @@ __global__ void __launch_bounds__(192, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(v_ready + 8 * st);
         }
-    } else if (warp == 5) {
+    } else if (warp == kMma) {
         // ================= MMA issuer =================
+        // order per KV tile j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1): each Q tile's softmax
+        // overlaps the other tile's products
         const uint32_t idesc_s = instr_desc_bf16(kTcRows, kTcKeys, false);
         const uint32_t idesc_o = instr_desc_bf16(kTcRows, kTcD, true);
         bool alive = true;
-        if (lane == 0) alive = mbar_wait_bounded(q_full, 0);
-        auto issue_s = [&](int j) -> bool {
-            const int st = j % kTcStages, round = j / kTcStages;
-            if (!mbar_wait_bounded(kv_full + 8 * st, round & 1)) return false;
+        auto kv_landed = [&](int j) { return mbar_wait_bounded(kv_full + 8 * (j % kTcStages), (j / kTcStages) & 1); };
+        auto issue_s = [&](int t, int j) {
             tc_fence_after();
-            const uint32_t kb = base + kTcKV + st * 2 * kTcOperand;
-            const uint32_t d = tmem + (j & 1) * kTcKeys;
+            const uint32_t kb = base + kTcKV + (j % kTcStages) * 2 * kTcKVBytes;
+            const uint32_t qb = base + kTcQ + t * kTcQBytes;
 #pragma unroll
             for (int ks = 0; ks < kTcD / 16; ++ks) {
-                const uint32_t off = (ks >> 2) * kTcChunk + (ks & 3) * 32;
-                umma_ss(d, smem_desc(base + kTcQ + off, 16, 1024), smem_desc(kb + off, 16, 1024), idesc_s, ks > 0);
+                umma_ss(tmem + kTcSCol + t * kTcKeys,
+                        smem_desc(qb + (ks >> 2) * kTcQChunk + (ks & 3) * 32, 16, 1024),
+                        smem_desc(kb + (ks >> 2) * kTcKVChunk + (ks & 3) * 32, 16, 1024), idesc_s, ks > 0);
             }
-            umma_commit(s_full + 8 * (j & 1));
+            umma_commit(s_full + 8 * t);
+        };
+        auto issue_pv = [&](int t, int j) -> bool {
+            if (!mbar_wait_bounded(p_full + 8 * t, j & 1)) return false;
+            if (!mbar_wait_bounded(v_ready + 8 * (j % kTcStages), (j / kTcStages) & 1)) return false;
+            tc_fence_after();
+            const uint32_t vb = base + kTcKV + (j % kTcStages) * 2 * kTcKVBytes + kTcKVBytes;
+#pragma unroll
+            for (int ks = 0; ks < kTcKeys / 16; ++ks) {
+                umma_ss(tmem + kTcOCol + t * kTcD, smem_desc(base + kTcP + t * kTcPBytes + ks * 32, 16, 1024),
+                        smem_desc(vb + ks * 16 * 128, kTcKVChunk, 1024), idesc_o, j > 0 || ks > 0);
+            }
+            umma_commit(pv_done + 8 * t);
             return true;
         };
-        if (lane == 0 && alive) alive = issue_s(0);
-        for (int j = 0; j < ntiles; ++j) {
-            alive = __shfl_sync(0xffffffffu, alive, 0) && !*abort_flag;
-            if (!alive) break;
-            if (lane == 0) {
-                if (j + 1 < ntiles) alive = issue_s(j + 1);
-                // P_j written (and O rescaled) by the softmax warps; V's empty rows zeroed
-                const int st = j % kTcStages;
-                if (alive) alive = mbar_wait_bounded(p_full, j & 1);
-                if (alive) alive = mbar_wait_bounded(v_ready + 8 * st, (j / kTcStages) & 1);
-                if (alive) {
-                    tc_fence_after();
-                    const uint32_t vb = base + kTcKV + st * 2 * kTcOperand + kTcOperand;
-#pragma unroll
-                    for (int ks = 0; ks < kTcKeys / 16; ++ks) {
-                        const uint64_t a = smem_desc(base + kTcP + (ks >> 2) * kTcChunk + (ks & 3) * 32, 16, 1024);
-                        const uint64_t b = smem_desc(vb + ks * 16 * 128, kTcChunk, 1024);
-                        umma_ss(tmem + 256, a, b, idesc_o, j > 0 || ks > 0);
+        if (lane == 0) {
+            alive = mbar_wait_bounded(q_full, 0) && kv_landed(0);
+            if (alive)
+                for (int t = 0; t < kTcQT; ++t)
+                    if (ntq[t] > 0) issue_s(t, 0);
+            for (int j = 0; j < ntiles && alive && !*abort_flag; ++j) {
+                const bool next = j + 1 < ntiles;
+                for (int t = 0; t < kTcQT && alive; ++t) {
+                    if (j < ntq[t]) alive = issue_pv(t, j);
+                    if (alive && j + 1 < ntq[t]) {
+                        alive = kv_landed(j + 1);
+                        if (alive) issue_s(t, j + 1);
                     }
-                    umma_commit(pv_done);
-                    umma_commit(kv_empty + 8 * st);
                 }
+                (void)next;
+                if (alive) umma_commit(kv_empty + 8 * (j % kTcStages));
             }
-        }
-        if (!__shfl_sync(0xffffffffu, alive, 0)) {
-            if (lane == 0) {
+            if (!alive) {
                 count_error(p.err);
                 atomicExch(&abort_sh, 1);
             }
         }
+        __syncwarp();
     } else {
-        // ================= softmax (warps 0-3): thread = query row =================
-        const int r = threadIdx.x;                 // 0..127 = TMEM lane
-        const int qpos = pos0 + row0 + r;          // this row's position (rows past nq: unused)
-        const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+        // ================= softmax: warpgroup t = Q tile t, thread = query row =================
+        const int t = warp >> 2;
+        const int r = threadIdx.x & 127;             // TMEM lane
+        const int qrow = row0 + t * kTcRows + r;     // query row in the sequence
+        const int qpos = pos0 + qrow;
+        const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        const uint32_t s_addr = lane_addr + kTcSCol + t * kTcKeys, o_addr = lane_addr + kTcOCol + t * kTcD;
+        const uint32_t p_row = base + kTcP + t * kTcPBytes + r * 128;
         float m_ref = -INFINITY, l = 0.f;
         bool alive = true;
-        for (int j = 0; j < ntiles; ++j) {
-            if (!alive || *abort_flag) break;
+        const int nt = ntq[t];
+        for (int j = 0; j < nt; ++j) {
+            if (*abort_flag) {
+                alive = false;
+                break;
+            }
             // blocks of this tile that hold tokens (in the table, id in range)
             unsigned okmask = 0;
 #pragma unroll
-            for (int b = 0; b < 8; ++b) {
-                const int jb = j * 8 + b;
+            for (int b = 0; b < kTcBlocks; ++b) {
+                const int jb = j * kTcBlocks + b;
                 const int id = jb < nblk_seq ? __ldg(tab + jb) : -1;
                 if (id >= 0 && id < p.num_blocks) okmask |= 1u << b;
             }
-            bool w1 = mbar_wait_bounded(s_full + 8 * (j & 1), (j >> 1) & 1);
+            const bool w1 = mbar_wait_bounded(s_full + 8 * t, j & 1);
             if (!__all_sync(0xffffffffu, w1)) {
                 alive = false;
                 break;
             }
             tc_fence_after();
-            // scores of keys j*128 + c, masked: causal, block id out of range
             float x[kTcKeys];
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
+            for (int c2 = 0; c2 < kTcKeys / 32; ++c2) {
                 float v[32];
-                tmem_ld32(lane_addr + (j & 1) * kTcKeys + 32 * c4, v);
+                tmem_ld32(s_addr + 32 * c2, v);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) x[32 * c4 + i] = v[i];
+                for (int i = 0; i < 32; ++i) x[32 * c2 + i] = v[i];
             }
             tmem_wait_ld();
             float mx = -INFINITY;
+            const int k0 = j * kTcKeys;
+            if (k0 + kTcKeys - 1 <= qpos && okmask == (1u << kTcBlocks) - 1u) {
 #pragma unroll
-            for (int c = 0; c < kTcKeys; ++c) {
-                const int kpos = j * kTcKeys + c;
-                const bool valid = kpos <= qpos && ((okmask >> (c >> 4)) & 1u);
-                x[c] = valid ? x[c] * p.score_scale : -INFINITY;
-                mx = fmaxf(mx, x[c]);
+                for (int c = 0; c < kTcKeys; ++c) {
+                    x[c] *= p.score_scale;
+                    mx = fmaxf(mx, x[c]);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < kTcKeys; ++c) {
+                    const bool valid = k0 + c <= qpos && ((okmask >> (c >> 4)) & 1u);
+                    x[c] = valid ? x[c] * p.score_scale : -INFINITY;
+                    mx = fmaxf(mx, x[c]);
+                }
             }
             // the reference max moves only when a score exceeds it by more than 2^8
             float alpha = 1.f;
@@ -363,10 +404,18 @@ __global__ void __launch_bounds__(192, 1)
             const float m_new = move ? mx : m_ref;
             if (move && m_ref != -INFINITY) alpha = fast_exp2(m_ref - m_new);
             const float mu = m_new == -INFINITY ? 0.f : m_new;
+            // P row as bf16 (computed before waiting for the previous PV)
+            uint32_t pw[kTcKeys / 2];
             float sum = 0.f;
+#pragma unroll
+            for (int e = 0; e < kTcKeys / 2; ++e) {
+                const float p0 = fast_exp2(x[2 * e] - mu), p1 = fast_exp2(x[2 * e + 1] - mu);
+                sum += p0 + p1;
+                pw[e] = pack_bf16x2(p0, p1);
+            }
             // PV_{j-1} must be done before P is overwritten and before O is read
             if (j > 0) {
-                bool w2 = mbar_wait_bounded(pv_done, (j - 1) & 1);
+                const bool w2 = mbar_wait_bounded(pv_done + 8 * t, (j - 1) & 1);
                 if (!__all_sync(0xffffffffu, w2)) {
                     alive = false;
                     break;
@@ -374,60 +423,46 @@ __global__ void __launch_bounds__(192, 1)
                 tc_fence_after();
                 if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-                    for (int c4 = 0; c4 < 4; ++c4) {
+                    for (int c4 = 0; c4 < kTcD / 32; ++c4) {
                         float v[32];
-                        tmem_ld32(lane_addr + 256 + 32 * c4, v);
+                        tmem_ld32(o_addr + 32 * c4, v);
                         tmem_wait_ld();
 #pragma unroll
                         for (int i = 0; i < 32; ++i) v[i] *= alpha;
-                        tmem_st32(lane_addr + 256 + 32 * c4, v);
+                        tmem_st32(o_addr + 32 * c4, v);
                     }
                     tmem_wait_st();
                 }
             }
-            l *= alpha;
+            l = l * alpha + sum;
             m_ref = m_new;
-            // P row r as bf16 into the K-major 128-byte-swizzled operand: keys 64c..64c+63 in
-            // column chunk c, 16-byte piece q of the row at ((q ^ (r & 7)) << 4)
+            // P row into the K-major 128-byte-swizzled operand: 16-byte piece q at ((q ^ (r & 7)) << 4)
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float p0 = fast_exp2(x[64 * c + 8 * q + 2 * e] - mu);
-                        const float p1 = fast_exp2(x[64 * c + 8 * q + 2 * e + 1] - mu);
-                        sum += p0 + p1;
-                        w[e] = pack_bf16x2(p0, p1);
-                    }
-                    const uint32_t a = base + kTcP + c * kTcChunk + r * 128 + ((q ^ (r & 7)) << 4);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(w[0]), "r"(w[1]),
-                                 "r"(w[2]), "r"(w[3])
-                                 : "memory");
-                }
-            l += sum;
+            for (int q = 0; q < 8; ++q)
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(p_row + ((q ^ (r & 7)) << 4)),
+                             "r"(pw[4 * q]), "r"(pw[4 * q + 1]), "r"(pw[4 * q + 2]), "r"(pw[4 * q + 3])
+                             : "memory");
             fence_proxy_async_smem();  // generic-proxy P stores -> read by the tensor core
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
+            if (lane == 0) mbar_arrive(p_full + 8 * t);
         }
         if (!alive && lane == 0) {
             count_error(p.err);
             atomicExch(&abort_sh, 1);
         }
         // epilogue: wait for the last PV, normalise and store the row
-        if (alive && !*abort_flag) {
-            bool w3 = mbar_wait_bounded(pv_done, (ntiles - 1) & 1);
+        if (alive && nt > 0 && !*abort_flag) {
+            const bool w3 = mbar_wait_bounded(pv_done + 8 * t, (nt - 1) & 1);
             if (__all_sync(0xffffffffu, w3)) {
                 tc_fence_after();
                 const float inv = l > 0.f ? 1.f / l : 0.f;
-                const bool store = row0 + r < nq;
-                __nv_bfloat16* out = p.out + ((size_t)(qs0 + row0 + r) * p.num_heads + h) * kTcD;
+                const bool store = qrow < nq;
+                __nv_bfloat16* out = p.out + ((size_t)(qs0 + (store ? qrow : 0)) * p.num_heads + h) * kTcD;
 #pragma unroll 1
-                for (int c4 = 0; c4 < 4; ++c4) {
+                for (int c4 = 0; c4 < kTcD / 32; ++c4) {
                     float v[32];
-                    tmem_ld32(lane_addr + 256 + 32 * c4, v);
+                    tmem_ld32(o_addr + 32 * c4, v);
                     tmem_wait_ld();
                     if (store) {
 #pragma unroll
@@ -451,7 +486,7 @@ __global__ void __launch_bounds__(192, 1)
     // ---- every role is done with TMEM and the ring
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == kMma) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
     }
@@ -462,8 +497,8 @@ cudaError_t launch_prefill_tc(const CUtensorMap& tmQ, const CUtensorMap& tmK, co
     const int smem = kTcSmem + 1024;
     cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    const int tiles = (max_query_len + kTcRows - 1) / kTcRows;
-    return launch_pdl(prefill_tc_kernel, dim3(tiles, p.num_seqs, p.num_heads), dim3(192), smem, stream, tmQ, tmK,
+    const int tiles = (max_query_len + kTcQT * kTcRows - 1) / (kTcQT * kTcRows);
+    return launch_pdl(prefill_tc_kernel, dim3(tiles, p.num_seqs, p.num_heads), dim3(320), smem, stream, tmQ, tmK,
                       tmV, p);
 }
 
