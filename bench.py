@@ -27,6 +27,11 @@ multi-token KV write, then causal paged attention over them; metric TFLOP/s of
 the causal attention (4 * Hq * D * sum over query rows of keys attended),
 roofline against the measured dense bf16 tensor peak.
 
+--workload beam measures the beam-search step (a separate line): the host
+block-manager work of every step (forks, frees, appends with copy-on-write,
+tables, prefix groups) is done ahead and timed apart; the timed device step is
+copy-on-write copies + KV write + shared-prefix decode with that step's inputs.
+
 --swap measures block swap instead (a separate line, not the headline): a
 quarter of the gqa70b batch (64 sequences x 4,096 tokens, 1 GiB of K+V) moves
 from scattered device blocks to a page-locked host pool and back through
@@ -64,6 +69,9 @@ DESCR = {
     "fp8_long": "FP8 E4M3 cache, GQA 32/8, head_dim 128, 128 seqs, lengths log-U[256, 32768], write + split decode",
     "prefill70b": "prompt pass, Llama-3.1-70B shape: 64 q / 8 kv heads, head_dim 128, bf16, 16 prompts of "
                   "U[512, 4096] tokens: multi-token KV write + causal paged attention",
+    "beam": "beam search: 16 requests x 4 beams over a 1000-token prompt, GQA 32/8, head_dim 128, bf16; every "
+            "step forks the kept beams, frees the old ones, copies shared partial blocks on write, writes one token "
+            "per beam and decodes (shared-prefix decode)",
 }
 
 
@@ -679,6 +687,129 @@ def run_prefill(args, w0, device, rank, world):
         print(json.dumps(line), flush=True)
 
 
+class BeamStep:
+    """A beam-search trace: host decisions for every step prepared ahead (their
+    host time measured), device inputs of every step resident before timing."""
+
+    def __init__(self, w, device, total_steps):
+        import paged_kv_cache_404_b200 as pkv
+        self.pkv, self.w, self.device = pkv, w, device
+        R, B, P = w.num_prompts, w.samples, w.prefix_len
+        self.S = R * B
+        NB = W.pool_blocks(w, R * (-(-P // 16)) + R * B * (total_steps // 16 + 3))
+        bm = pkv.BlockManager(NB, 16, free_order=W.free_order(w, NB))
+        self.k_pool, self.v_pool = W.stale_fill(w, NB, device)
+        pk, pv = W.logical_kv(w, R * P, device, stream=50)
+        beams = []
+        for r in range(R):
+            p = bm.alloc_seq(P)
+            pkv.paged_kv_write(pk[r * P:(r + 1) * P], pv[r * P:(r + 1) * P],
+                               torch.from_numpy(bm.slots(p, 0, P)).to(device), self.k_pool, self.v_pool)
+            beams.append([p] + [bm.fork(p) for _ in range(B - 1)])
+        beams = np.asarray(beams, dtype=np.int32)
+        self.max_len = P + total_steps
+        maxb = -(-self.max_len // 16)
+        self.steps, host_s, self.pairs_total = [], 0.0, 0
+        for t in range(total_steps):
+            t0 = time.perf_counter()
+            parents = W.beam_parents(w, t)
+            # every request's kept beams fork from its current ones, then the old beams go
+            par = np.take_along_axis(beams, parents, axis=1).ravel()
+            kids = bm.fork_many(par)
+            bm.free_many(beams.ravel())
+            beams = kids.reshape(R, B)
+            flat = kids
+            slots, pairs = bm.append_tokens(flat)
+            tabs, lens = bm.tables(flat, maxb, pad=-1)
+            offs, mem, sh = bm.prefix_groups(flat)
+            host_s += time.perf_counter() - t0
+            g = lambda a, dt=torch.int32: torch.from_numpy(np.asarray(a)).to(device=device, dtype=dt)  # noqa: E731
+            self.steps.append(dict(slots=g(slots, torch.int64), pairs=g(pairs, torch.int64) if len(pairs) else None,
+                                   tables=g(tabs), lens=g(lens), offs=g(offs), mem=g(mem), sh=g(sh),
+                                   kv_bytes=int(lens.astype(np.int64).sum()) * w.num_kv_heads * w.head_dim * 2 * 2,
+                                   npairs=len(pairs)))
+            self.pairs_total += len(pairs)
+        self.host_us_per_step = 1e6 * host_s / total_steps
+        self.k_new, self.v_new = W.new_tokens(w, self.S, device)
+        self.q = W.queries(w, self.S, device)
+        self.out = torch.empty_like(self.q)
+        self.ws = pkv.decode_workspace(self.S, w.num_heads, w.head_dim, self.max_len, 0, device=device, shared=True)
+        self.err = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def copy_and_write(self, t):
+        st = self.steps[t]
+        if st["pairs"] is not None:
+            self.pkv.copy_blocks(self.k_pool, self.v_pool, st["pairs"], err_count=self.err)
+        self.pkv.paged_kv_write(self.k_new, self.v_new, st["slots"], self.k_pool, self.v_pool, err_count=self.err)
+
+    def decode(self, t):
+        st = self.steps[t]
+        self.pkv.paged_attention_decode_shared(self.out, self.q, self.k_pool, self.v_pool, st["tables"], st["lens"],
+                                               self.w.scale, self.max_len, self.ws, st["offs"], st["mem"], st["sh"],
+                                               err_count=self.err)
+
+
+def run_beam(args, w0, device, rank, world):
+    w = rank_workload(w0, rank)
+    step = BeamStep(w, device, args.warmup + args.steps)
+    stream = torch.cuda.current_stream()
+    for t in range(args.warmup):
+        step.copy_and_write(t)
+        step.decode(t)
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    with ClockSampler(device) as clk:
+        a0 = torch.cuda.Event(enable_timing=True)
+        z0 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for i, (a, b, c) in enumerate(ev):
+            t = args.warmup + i
+            a.record(stream)
+            step.copy_and_write(t)
+            b.record(stream)
+            step.decode(t)
+            c.record(stream)
+        z0.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    total_ms = reduce_max(a0.elapsed_time(z0), world, device)
+    timed = step.steps[args.warmup:]
+    kv = sum(st["kv_bytes"] for st in timed)
+    value = kv * world / (total_ms / 1e3) / 1e9
+    dec_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
+    cw_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
+    peak, peak_kind = measured_peak_hbm()
+    achieved = kv / args.steps / (dec_ms / 1e3) / 1e9
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = cpu_baseline(w0)
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) K/V/q, seeded beam choices and block placement)",
+            "config": {"workload": "beam: " + DESCR["beam"], "global_batch": step.S * world,
+                       "seq_len": step.max_len, "parallelism": "replicas: requests sharded by rank, no collective",
+                       "l2": "logical KV bytes counted (the prompt is shared by the 4 beams of a request)"},
+            "us_decode": round(1e3 * dec_ms, 2), "us_copy_and_write": round(1e3 * cw_ms, 2),
+            "copy_pairs_per_step": round(sum(st["npairs"] for st in timed) / args.steps, 2),
+            "host_block_manager_us_per_step": round(step.host_us_per_step, 1),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": None,
+                         "kernel": "paged_attention_decode_shared call (logical bytes; shared prompt read once per "
+                                   "request)", "peak_source": peak_kind},
+            "cpu_baseline": cpu, "e2e": None, "gpu_launches": sum(4 + (st["npairs"] > 0) for st in timed),
+            "device_errors": int(step.err.item()), "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+
+
 def run_swap(args, device):
     """Swap-out and swap-in throughput of pkv_swap_blocks over the host link."""
     import paged_kv_cache_404_b200 as pkv
@@ -790,7 +921,7 @@ def main(argv=None):
     if args.swap:
         run_swap(args, torch.device("cuda", local))
         return
-    if args.workload == "prefill70b":
+    if args.workload in ("prefill70b", "beam"):
         if world > 1:
             import datetime
             import torch.distributed as dist
@@ -798,7 +929,10 @@ def main(argv=None):
                                     device_id=torch.device("cuda", local))
             dist.barrier()
             pkv_build.build()
-        run_prefill(args, w0, torch.device("cuda", local), rank, world)
+        if args.workload == "prefill70b":
+            run_prefill(args, w0, torch.device("cuda", local), rank, world)
+        else:
+            run_beam(args, w0, torch.device("cuda", local), rank, world)
         if world > 1:
             import torch.distributed as dist
             dist.barrier()

@@ -353,6 +353,12 @@ void pkv_bm_destroy(pkv_block_manager* bm);
 int pkv_bm_alloc_seq(pkv_block_manager* bm, int num_tokens, int32_t* seq_out);
 /* New sequence sharing every block of `parent` (reference counts + 1). */
 int pkv_bm_fork(pkv_block_manager* bm, int32_t parent, int32_t* child_out);
+/* Batched fork / free (one call for a whole step of beam search): fork_many
+ * forks parents[i] into children_out[i] in order; free_many frees seqs[0..n)
+ * in order (each at most once).  Arguments are checked before anything
+ * changes. */
+int pkv_bm_fork_many(pkv_block_manager* bm, const int32_t* parents, int n, int32_t* children_out);
+int pkv_bm_free_many(pkv_block_manager* bm, const int32_t* seqs, int n);
 /* Reserve one new token slot for each of seqs[0..n) in that order.  slots_out
  * [n] receives the slots; cow_pairs_out [n][2] receives the (src, dst) block
  * pairs to copy before writing (num_pairs_out of them).  On PKV_ENOMEM the

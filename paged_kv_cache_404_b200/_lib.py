@@ -34,6 +34,8 @@ SIGNATURES = {
     "pkv_bm_destroy": (None, [_p]),
     "pkv_bm_alloc_seq": (_i, [_p, _i, _p]),
     "pkv_bm_fork": (_i, [_p, C.c_int32, _p]),
+    "pkv_bm_fork_many": (_i, [_p, _p, _i, _p]),
+    "pkv_bm_free_many": (_i, [_p, _p, _i]),
     "pkv_bm_append_tokens": (_i, [_p, _p, _i, _p, _p, _p, _p]),
     "pkv_bm_free_seq": (_i, [_p, C.c_int32]),
     "pkv_bm_num_free": (_i, [_p]),

@@ -45,6 +45,17 @@ class BlockManager:
         L.check("pkv_bm_fork", self._lib.pkv_bm_fork(self._h, int(parent), C.byref(out)))
         return out.value
 
+    def fork_many(self, parents):
+        """Fork every parent, in order; returns the children (int32 array)."""
+        par = np.ascontiguousarray(parents, dtype=np.int32)
+        out = np.empty(max(par.size, 1), dtype=np.int32)
+        L.check("pkv_bm_fork_many", self._lib.pkv_bm_fork_many(self._h, par.ctypes.data, par.size, out.ctypes.data))
+        return out[:par.size].copy()
+
+    def free_many(self, seqs):
+        s = np.ascontiguousarray(seqs, dtype=np.int32)
+        L.check("pkv_bm_free_many", self._lib.pkv_bm_free_many(self._h, s.ctypes.data, s.size))
+
     def append_tokens(self, seqs):
         """One new slot per sequence, in order. Returns (slots int64 [n], cow pairs int64 [k, 2])."""
         seqs = np.ascontiguousarray(seqs, dtype=np.int32)

@@ -187,6 +187,28 @@ int pkv_bm_fork(pkv_block_manager* bm, int32_t parent, int32_t* child_out) {
     return PKV_OK;
 }
 
+int pkv_bm_fork_many(pkv_block_manager* bm, const int32_t* parents, int n, int32_t* children_out) {
+    if (bm == nullptr || n < 0 || (n > 0 && (parents == nullptr || children_out == nullptr))) return PKV_EINVAL;
+    for (int i = 0; i < n; ++i)
+        if (int st = bm->resident(parents[i])) return st;  // checked first: nothing changes on error
+    for (int i = 0; i < n; ++i) {
+        int st = pkv_bm_fork(bm, parents[i], &children_out[i]);
+        if (st != PKV_OK) return st;
+    }
+    return PKV_OK;
+}
+
+int pkv_bm_free_many(pkv_block_manager* bm, const int32_t* seqs, int n) {
+    if (bm == nullptr || n < 0 || (n > 0 && seqs == nullptr)) return PKV_EINVAL;
+    for (int i = 0; i < n; ++i) {
+        if (!bm->valid_seq(seqs[i])) return PKV_ENOENT;
+        for (int j = 0; j < i; ++j)
+            if (seqs[j] == seqs[i]) return PKV_EINVAL;  // a sequence listed twice
+    }
+    for (int i = 0; i < n; ++i) pkv_bm_free_seq(bm, seqs[i]);
+    return PKV_OK;
+}
+
 int pkv_bm_append_tokens(pkv_block_manager* bm, const int32_t* seqs, int n, int64_t* slots_out,
                          int64_t* cow_pairs_out, int* num_pairs_out, int* num_done_out) {
     if (bm == nullptr || n < 0 || (n > 0 && (seqs == nullptr || slots_out == nullptr || cow_pairs_out == nullptr)))

@@ -52,6 +52,7 @@ constexpr int kTcSmem = kTcKV + kTcStages * 2 * kTcKVBytes;  // 192 KB
 // TMEM columns: S of Q tile t at t*64, O of Q tile t at 128 + t*128
 constexpr int kTcSCol = 0, kTcOCol = 128;
 constexpr float kRescaleThreshold = 8.f;       // log2 of the largest factor p may exceed 1 by
+constexpr int kTcOkWords = 64;                 // validity bits kept in shared memory for 2048 blocks
 
 // ---- tcgen05 wrappers -----------------------------------------------------------
 
@@ -137,6 +138,7 @@ __global__ void __launch_bounds__(320, 1)
     __shared__ __align__(8) uint64_t bars[16];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
+    __shared__ uint32_t ok_bits[kTcOkWords];  // block b of the sequence holds tokens (table, id in range)
     volatile int* abort_flag = &abort_sh;
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
     const uint32_t b0 = smem_u32(&bars[0]);
@@ -354,6 +356,19 @@ __global__ void __launch_bounds__(320, 1)
         float m_ref = -INFINITY, l = 0.f;
         bool alive = true;
         const int nt = ntq[t];
+        // validity of the blocks this CTA reads, once, into shared memory (both
+        // warpgroups together; the named barrier counts their 256 threads only)
+        const int nblk_cta = min(nblk_seq, (last_pos / kBlockSize) + 1);
+        const bool bits_in_smem = nblk_cta <= 32 * kTcOkWords;
+        if (bits_in_smem) {
+            for (int w = threadIdx.x; w < kTcOkWords; w += 256) ok_bits[w] = 0u;
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            for (int b = threadIdx.x; b < nblk_cta; b += 256) {
+                const int id = __ldg(tab + b);
+                if (id >= 0 && id < p.num_blocks) atomicOr(&ok_bits[b >> 5], 1u << (b & 31));
+            }
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+        }
         for (int j = 0; j < nt; ++j) {
             if (*abort_flag) {
                 alive = false;
@@ -361,11 +376,15 @@ __global__ void __launch_bounds__(320, 1)
             }
             // blocks of this tile that hold tokens (in the table, id in range)
             unsigned okmask = 0;
+            if (bits_in_smem) {
+                okmask = (ok_bits[(j * kTcBlocks) >> 5] >> ((j * kTcBlocks) & 31)) & ((1u << kTcBlocks) - 1u);
+            } else {
 #pragma unroll
-            for (int b = 0; b < kTcBlocks; ++b) {
-                const int jb = j * kTcBlocks + b;
-                const int id = jb < nblk_seq ? __ldg(tab + jb) : -1;
-                if (id >= 0 && id < p.num_blocks) okmask |= 1u << b;
+                for (int b = 0; b < kTcBlocks; ++b) {
+                    const int jb = j * kTcBlocks + b;
+                    const int id = jb < nblk_seq ? __ldg(tab + jb) : -1;
+                    if (id >= 0 && id < p.num_blocks) okmask |= 1u << b;
+                }
             }
             const bool w1 = mbar_wait_bounded(s_full + 8 * t, j & 1);
             if (!__all_sync(0xffffffffu, w1)) {
@@ -382,22 +401,25 @@ __global__ void __launch_bounds__(320, 1)
                 for (int i = 0; i < 32; ++i) x[32 * c2 + i] = v[i];
             }
             tmem_wait_ld();
-            float mx = -INFINITY;
             const int k0 = j * kTcKeys;
             if (k0 + kTcKeys - 1 <= qpos && okmask == (1u << kTcBlocks) - 1u) {
 #pragma unroll
-                for (int c = 0; c < kTcKeys; ++c) {
-                    x[c] *= p.score_scale;
-                    mx = fmaxf(mx, x[c]);
-                }
+                for (int c = 0; c < kTcKeys; ++c) x[c] *= p.score_scale;
             } else {
 #pragma unroll
                 for (int c = 0; c < kTcKeys; ++c) {
                     const bool valid = k0 + c <= qpos && ((okmask >> (c >> 4)) & 1u);
                     x[c] = valid ? x[c] * p.score_scale : -INFINITY;
-                    mx = fmaxf(mx, x[c]);
                 }
             }
+            // max as 8 independent chains, then a tree (short dependency chains)
+            float mx8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mx8[i] = x[i];
+#pragma unroll
+            for (int c = 8; c < kTcKeys; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);
+            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
             // the reference max moves only when a score exceeds it by more than 2^8
             float alpha = 1.f;
             const bool move = mx > m_ref + kRescaleThreshold || m_ref == -INFINITY;
@@ -406,13 +428,14 @@ __global__ void __launch_bounds__(320, 1)
             const float mu = m_new == -INFINITY ? 0.f : m_new;
             // P row as bf16 (computed before waiting for the previous PV)
             uint32_t pw[kTcKeys / 2];
-            float sum = 0.f;
+            float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int e = 0; e < kTcKeys / 2; ++e) {
                 const float p0 = fast_exp2(x[2 * e] - mu), p1 = fast_exp2(x[2 * e + 1] - mu);
-                sum += p0 + p1;
+                sum8[e & 7] += p0 + p1;
                 pw[e] = pack_bf16x2(p0, p1);
             }
+            const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
             // PV_{j-1} must be done before P is overwritten and before O is read
             if (j > 0) {
                 const bool w2 = mbar_wait_bounded(pv_done + 8 * t, (j - 1) & 1);

@@ -288,3 +288,66 @@ def test_prefix_cache_traces_match_reference(BM, seed):
             _same_state(bm, ref, live)
             assert bm.num_cached_blocks() == len(ref.cache)
     _same_state(bm, ref, live)
+
+
+def test_beam_search_trace_matches_reference(BM):
+    """The full beam workload's allocator trace (16 requests x 4 beams, 48 steps
+    of fork / free / append with copy-on-write) on both managers."""
+    import workloads as W
+    w = W.WORKLOADS["beam"]
+    R, B = w.num_prompts, w.samples
+    NB = R * (-(-w.prefix_len // 16)) + R * B * (w.len_hi // 16 + 3)
+    order = W.free_order(w, NB)
+    bm, ref = BM(NB, 16, free_order=order), RefBlockManager(NB, 16, free_order=order)
+    beams = []
+    for r in range(R):
+        p = bm.alloc_seq(w.prefix_len)
+        assert ref.alloc_seq(w.prefix_len) == p
+        kids = [bm.fork(p) for _ in range(B - 1)]
+        assert [ref.fork(p) for _ in range(B - 1)] == kids
+        beams.append([p] + kids)
+    pairs_total = 0
+    for t in range(w.len_hi):
+        parents = W.beam_parents(w, t)
+        new = []
+        for r, old in enumerate(beams):
+            kids = [bm.fork(old[int(q)]) for q in parents[r]]
+            assert [ref.fork(old[int(q)]) for q in parents[r]] == kids
+            for s in old:
+                bm.free_seq(s)
+                ref.free_seq(s)
+            new.append(kids)
+        beams = new
+        flat = [s for kids in beams for s in kids]
+        slots, pairs = bm.append_tokens(flat)
+        res = [ref.append_token(s) for s in flat]
+        assert slots.tolist() == [x[0] for x in res]
+        assert [tuple(x) for x in pairs.tolist()] == [x[1] for x in res if x[1] is not None]
+        pairs_total += len(pairs)
+        if t % 8 == 0:
+            _same_state(bm, ref, flat)
+    _same_state(bm, ref, [s for kids in beams for s in kids])
+    assert pairs_total > 0
+
+
+def test_fork_many_and_free_many_equal_single_calls(BM):
+    from paged_kv_cache_404_b200 import PagedKVError
+    a, b = BM(64, 16), BM(64, 16)
+    for m in (a, b):
+        m.alloc_seq(40)
+        m.alloc_seq(17)
+    kids_a = a.fork_many([0, 1, 0, 0])
+    kids_b = [b.fork(p) for p in [0, 1, 0, 0]]
+    assert kids_a.tolist() == kids_b
+    a.free_many([0, 3])
+    b.free_seq(0)
+    b.free_seq(3)
+    assert a.free_list().tolist() == b.free_list().tolist()
+    for blk in range(64):
+        assert a.refcount(blk) == b.refcount(blk)
+    with pytest.raises(PagedKVError):
+        a.free_many([2, 2])            # listed twice: nothing freed
+    assert a.seq_len(2) == 40
+    with pytest.raises(PagedKVError):
+        a.fork_many([1, 99])           # unknown parent: nothing forked
+    assert a.fork_many([1]).tolist() == [6]

@@ -17,6 +17,9 @@ Workloads are shaped like the PagedAttention pages' examples:
 - "fp8_long": FP8 E4M3 cache, log-uniform context lengths 256..32,768.
 - "prefill70b": the prompt pass of the Llama-3.1-70B shape: 16 prompts of
   512..4,096 tokens written into blocks and attended causally.
+- "beam": beam search, 16 requests x 4 beams over a 1,000-token prompt; at
+  every step each request keeps 4 beams drawn (seeded) from its current ones:
+  forks, frees and copy-on-write at every step.
 """
 from dataclasses import dataclass, replace
 import math
@@ -64,6 +67,8 @@ WORKLOADS = {
                               num_prompts=64, samples=3, prefix_len=1000),
     "fp8_long": Workload("fp8_long", 32, 8, 128, "fp8", "bf16", 128, "loguniform", 256, 32768, seed=5),
     "prefill70b": Workload("prefill70b", 64, 8, 128, "bf16", "bf16", 16, "uniform", 512, 4096, seed=6),
+    "beam": Workload("beam", 32, 8, 128, "bf16", "bf16", 64, "beam", 0, 48, seed=7,
+                     num_prompts=16, samples=4, prefix_len=1000),
 }
 
 TINY_LENS = (1, 15, 16, 40)
@@ -89,6 +94,9 @@ def context_lens(w: Workload) -> np.ndarray:
         return rng.integers(w.len_lo, w.len_hi + 1, size=w.num_seqs).astype(np.int32)
     if w.lens == "const":
         return np.full(w.num_seqs, w.len_lo, dtype=np.int32)
+    if w.lens == "beam":
+        # every beam has the same length; this is the one half-way through the trace
+        return np.full(w.num_seqs, w.prefix_len + w.len_hi // 2 + 1, dtype=np.int32)
     if w.lens == "loguniform":
         u = rng.uniform(math.log(w.len_lo), math.log(w.len_hi), size=w.num_seqs)
         return np.minimum(np.floor(np.exp(u)), w.len_hi).astype(np.int32)
@@ -99,6 +107,14 @@ def continuation_lens(w: Workload) -> np.ndarray:
     """Shared-prefix workload: private continuation length of each sample, U{0..len_hi}."""
     rng = _np_rng(w, 2)
     return rng.integers(0, w.len_hi + 1, size=w.num_prompts * w.samples).astype(np.int32)
+
+
+def beam_parents(w: Workload, step: int) -> np.ndarray:
+    """Beam workload: for every request, which of its current beams each of the
+    next step's beams continues (int32 [num_prompts, samples], seeded draws with
+    replacement; a beam drawn by none is dropped)."""
+    rng = np.random.default_rng([w.seed, 9, step])
+    return rng.integers(0, w.samples, size=(w.num_prompts, w.samples)).astype(np.int32)
 
 
 def allocation_order(w: Workload):
