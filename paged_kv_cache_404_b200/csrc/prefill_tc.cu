@@ -295,16 +295,20 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t idesc_s = instr_desc_bf16(kTcRows, kTcKeys, false);
         const uint32_t idesc_o = instr_desc_bf16(kTcRows, kTcD, true);
         bool alive = true;
+        // descriptors of an operand's first k-step; a k-step adds its byte offset >> 4 to
+        // the start-address field (all of shared memory is below 2^18 bytes: no carry)
+        const uint64_t dq0 = smem_desc(base + kTcQ, 16, 1024), dp0 = smem_desc(base + kTcP, 16, 1024);
+        const uint64_t dkv0 = smem_desc(base + kTcKV, 16, 1024);
+        const uint64_t dvv0 = smem_desc(base + kTcKV + kTcKVBytes, kTcKVChunk, 1024);
         auto kv_landed = [&](int j) { return mbar_wait_bounded(kv_full + 8 * (j % kTcStages), (j / kTcStages) & 1); };
         auto issue_s = [&](int t, int j) {
             tc_fence_after();
-            const uint32_t kb = base + kTcKV + (j % kTcStages) * 2 * kTcKVBytes;
-            const uint32_t qb = base + kTcQ + t * kTcQBytes;
+            const uint64_t dk = dkv0 + (uint64_t)(((j % kTcStages) * 2 * kTcKVBytes) >> 4);
+            const uint64_t dq = dq0 + (uint64_t)((t * kTcQBytes) >> 4);
 #pragma unroll
             for (int ks = 0; ks < kTcD / 16; ++ks) {
-                umma_ss(tmem + kTcSCol + t * kTcKeys,
-                        smem_desc(qb + (ks >> 2) * kTcQChunk + (ks & 3) * 32, 16, 1024),
-                        smem_desc(kb + (ks >> 2) * kTcKVChunk + (ks & 3) * 32, 16, 1024), idesc_s, ks > 0);
+                umma_ss(tmem + kTcSCol + t * kTcKeys, dq + (uint64_t)((((ks >> 2) * kTcQChunk) + (ks & 3) * 32) >> 4),
+                        dk + (uint64_t)((((ks >> 2) * kTcKVChunk) + (ks & 3) * 32) >> 4), idesc_s, ks > 0);
             }
             umma_commit(s_full + 8 * t);
         };
@@ -312,11 +316,12 @@ __global__ void __launch_bounds__(320, 1)
             if (!mbar_wait_bounded(p_full + 8 * t, j & 1)) return false;
             if (!mbar_wait_bounded(v_ready + 8 * (j % kTcStages), (j / kTcStages) & 1)) return false;
             tc_fence_after();
-            const uint32_t vb = base + kTcKV + (j % kTcStages) * 2 * kTcKVBytes + kTcKVBytes;
+            const uint64_t dv = dvv0 + (uint64_t)(((j % kTcStages) * 2 * kTcKVBytes) >> 4);
+            const uint64_t dp = dp0 + (uint64_t)((t * kTcPBytes) >> 4);
 #pragma unroll
             for (int ks = 0; ks < kTcKeys / 16; ++ks) {
-                umma_ss(tmem + kTcOCol + t * kTcD, smem_desc(base + kTcP + t * kTcPBytes + ks * 32, 16, 1024),
-                        smem_desc(vb + ks * 16 * 128, kTcKVChunk, 1024), idesc_o, j > 0 || ks > 0);
+                umma_ss(tmem + kTcOCol + t * kTcD, dp + (uint64_t)((ks * 32) >> 4),
+                        dv + (uint64_t)((ks * 16 * 128) >> 4), idesc_o, j > 0 || ks > 0);
             }
             umma_commit(pv_done + 8 * t);
             return true;
