@@ -108,9 +108,13 @@ def measured_peak_hbm():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash():
+DECODE_SOURCES = ("decode_tc.cu", "pkv_common.cuh", "decode_plan.cu", "api.cu")
+PREFILL_SOURCES = ("prefill_tc.cu", "pkv_common.cuh", "api.cu")
+
+
+def kernel_source_hash(files=DECODE_SOURCES):
     h = hashlib.sha256()
-    for f in ("decode_tc.cu", "pkv_common.cuh", "decode_plan.cu", "api.cu"):
+    for f in files:
         with open(os.path.join(ROOT, "paged_kv_cache_404_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -125,7 +129,8 @@ def ncu_traffic(workload):
             rec = json.load(f).get(workload)
     except Exception:  # noqa: BLE001
         return None
-    if not rec or rec.get("source_hash") != kernel_source_hash():
+    files = PREFILL_SOURCES if workload == "prefill70b" else DECODE_SOURCES
+    if not rec or rec.get("source_hash") != kernel_source_hash(files):
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -408,9 +413,10 @@ def oracle_sample_step(w: W.Workload, num_seqs: int, seed_offset=0):
     """Oracle inputs for `num_seqs` sequences of the workload (host, CPU
     generator): pool, tables, lengths, q and the step's new tokens."""
     import oracle
-    lens = W.context_lens(w)
     if w.lens == "shared":
         lens = (w.prefix_len + W.continuation_lens(w) + 1).astype(np.int32)
+    else:
+        lens = W.context_lens(w)
     lens = lens[seed_offset:seed_offset + num_seqs]
     wn = W.scaled(w, num_seqs=len(lens))
     need = int(sum(-(-int(L) // 16) for L in lens))
@@ -571,7 +577,7 @@ def prefill_cpu_baseline(w, target_s=12.0):
     import oracle
     rng = np.random.default_rng(7)
     lens = W.context_lens(w)
-    L = int(lens[0])
+    L = int(lens.max())   # rows of the longest prompt: the costliest per row
     NB = -(-L // 16)
     tabs = np.arange(NB, dtype=np.int32)[None]
     g = torch.Generator().manual_seed(1234)
@@ -679,7 +685,7 @@ def run_prefill(args, w0, device, rank, world):
             "prompt_tokens_per_s": round(step.total * world * args.steps / (total_ms / 1e3), 1),
             "us_attention": round(1e3 * att_ms, 2), "us_write": round(1e3 * wr_ms, 2),
             "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                         "frac": round(achieved / peak, 4), "traffic": None,
+                         "frac": round(achieved / peak, 4), "traffic": ncu_traffic("prefill70b"),
                          "kernel": "prefill_tc_kernel (tcgen05.mma, TMEM accumulators)" if os.environ.get("PKV_PREFILL_KERNEL", "")[:1] != "m" else "prefill_kernel (mma.sync m16n8k16)", "peak_source": peak_kind},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps, "device_errors": int(step.err.item()),
             "clocks": clk.summary(),
@@ -867,6 +873,22 @@ def run_swap(args, device):
     ok = bool(torch.equal(dk[torch.from_numpy(probe[:, 1]).to(device)].cpu(), hk[torch.from_numpy(probe[:, 0])]))
     ok = ok and int(err.item()) == 0
     gbs = lambda ms: round(nbytes / (ms / 1e3) / 1e9, 2)  # noqa: E731
+    # the oracle's block copy between host pools, on this host, for a bounded sample of the pairs
+    cpu = None
+    if not args.no_cpu_baseline:
+        import oracle
+        nsamp = min(len(out_pairs), 4096)
+        hk_np = hk.view(torch.int16).numpy()
+        hv_np = hv.view(torch.int16).numpy()
+        dk_h = dk[:nsamp * 2].cpu().view(torch.int16).numpy()
+        dv_h = dv[:nsamp * 2].cpu().view(torch.int16).numpy()
+        samp = np.stack([np.arange(nsamp) * 2, np.arange(nsamp)], axis=1).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.swap_blocks(hk_np, hv_np, dk_h, dv_h, samp)
+        dt = time.perf_counter() - t0
+        cpu = {"value": round(2 * nsamp * dk[0].numel() * 2 / dt / 1e9, 3), "unit": "GB/s", "cores": 1,
+               "kind": "oracle", "sample": "%d block pairs (K and V, %d KiB each) host pool to host pool, %.3f s" % (
+                   nsamp, dk[0].numel() * 2 // 1024, dt)}
     line = {
         "metric": "block swap over the host link: GB/s (K+V bytes moved / time)",
         "value": round(2 * nbytes / ((out_ms + in_ms) / 1e3) / 1e9, 2),
@@ -883,7 +905,7 @@ def run_swap(args, device):
                      "peak": round(2 * nbytes / ((d2h_ms + h2d_ms) / 1e3) / 1e9, 2), "unit": "GB/s",
                      "frac": round((d2h_ms + h2d_ms) / (out_ms + in_ms), 4),
                      "peak_source": "contiguous cudaMemcpyAsync of the same bytes, measured in this run"},
-        "gpu_launches": 2 * reps, "bytes_restored": ok, "clocks": clk.summary(),
+        "gpu_launches": 2 * reps, "bytes_restored": ok, "cpu_baseline": cpu, "clocks": clk.summary(),
     }
     print(json.dumps(line), flush=True)
 
