@@ -151,3 +151,14 @@ def test_warp_mma_kernel_agrees(tmp_path):
     env = dict(os.environ, PKV_PREFILL_KERNEL="mma")
     r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout[-2000:] + r.stderr[-2000:]
+
+
+def test_sequences_without_queries_and_oversized_launch():
+    """A sequence with no new tokens between others, and max_query_len above the
+    longest: nothing is written for the empty one, the others match the oracle."""
+    c = PrefillCase(16, 4, [50, 40, 90], [20, 0, 90], seed=45)
+    got = out_to_f64(c.run(max_query_len=300))
+    ref, bad = c.oracle()
+    assert bad == 0 and int(c.err.item()) == 0
+    assert c.qs.tolist() == [0, 20, 20, 110]
+    assert_close(got, ref, "bf16", "empty query list")

@@ -230,3 +230,26 @@ def test_prefix_cache_end_to_end():
                                                      np.arange(nb, dtype=np.int32)[None], lens[i:i + 1], w.scale)
         assert bad == 0
         assert_close(out_to_f64(out)[i:i + 1], ref_out, "bf16", "request %d" % i)
+
+
+@pytest.mark.parametrize("Hq,Hkv,D,dtype", [(2, 2, 64, "f32"), (16, 4, 64, "bf16"), (32, 2, 128, "bf16")])
+def test_hints_ignored_where_no_grouped_kernel_exists(Hq, Hkv, D, dtype):
+    """fp32, head_dim 64 and 16 query heads per KV head have no grouped kernel:
+    the shared entry point runs the plain decode (in its own workspace layout)
+    and gives the plain decode's bits."""
+    import paged_kv_cache_404_b200 as pkv
+    w = W.Workload("hint", Hq, Hkv, D, dtype, dtype, 3, "uniform", 1, 1, seed=13)
+    bm, ids, kp, vp, tabs, lens = _fork_family(w, 2, 150, [0, 7, 60], seed=13)
+    offs, mem, sh = bm.prefix_groups(ids)
+    assert len(sh) == 1
+    q = W.queries(w, 3, "cuda")
+    g_t, g_l = torch.from_numpy(tabs).cuda(), torch.from_numpy(lens).cuda()
+    max_len = int(lens.max())
+    out, err, ws = _grouped(q, kp, vp, g_t, g_l, w.scale, max_len, offs, mem, sh)
+    assert err == 0 and _hdr(ws)[1] == 0
+    plain = torch.empty_like(q)
+    ws2 = pkv.decode_workspace(3, Hq, D, max_len)
+    pkv.paged_attention_decode(plain, q, kp, vp, g_t, g_l, w.scale, max_len, ws2)
+    torch.cuda.synchronize()
+    bits = torch.int32 if dtype == "f32" else torch.int16
+    assert torch.equal(out.view(bits), plain.view(bits))
