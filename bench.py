@@ -197,7 +197,7 @@ class ClockSampler:
 class Step:
     """Device-resident inputs of one decode step and the calls that run it."""
 
-    def __init__(self, w: W.Workload, device, partition=0, prefix_groups=True):
+    def __init__(self, w: W.Workload, device, partition=0, prefix_groups=True, cont=None):
         import paged_kv_cache_404_b200 as pkv
         self.pkv = pkv
         self.w = w
@@ -205,7 +205,7 @@ class Step:
         self.partition = partition
         self.groups = None
         if w.lens == "shared":
-            self._setup_shared()
+            self._setup_shared(cont)
         else:
             self._setup_flat()
         self.max_len = int(self.lens.max())
@@ -248,11 +248,13 @@ class Step:
         self.k_new, self.v_new = W.new_tokens(w, self.S, dev)
         self.NB = NB
 
-    def _setup_shared(self):
+    def _setup_shared(self, cont=None):
         """Prompts written once and forked; continuations replayed token by token
-        (copy-on-write on first divergence); the step is the next token of all."""
+        (copy-on-write on first divergence); the step is the next token of all.
+        cont: continuation lengths (default: the workload's; all zero makes the
+        step the divergence step, where every prompt's partly filled block splits)."""
         pkv, w, dev = self.pkv, self.w, self.device
-        cont = W.continuation_lens(w)
+        cont = W.continuation_lens(w) if cont is None else np.asarray(cont, np.int32)
         S = self.S = w.num_prompts * w.samples
         est = w.num_prompts * (-(-w.prefix_len // 16)) + int(sum(-(-(int(c) + 17) // 16) for c in cont)) + S
         NB = int(math.ceil(est * w.pool_factor))
@@ -277,6 +279,10 @@ class Step:
         self.slots, self.pairs = bm.append_tokens(ids)
         self.tables, self.lens = bm.tables(ids, max(-(-int(bm.seq_len(s)) // 16) for s in ids), pad=-1)
         self.groups = bm.prefix_groups(ids)
+        # memory saved by sharing: physical blocks in use vs one private copy per sequence
+        used = len({int(b) for row in self.tables for b in row if b >= 0})
+        private = int(sum(-(-int(L) // 16) for L in self.lens))
+        self.mem_saving = 1.0 - used / private
         self.k_pool, self.v_pool, self.k_scale, self.v_scale = kp, vp, 1.0, 1.0
         self.q = W.queries(w, S, dev)
         self.k_new, self.v_new = W.new_tokens(w, S, dev)
@@ -336,6 +342,30 @@ def time_steps(step: Step, steps: int, warmup: int, world: int, device):
     decode_ms = [b.elapsed_time(c) for _, b, c in ev]
     write_ms = [a.elapsed_time(b) for a, b, _ in ev]
     return total_ms, decode_ms, write_ms
+
+
+def divergence_step(w, device, args):
+    """The shared-prefix step right after the prompts: all continuations empty, so
+    every prompt's partly filled last block is copied for all but its last holder."""
+    step = Step(w, device, prefix_groups=not args.no_prefix_groups, cont=np.zeros(w.num_prompts * w.samples))
+    reps = 20
+    for _ in range(3):
+        step.run()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+    for a, b, c in ev:
+        a.record()
+        step.copy_and_write()
+        b.record()
+        step.decode()
+        c.record()
+    torch.cuda.synchronize()
+    cw = statistics.median(a.elapsed_time(b) for a, b, _ in ev)
+    dec = statistics.median(b.elapsed_time(c) for _, b, c in ev)
+    npairs = len(step.pairs)
+    block_bytes = step.k_pool[0].numel() * step.k_pool.element_size()
+    return {"copy_pairs": npairs, "copy_bytes": 2 * npairs * block_bytes, "us_copy_and_write": round(1e3 * cw, 2),
+            "us_decode": round(1e3 * dec, 2), "device_errors": int(step.err.item())}
 
 
 def time_e2e(step: Step, steps: int, warmup: int, world: int):
@@ -1021,6 +1051,9 @@ def main(argv=None):
             "gpu_launches": step.launches * args.steps, "device_errors": err,
             "clocks": clk.summary(),
         }
+        if w.lens == "shared":
+            line["memory_saving_by_sharing"] = round(step.mem_saving, 4)
+            line["divergence_step"] = divergence_step(w, device, args)
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
