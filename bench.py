@@ -25,7 +25,9 @@ sample of the same workload, on this host's cores.
 prompts of 512..4,096 tokens (Llama-3.1-70B shape) written into blocks with the
 multi-token KV write, then causal paged attention over them; metric TFLOP/s of
 the causal attention (4 * Hq * D * sum over query rows of keys attended),
-roofline against the measured dense bf16 tensor peak.
+roofline against the measured dense bf16 tensor peak.  --workload
+prefill70b_fp8 is the same pass over an FP8 E4M3 cache (the products run in
+f16, whose dense tensor rate equals bf16's).
 
 --workload beam measures the beam-search step (a separate line): the host
 block-manager work of every step (forks, frees, appends with copy-on-write,
@@ -69,6 +71,9 @@ DESCR = {
     "fp8_long": "FP8 E4M3 cache, GQA 32/8, head_dim 128, 128 seqs, lengths log-U[256, 32768], write + split decode",
     "prefill70b": "prompt pass, Llama-3.1-70B shape: 64 q / 8 kv heads, head_dim 128, bf16, 16 prompts of "
                   "U[512, 4096] tokens: multi-token KV write + causal paged attention",
+    "prefill70b_fp8": "prompt pass, Llama-3.1-70B shape: 64 q / 8 kv heads, head_dim 128, bf16 q, FP8 E4M3 cache "
+                      "(per-tensor scales), 16 prompts of U[512, 4096] tokens: multi-token KV write (quantising) + "
+                      "causal paged attention",
     "beam": "beam search: 16 requests x 4 beams over a 1000-token prompt, GQA 32/8, head_dim 128, bf16; every "
             "step forks the kept beams, frees the old ones, copies shared partial blocks on write, writes one token "
             "per beam and decodes (shared-prefix decode)",
@@ -129,7 +134,7 @@ def ncu_traffic(workload):
             rec = json.load(f).get(workload)
     except Exception:  # noqa: BLE001
         return None
-    files = PREFILL_SOURCES if workload == "prefill70b" else DECODE_SOURCES
+    files = PREFILL_SOURCES if workload.startswith("prefill") else DECODE_SOURCES
     if not rec or rec.get("source_hash") != kernel_source_hash(files):
         return None
     return rec.get("dram_bytes_per_launch")
@@ -506,7 +511,7 @@ def run_reference(args, w, rank, world):
     if rank != 0:
         return
     import oracle
-    if w.name == "prefill70b":
+    if w.name.startswith("prefill"):
         t0 = time.perf_counter()
         samples = [prefill_cpu_baseline(w, target_s=2.0) for _ in range(args.steps)]
         total = time.perf_counter() - t0
@@ -515,7 +520,7 @@ def run_reference(args, w, rank, world):
                 "value": value, "unit": "TFLOP/s", "impl": "reference", "n_gpus": world, "steps": args.steps,
                 "warmup": 0, "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": "prefill70b: " + DESCR["prefill70b"], "parallelism": "cpu (OpenMP)"},
+                "config": {"workload": w.name + ": " + DESCR[w.name], "parallelism": "cpu (OpenMP)"},
                 "cpu_baseline": dict(samples[-1], value=value),
                 "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
@@ -582,6 +587,10 @@ class PrefillStep:
         tables, self.lens = bm.tables(ids, max(-(-int(L) // 16) for L in lens), pad=-1)
         self.k_pool, self.v_pool = W.stale_fill(w, NB, device)
         self.k_new, self.v_new = W.logical_kv(w, self.total, device, stream=80)
+        self.fp8 = w.cache_dtype == "fp8"
+        # FP8: per-tensor scales amax / 448 of the prompt's K and V
+        self.k_scale = float(self.k_new.abs().max().float().item()) / 448.0 if self.fp8 else 1.0
+        self.v_scale = float(self.v_new.abs().max().float().item()) / 448.0 if self.fp8 else 1.0
         self.q = W.queries(W.scaled(w, num_seqs=self.total), self.total, device)
         self.out = torch.empty_like(self.q)
         self.g_slots = torch.from_numpy(slots.astype(np.int64)).to(device)
@@ -592,14 +601,16 @@ class PrefillStep:
         self.err = torch.zeros(1, dtype=torch.int32, device=device)
         L64 = self.lens.astype(np.float64)
         self.flops = 4.0 * w.num_heads * w.head_dim * float((L64 * (L64 + 1) / 2).sum())
-        self.kv_bytes = self.total * w.num_kv_heads * w.head_dim * 2 * 2
+        self.kv_bytes = self.total * w.num_kv_heads * w.head_dim * 2 * (1 if self.fp8 else 2)
 
     def write(self):
-        self.pkv.paged_kv_write(self.k_new, self.v_new, self.g_slots, self.k_pool, self.v_pool, err_count=self.err)
+        self.pkv.paged_kv_write(self.k_new, self.v_new, self.g_slots, self.k_pool, self.v_pool, self.k_scale,
+                                self.v_scale, err_count=self.err)
 
     def attend(self):
         self.pkv.paged_attention_prefill(self.out, self.q, self.k_pool, self.v_pool, self.g_tables, self.g_lens,
-                                         self.g_qs, self.w.scale, self.max_q, err_count=self.err)
+                                         self.g_qs, self.w.scale, self.max_q, err_count=self.err,
+                                         k_scale=self.k_scale, v_scale=self.v_scale)
 
 
 def prefill_cpu_baseline(w, target_s=12.0):
@@ -616,10 +627,17 @@ def prefill_cpu_baseline(w, target_s=12.0):
     q = torch.randn((L, w.num_heads, w.head_dim), generator=g).to(torch.bfloat16)
     bits = lambda t: t.view(torch.int16).numpy().view(np.uint16)  # noqa: E731
     qs = np.array([0, L], np.int32)
+    fp8 = w.cache_dtype == "fp8"
+    if fp8:   # E4M3 codes of the same values (scale 1: |x| < 448)
+        kb = kp.float().to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        vb = vp.float().to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    else:
+        kb, vb = bits(kp), bits(vp)
+    cdt = oracle.FP8_E4M3 if fp8 else oracle.BF16
 
     def run(rows):
         t0 = time.perf_counter()
-        oracle.paged_attention_prefill(bits(q), oracle.BF16, bits(kp), bits(vp), oracle.BF16, tabs,
+        oracle.paged_attention_prefill(bits(q), oracle.BF16, kb, vb, cdt, tabs,
                                        np.array([L], np.int32), qs, w.scale, rows=rows)
         return time.perf_counter() - t0
 
@@ -705,17 +723,18 @@ def run_prefill(args, w0, device, rank, world):
             "metric": "causal paged prefill attention TFLOP/s (4*Hq*D*keys attended per query row)",
             "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16 (fp32 accumulate)",
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16 q, fp8 e4m3 cache (f16 products, fp32 accumulate)" if step.fp8 else "bf16 (fp32 accumulate)",
             "data": "synthetic (seeded N(0,1) q/K/V, seeded block placement)",
-            "config": {"workload": "prefill70b: " + DESCR["prefill70b"], "global_batch": step.S * world,
+            "config": {"workload": w0.name + ": " + DESCR[w0.name], "global_batch": step.S * world,
                        "seq_len": step.max_q, "prompt_tokens": step.total,
                        "parallelism": "replicas: prompts sharded by rank, no collective",
                        "l2": "inputs larger than L2 (q %.0f MB + K/V %.0f MB per GPU vs 126 MB L2)" % (
-                           step.q.numel() * 2 / 1e6, 2 * step.k_pool.numel() * 2 / 1e6)},
+                           step.q.numel() * 2 / 1e6, 2 * step.k_pool.numel() * step.k_pool.element_size() / 1e6)},
             "prompt_tokens_per_s": round(step.total * world * args.steps / (total_ms / 1e3), 1),
             "us_attention": round(1e3 * att_ms, 2), "us_write": round(1e3 * wr_ms, 2),
             "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                         "frac": round(achieved / peak, 4), "traffic": ncu_traffic("prefill70b"),
+                         "frac": round(achieved / peak, 4), "traffic": ncu_traffic(w0.name),
                          "kernel": "prefill_tc_kernel (tcgen05.mma, TMEM accumulators)" if os.environ.get("PKV_PREFILL_KERNEL", "")[:1] != "m" else "prefill_kernel (mma.sync m16n8k16)", "peak_source": peak_kind},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps, "device_errors": int(step.err.item()),
             "clocks": clk.summary(),
@@ -973,7 +992,7 @@ def main(argv=None):
     if args.swap:
         run_swap(args, torch.device("cuda", local))
         return
-    if args.workload in ("prefill70b", "beam"):
+    if args.workload.startswith("prefill") or args.workload == "beam":
         if world > 1:
             import datetime
             import torch.distributed as dist
@@ -981,7 +1000,7 @@ def main(argv=None):
                                     device_id=torch.device("cuda", local))
             dist.barrier()
             pkv_build.build()
-        if args.workload == "prefill70b":
+        if args.workload.startswith("prefill"):
             run_prefill(args, w0, torch.device("cuda", local), rank, world)
         else:
             run_beam(args, w0, torch.device("cuda", local), rank, world)

@@ -269,11 +269,16 @@ int pkv_paged_attention_decode_shared(void* out, const void* q, int q_dtype,
  *   context_lens    int32 [num_seqs]; query_start int32 [num_seqs + 1], query_start[0] = 0,
  *                   query_start[num_seqs] = total_query_tokens
  *   max_query_len   >= every nq_s (sizes the launch; rows past it are not computed)
- * Supported: bf16 q, bf16 cache, head_dim 128, block_size 16, any GQA group.
- * The product runs on the tcgen05 tensor cores (TMEM accumulators); setting
- * the environment variable PKV_PREFILL_KERNEL=mma before the first call
- * selects the warp-level mma.sync kernel instead (same results, for
- * comparison).
+ *   k_scale, v_scale  FP8 cache only (ignored for bf16): a stored code c stands
+ *                   for c * k_scale (c * v_scale), as pkv_paged_kv_write quantised it
+ * Supported: bf16 q, bf16 or FP8 E4M3 cache, head_dim 128, block_size 16, any
+ * GQA group.  The product runs on the tcgen05 tensor cores (TMEM
+ * accumulators).  With an FP8 cache the codes become f16 in shared memory
+ * (exactly) and q is taken into f16 (exact inside the f16 range; entries past
+ * +-65504 saturate there), so both operands of every product are f16.
+ * Setting the environment variable PKV_PREFILL_KERNEL=mma before the first
+ * call selects the warp-level mma.sync kernel instead (same results, bf16
+ * cache only: an FP8 cache then returns PKV_EUNSUPPORTED; for comparison).
  * Device-data errors (a table entry out of range among the blocks a sequence
  * reads: its tokens are left out; nq_s > context_lens[s] or a context longer
  * than the table: the sequence's rows are zeroed) are counted into err_count.
@@ -284,7 +289,7 @@ int pkv_paged_attention_prefill(void* out, const void* q, int q_dtype,
                                 const int32_t* context_lens, const int32_t* query_start, int num_seqs,
                                 int total_query_tokens, int max_query_len, int num_blocks, int block_size,
                                 int num_heads, int num_kv_heads, int head_dim, float scale,
-                                int32_t* err_count, void* stream);
+                                float k_scale, float v_scale, int32_t* err_count, void* stream);
 
 /* ------------------------------------------------------------------------
  * Copy-on-write block copy: for every pair (src, dst) copy the whole physical

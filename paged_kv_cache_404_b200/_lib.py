@@ -27,7 +27,7 @@ SIGNATURES = {
     "pkv_paged_attention_decode_shared": (_i, [_p, _p, _i, _p, _p, _i, _p, _i, _p, _i, _i, _i, _i, _i, _i, _i,
                                                _f, _f, _f, _i, _p, _p, _i, _p, _i, _p, _z, _p, _p]),
     "pkv_paged_attention_prefill": (_i, [_p, _p, _i, _p, _p, _i, _p, _i, _p, _p, _i, _i, _i, _i, _i, _i, _i,
-                                         _i, _f, _p, _p]),
+                                         _i, _f, _f, _f, _p, _p]),
     "pkv_copy_blocks": (_i, [_p, _p, _z, _p, _i, _i, _p, _p]),
     "pkv_swap_blocks": (_i, [_p, _p, _i, _p, _p, _i, _z, _p, _i, _p, _p]),
     "pkv_bm_create": (_i, [_i, _i, _p, _i, C.POINTER(_p)]),

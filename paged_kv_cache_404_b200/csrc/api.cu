@@ -3,6 +3,7 @@
 // every buffer belongs to the caller.
 #include <cudaTypedefs.h>
 
+#include <cmath>
 #include <cstdlib>
 
 #include "pagedkv.h"
@@ -26,7 +27,7 @@ cudaError_t launch_decode_merge(const DecodeParams& p, int out_dtype, cudaStream
 cudaError_t launch_prefill(const CUtensorMap& tmK, const CUtensorMap& tmV, const PrefillParams& p, int max_query_len,
                            cudaStream_t stream);
 cudaError_t launch_prefill_tc(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                              const PrefillParams& p, int max_query_len, cudaStream_t stream);
+                              const PrefillParams& p, bool fp8, int max_query_len, cudaStream_t stream);
 }  // namespace pkv
 
 using namespace pkv;
@@ -351,14 +352,17 @@ int pkv_paged_attention_prefill(void* out, const void* q, int q_dtype, const voi
                                 int cache_dtype, const int32_t* block_tables, int max_blocks_per_seq,
                                 const int32_t* context_lens, const int32_t* query_start, int num_seqs,
                                 int total_query_tokens, int max_query_len, int num_blocks, int block_size,
-                                int num_heads, int num_kv_heads, int head_dim, float scale, int32_t* err_count,
-                                void* stream) {
+                                int num_heads, int num_kv_heads, int head_dim, float scale, float k_scale,
+                                float v_scale, int32_t* err_count, void* stream) {
     if (num_seqs < 0 || max_blocks_per_seq <= 0 || max_query_len < 0 || total_query_tokens < 0 || num_blocks <= 0 ||
         block_size <= 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0)
         return PKV_EINVAL;
     if (num_heads % num_kv_heads != 0) return PKV_EINVAL;
     if (block_size != kBlockSize) return PKV_EUNSUPPORTED;
-    if (q_dtype != PKV_BF16 || cache_dtype != PKV_BF16 || head_dim != 128) return PKV_EUNSUPPORTED;
+    const bool fp8 = cache_dtype == PKV_FP8_E4M3;
+    if (q_dtype != PKV_BF16 || (cache_dtype != PKV_BF16 && !fp8) || head_dim != 128) return PKV_EUNSUPPORTED;
+    if (fp8 && prefill_kernel_choice() == 1) return PKV_EUNSUPPORTED;  // the mma.sync kernel reads bf16 only
+    if (fp8 && !(std::isfinite(k_scale) && std::isfinite(v_scale))) return PKV_EINVAL;
     if (num_seqs == 0 || max_query_len == 0 || total_query_tokens == 0) return PKV_OK;
     if (num_seqs > 65535 || num_heads > 65535) return PKV_EUNSUPPORTED;
     if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens || !query_start) return PKV_EINVAL;
@@ -376,7 +380,8 @@ int pkv_paged_attention_prefill(void* out, const void* q, int q_dtype, const voi
     p.num_blocks = num_blocks;
     p.num_heads = num_heads;
     p.group = num_heads / num_kv_heads;
-    p.score_scale = scale * 1.4426950408889634f;
+    p.score_scale = scale * (fp8 ? k_scale : 1.f) * 1.4426950408889634f;
+    p.out_scale = fp8 ? v_scale : 1.f;
     p.err = err_count;
     CUtensorMap tmK, tmV;
     const long long slots = (long long)num_blocks * block_size;
@@ -390,7 +395,7 @@ int pkv_paged_attention_prefill(void* out, const void* q, int q_dtype, const voi
         // q viewed as [total_q][heads][head_dim]; boxes of 128 rows x 1 head x 128 bytes
         CUtensorMap tmQ;
         if (!rows_tensor_map(&tmQ, q, head_dim, num_heads, total_query_tokens, 128)) return PKV_ECUDA;
-        e = launch_prefill_tc(tmQ, tmK, tmV, p, max_query_len, static_cast<cudaStream_t>(stream));
+        e = launch_prefill_tc(tmQ, tmK, tmV, p, fp8, max_query_len, static_cast<cudaStream_t>(stream));
     }
     return e == cudaSuccess ? PKV_OK : PKV_ECUDA;
 }

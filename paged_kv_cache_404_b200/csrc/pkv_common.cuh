@@ -138,7 +138,8 @@ struct PrefillParams {
     int num_blocks;
     int num_heads;
     int group;
-    float score_scale;  // scale * log2(e)
+    float score_scale;  // scale * k_scale * log2(e)
+    float out_scale;    // v_scale (1 for a bf16 cache)
     int32_t* err;
 };
 

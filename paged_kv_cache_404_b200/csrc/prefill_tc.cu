@@ -8,7 +8,7 @@
 // holds).
 //
 // One CTA per (sequence, 256 query rows = two Q tiles of 128, query head); ten
-// warps:
+// warps for a bf16 cache:
 //  - warp 8 (producer): TMA-loads the two Q tiles once and, per 64-key tile, the
 //    K and V of 4 blocks of the table (16-slot x 1-head x 128-byte boxes,
 //    128-byte swizzle) into a 3-stage ring; V rows that hold no token of the context
@@ -27,6 +27,14 @@
 //    stores the rows.
 // The products are issued PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), ..., so that
 // each warpgroup's softmax runs while the tensor core works for the other.
+//
+// FP8 E4M3 cache (14 warps): the products run in f16, which holds every E4M3
+// value exactly.  Warp 8 TMA-loads the codes (128-byte rows) into a 2-deep
+// staging ring; warps 10-13 each turn one 16-slot block of a tile into f16 in the
+// ring the tensor core reads (and zero V where no token is), then arrive on the
+// stage's barriers; the softmax warps first take their Q tile from bf16 into f16
+// in place and write P as f16.  k_scale folds into the score scale and v_scale
+// into the final normalisation.
 #include "pkv_common.cuh"
 
 namespace pkv {
@@ -49,6 +57,11 @@ constexpr int kTcQ = 0;                                    // Q tile t at kTcQ +
 constexpr int kTcP = kTcQ + kTcQT * kTcQBytes;             // P tile t at kTcP + t * kTcPBytes
 constexpr int kTcKV = kTcP + kTcQT * kTcPBytes;            // stage st: K, then V
 constexpr int kTcSmem = kTcKV + kTcStages * 2 * kTcKVBytes;  // 192 KB
+// FP8 cache: E4M3 K and V tiles land in a 2-deep staging ring (64 rows x 128 bytes
+// each), then become f16 in the ring above
+constexpr int kTcStgBytes = kTcKeys * 128;
+constexpr int kTcStg = kTcSmem;
+constexpr int kTcSmemFp8 = kTcStg + 2 * 2 * kTcStgBytes;  // 224 KB
 // TMEM columns: S of Q tile t at t*64, O of Q tile t at 128 + t*128
 constexpr int kTcSCol = 0, kTcOCol = 128;
 constexpr float kRescaleThreshold = 8.f;       // log2 of the largest factor p may exceed 1 by
@@ -67,10 +80,35 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes,
     return d;
 }
 
-// Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator, M x N.
-__host__ __device__ constexpr uint32_t instr_desc_bf16(int M, int N, bool b_mn_major) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
-           ((uint32_t)(M >> 4) << 24);
+// Instruction descriptor, kind::f16: A and B both bf16 (or both f16), fp32 accumulator, M x N.
+__host__ __device__ constexpr uint32_t instr_desc_16(int M, int N, bool b_mn_major, bool f16) {
+    return (1u << 4) | ((f16 ? 0u : 1u) << 7) | ((f16 ? 0u : 1u) << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// 16 E4M3 codes (one 16-byte chunk) -> 16 f16 values in two 16-byte words (exact)
+__device__ __forceinline__ void e4m3x16_to_f16(const uint4 c, uint4& lo, uint4& hi) {
+    lo.x = e4m3x2_to_f16x2(c.x);
+    lo.y = e4m3x2_to_f16x2(c.x >> 16);
+    lo.z = e4m3x2_to_f16x2(c.y);
+    lo.w = e4m3x2_to_f16x2(c.y >> 16);
+    hi.x = e4m3x2_to_f16x2(c.z);
+    hi.y = e4m3x2_to_f16x2(c.z >> 16);
+    hi.z = e4m3x2_to_f16x2(c.w);
+    hi.w = e4m3x2_to_f16x2(c.w >> 16);
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4 v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// two bf16 (one word) -> two f16, saturating at +-65504 (exact inside the f16 normal range)
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+    uint32_t r;
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(__uint_as_float(w & 0xFFFF0000u)),
+        "f"(__uint_as_float(w << 16)));
+    return r;
 }
 
 __device__ __forceinline__ void umma_ss(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, bool accumulate) {
@@ -130,12 +168,14 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 
 }  // namespace
 
-__global__ void __launch_bounds__(320, 1)
+template <bool FP8>
+__global__ void __launch_bounds__(FP8 ? 448 : 320, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
-    // kv_full[3], kv_empty[3], v_ready[3], q_full, s_full[2], p_full[2], pv_done[2]
-    __shared__ __align__(8) uint64_t bars[16];
+    // kv_full[3], kv_empty[3], v_ready[3], q_full, s_full[2], p_full[2], pv_done[2],
+    // FP8: stg_full[2], stg_empty[2], q_ready
+    __shared__ __align__(8) uint64_t bars[21];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
     __shared__ uint32_t ok_bits[kTcOkWords];  // block b of the sequence holds tokens (table, id in range)
@@ -143,17 +183,18 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
     const uint32_t b0 = smem_u32(&bars[0]);
     const uint32_t kv_full = b0, kv_empty = b0 + 24, v_ready = b0 + 48, q_full = b0 + 72, s_full = b0 + 80,
-                   p_full = b0 + 96, pv_done = b0 + 112;
+                   p_full = b0 + 96, pv_done = b0 + 112, stg_full = b0 + 128, stg_empty = b0 + 144, q_ready = b0 + 160;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr int kProducer = 8, kMma = 9;
+    constexpr int kProducer = 8, kMma = 9, kConv0 = 10;  // FP8: warps 10-13 convert
+    constexpr int kConvWarps = kTcBlocks;
 
     const int s = blockIdx.y, h = blockIdx.z, kvh = h / p.group;
     const int tile = gridDim.x - 1 - blockIdx.x;
     if (threadIdx.x == 0) {
         for (int i = 0; i < kTcStages; ++i) {
-            mbar_init(kv_full + 8 * i, 1);
+            mbar_init(kv_full + 8 * i, FP8 ? kConvWarps : 1);
             mbar_init(kv_empty + 8 * i, 1);
-            mbar_init(v_ready + 8 * i, 1);
+            mbar_init(v_ready + 8 * i, FP8 ? kConvWarps : 1);
         }
         mbar_init(q_full, 1);
         for (int t = 0; t < kTcQT; ++t) {
@@ -161,6 +202,11 @@ __global__ void __launch_bounds__(320, 1)
             mbar_init(p_full + 8 * t, 4);
             mbar_init(pv_done + 8 * t, 1);
         }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(stg_full + 8 * i, 1);
+            mbar_init(stg_empty + 8 * i, kConvWarps);
+        }
+        mbar_init(q_ready, 8);  // FP8: each softmax warp has turned its rows of Q into f16
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -222,78 +268,194 @@ __global__ void __launch_bounds__(320, 1)
                 tma_load_3d(base + kTcQ + t * kTcQBytes + kTcQChunk, &tmQ, 64, h, qs0 + row0 + t * kTcRows, q_full);
             }
         }
-        for (int j = 0; j < ntiles && !*abort_flag; ++j) {
-            const int st = j % kTcStages, round = j / kTcStages;
-            // block ids of this tile: lanes 0..3; a block is loaded if it is in the table
-            // and its id is in range
-            const int jb = j * kTcBlocks + (lane & (kTcBlocks - 1));
-            int id = -1;
-            if (lane < kTcBlocks && jb < nblk_seq) id = __ldg(tab + jb);
-            const bool load = lane < kTcBlocks && jb < nblk_seq && id >= 0 && id < p.num_blocks;
-            if (lane < kTcBlocks && jb < nblk_seq && !load && h == 0 && jb >= count_from &&
-                jb <= last_pos / kBlockSize)
-                count_error(p.err);
-            const unsigned loaded = __ballot_sync(0xffffffffu, load);
-            bool go = true;
-            if (lane == 0 && round > 0) go = mbar_wait_bounded(kv_empty + 8 * st, (round - 1) & 1);
-            go = __shfl_sync(0xffffffffu, go, 0);
-            if (!go) {
-                if (lane == 0) {
+        if constexpr (FP8) {
+            // E4M3 tiles: TMA into a 2-deep staging ring, up to two tiles ahead of the
+            // converters (16-slot x 1-head x 128-byte boxes, 128-byte swizzle)
+            bool ok = true;
+            for (int j = 0; j < ntiles && !*abort_flag; ++j) {
+                const int jb = j * kTcBlocks + (lane & (kTcBlocks - 1));
+                int id = -1;
+                if (lane < kTcBlocks && jb < nblk_seq) id = __ldg(tab + jb);
+                const bool load = lane < kTcBlocks && jb < nblk_seq && id >= 0 && id < p.num_blocks;
+                if (lane < kTcBlocks && jb < nblk_seq && !load && h == 0 && jb >= count_from &&
+                    jb <= last_pos / kBlockSize)
                     count_error(p.err);
-                    atomicExch(&abort_sh, 1);
+                const unsigned loaded = __ballot_sync(0xffffffffu, load);
+                if (j >= 2) {
+                    bool free_slot = true;
+                    if (lane == 0) free_slot = mbar_wait_bounded(stg_empty + 8 * (j & 1), ((j >> 1) - 1) & 1);
+                    if (!(ok = __shfl_sync(0xffffffffu, free_slot, 0))) break;
                 }
-                break;
-            }
-            const uint32_t kdst = base + kTcKV + st * 2 * kTcKVBytes, vdst = kdst + kTcKVBytes;
-            if (lane == 0) mbar_arrive_expect_tx(kv_full + 8 * st, __popc(loaded) * 4 * (kBlockSize * 128));
-            __syncwarp();
-            if (load) {
-                const int row = id * kBlockSize;
-                const uint32_t off = lane * kBlockSize * 128;
-                tma_load_3d(kdst + off, &tmK, 0, kvh, row, kv_full + 8 * st);
-                tma_load_3d(kdst + kTcKVChunk + off, &tmK, 64, kvh, row, kv_full + 8 * st);
-                tma_load_3d(vdst + off, &tmV, 0, kvh, row, kv_full + 8 * st);
-                tma_load_3d(vdst + kTcKVChunk + off, &tmV, 64, kvh, row, kv_full + 8 * st);
-            }
-            // V rows with no token: whole blocks not loaded, and the slots past the context
-            // in the sequence's last block (once it has landed)
-            for (int b = 0; b < kTcBlocks; ++b) {
-                if ((loaded >> b) & 1u) continue;
-                for (int i = lane; i < kBlockSize * 16; i += 32) {
-                    const int r = b * kBlockSize + (i >> 4), c = i & 15;
-                    const uint32_t a = vdst + (c >> 3) * kTcKVChunk + r * 128 + ((c & 7) << 4);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0) : "memory");
+                const uint32_t kst = base + kTcStg + (j & 1) * 2 * kTcStgBytes, vst = kst + kTcStgBytes;
+                const uint32_t bar = stg_full + 8 * (j & 1);
+                if (lane == 0) mbar_arrive_expect_tx(bar, __popc(loaded) * 2 * (kBlockSize * 128));
+                __syncwarp();
+                if (load) {
+                    tma_load_3d(kst + lane * kBlockSize * 128, &tmK, 0, kvh, id * kBlockSize, bar);
+                    tma_load_3d(vst + lane * kBlockSize * 128, &tmV, 0, kvh, id * kBlockSize, bar);
                 }
             }
-            const int jt = (ctx % kBlockSize) ? nblk_seq - 1 : -1;
-            const int bt = jt - j * kTcBlocks;
-            if (bt >= 0 && bt < kTcBlocks && ((loaded >> bt) & 1u)) {
-                bool landed = true;
-                if (lane == 0) landed = mbar_wait_bounded(kv_full + 8 * st, round & 1);
-                if (!__shfl_sync(0xffffffffu, landed, 0)) {
+            if (!ok && lane == 0) {
+                count_error(p.err);
+                atomicExch(&abort_sh, 1);
+            }
+        } else {
+            for (int j = 0; j < ntiles && !*abort_flag; ++j) {
+                const int st = j % kTcStages, round = j / kTcStages;
+                // block ids of this tile: lanes 0..3; a block is loaded if it is in the table
+                // and its id is in range
+                const int jb = j * kTcBlocks + (lane & (kTcBlocks - 1));
+                int id = -1;
+                if (lane < kTcBlocks && jb < nblk_seq) id = __ldg(tab + jb);
+                const bool load = lane < kTcBlocks && jb < nblk_seq && id >= 0 && id < p.num_blocks;
+                if (lane < kTcBlocks && jb < nblk_seq && !load && h == 0 && jb >= count_from &&
+                    jb <= last_pos / kBlockSize)
+                    count_error(p.err);
+                const unsigned loaded = __ballot_sync(0xffffffffu, load);
+                bool go = true;
+                if (lane == 0 && round > 0) go = mbar_wait_bounded(kv_empty + 8 * st, (round - 1) & 1);
+                go = __shfl_sync(0xffffffffu, go, 0);
+                if (!go) {
                     if (lane == 0) {
                         count_error(p.err);
                         atomicExch(&abort_sh, 1);
                     }
                     break;
                 }
-                const int r0 = ctx % kBlockSize;
-                for (int i = lane; i < (kBlockSize - r0) * 16; i += 32) {
-                    const int r = bt * kBlockSize + r0 + (i >> 4), c = i & 15;
-                    const uint32_t a = vdst + (c >> 3) * kTcKVChunk + r * 128 + ((c & 7) << 4);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0) : "memory");
+                const uint32_t kdst = base + kTcKV + st * 2 * kTcKVBytes, vdst = kdst + kTcKVBytes;
+                if (lane == 0) mbar_arrive_expect_tx(kv_full + 8 * st, __popc(loaded) * 4 * (kBlockSize * 128));
+                __syncwarp();
+                if (load) {
+                    const int row = id * kBlockSize;
+                    const uint32_t off = lane * kBlockSize * 128;
+                    tma_load_3d(kdst + off, &tmK, 0, kvh, row, kv_full + 8 * st);
+                    tma_load_3d(kdst + kTcKVChunk + off, &tmK, 64, kvh, row, kv_full + 8 * st);
+                    tma_load_3d(vdst + off, &tmV, 0, kvh, row, kv_full + 8 * st);
+                    tma_load_3d(vdst + kTcKVChunk + off, &tmV, 64, kvh, row, kv_full + 8 * st);
+                }
+                // V rows with no token: whole blocks not loaded, and the slots past the context
+                // in the sequence's last block (once it has landed)
+                for (int b = 0; b < kTcBlocks; ++b) {
+                    if ((loaded >> b) & 1u) continue;
+                    for (int i = lane; i < kBlockSize * 16; i += 32) {
+                        const int r = b * kBlockSize + (i >> 4), c = i & 15;
+                        const uint32_t a = vdst + (c >> 3) * kTcKVChunk + r * 128 + ((c & 7) << 4);
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0) : "memory");
+                    }
+                }
+                const int jt = (ctx % kBlockSize) ? nblk_seq - 1 : -1;
+                const int bt = jt - j * kTcBlocks;
+                if (bt >= 0 && bt < kTcBlocks && ((loaded >> bt) & 1u)) {
+                    bool landed = true;
+                    if (lane == 0) landed = mbar_wait_bounded(kv_full + 8 * st, round & 1);
+                    if (!__shfl_sync(0xffffffffu, landed, 0)) {
+                        if (lane == 0) {
+                            count_error(p.err);
+                            atomicExch(&abort_sh, 1);
+                        }
+                        break;
+                    }
+                    const int r0 = ctx % kBlockSize;
+                    for (int i = lane; i < (kBlockSize - r0) * 16; i += 32) {
+                        const int r = bt * kBlockSize + r0 + (i >> 4), c = i & 15;
+                        const uint32_t a = vdst + (c >> 3) * kTcKVChunk + r * 128 + ((c & 7) << 4);
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0) : "memory");
+                    }
+                }
+                fence_proxy_async_smem();  // these generic stores are read by the tensor core
+                __syncwarp();
+                if (lane == 0) mbar_arrive(v_ready + 8 * st);
+            }
+        }
+    } else if (FP8 && warp >= kConv0) {
+        // ================= FP8 converters: warp kConv0 + b owns block b of each tile =================
+        // The E4M3 codes of the block's 16 K and V rows become f16 in the swizzled
+        // operand layout.  Lane order: item i = (row pair i >> 4, half (i >> 3) & 1,
+        // 16-code chunk i & 7); a pair's rows split their chunks 0-3 / 4-7 between the
+        // halves, so that each 8-lane quarter of a 16-byte access reads and writes 8
+        // distinct bank groups.
+        const int b = warp - kConv0;
+        bool ok = true;
+        for (int j = 0; j < ntiles && !*abort_flag; ++j) {
+            const int st = j % kTcStages, round = j / kTcStages;
+            const int jb = j * kTcBlocks + b;
+            int id = -1;
+            if (jb < nblk_seq) id = __ldg(tab + jb);
+            const bool blk = jb < nblk_seq && id >= 0 && id < p.num_blocks;  // warp-uniform
+            bool go = true;
+            if (lane == 0) {
+                if (round > 0) go = mbar_wait_bounded(kv_empty + 8 * st, (round - 1) & 1);
+                if (go) go = mbar_wait_bounded(stg_full + 8 * (j & 1), (j >> 1) & 1);
+            }
+            if (!(ok = __shfl_sync(0xffffffffu, go, 0))) break;
+            const uint32_t kst = base + kTcStg + (j & 1) * 2 * kTcStgBytes, vst = kst + kTcStgBytes;
+            const uint32_t kdst = base + kTcKV + st * 2 * kTcKVBytes, vdst = kdst + kTcKVBytes;
+            const int tail_from = ctx - j * kTcKeys;  // V rows from here on hold no token
+            uint32_t src[4], dlo[4], dhi[4];
+            int row[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = u * 32 + lane, c = i & 7;
+                const int r = b * kBlockSize + 2 * (i >> 4) + ((c >> 2) ^ ((i >> 3) & 1));
+                row[u] = r;
+                src[u] = (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
+                // f16 pieces 2c and 2c+1 of the row: column chunk c >> 2, slots swizzled by the row
+                dlo[u] = (uint32_t)((c >> 2) * kTcKVChunk + r * 128 + ((((2 * c) & 7) ^ (r & 7)) << 4));
+                dhi[u] = (uint32_t)((c >> 2) * kTcKVChunk + r * 128 + ((((2 * c + 1) & 7) ^ (r & 7)) << 4));
+            }
+            if (blk) {
+                uint4 kc[4], vc[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(kc[u].x), "=r"(kc[u].y), "=r"(kc[u].z), "=r"(kc[u].w)
+                                 : "r"(kst + src[u]));
+                    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(vc[u].x), "=r"(vc[u].y), "=r"(vc[u].z), "=r"(vc[u].w)
+                                 : "r"(vst + src[u]));
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    uint4 lo, hi;
+                    e4m3x16_to_f16(kc[u], lo, hi);
+                    st_shared_v4(kdst + dlo[u], lo);
+                    st_shared_v4(kdst + dhi[u], hi);
+                    if (row[u] < tail_from) {
+                        e4m3x16_to_f16(vc[u], lo, hi);
+                    } else {  // a slot past the context: no token, V stays zero
+                        lo = make_uint4(0u, 0u, 0u, 0u);
+                        hi = lo;
+                    }
+                    st_shared_v4(vdst + dlo[u], lo);
+                    st_shared_v4(vdst + dhi[u], hi);
+                }
+            } else {
+                // a block not loaded: its K stays as it was (its scores are masked), V is zero
+                const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    st_shared_v4(vdst + dlo[u], z);
+                    st_shared_v4(vdst + dhi[u], z);
                 }
             }
-            fence_proxy_async_smem();  // these generic stores are read by the tensor core
+            fence_proxy_async_smem();  // generic stores read by the tensor core; staging reads before TMA reuse
             __syncwarp();
-            if (lane == 0) mbar_arrive(v_ready + 8 * st);
+            if (lane == 0) {
+                mbar_arrive(stg_empty + 8 * (j & 1));
+                mbar_arrive(kv_full + 8 * st);
+                mbar_arrive(v_ready + 8 * st);
+            }
+        }
+        if (!ok && lane == 0) {
+            count_error(p.err);
+            atomicExch(&abort_sh, 1);
         }
     } else if (warp == kMma) {
         // ================= MMA issuer =================
         // order per KV tile j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1): each Q tile's softmax
         // overlaps the other tile's products
-        const uint32_t idesc_s = instr_desc_bf16(kTcRows, kTcKeys, false);
-        const uint32_t idesc_o = instr_desc_bf16(kTcRows, kTcD, true);
+        const uint32_t idesc_s = instr_desc_16(kTcRows, kTcKeys, false, FP8);
+        const uint32_t idesc_o = instr_desc_16(kTcRows, kTcD, true, FP8);
         bool alive = true;
         // descriptors of an operand's first k-step; a k-step adds its byte offset >> 4 to
         // the start-address field (all of shared memory is below 2^18 bytes: no carry)
@@ -327,7 +489,7 @@ __global__ void __launch_bounds__(320, 1)
             return true;
         };
         if (lane == 0) {
-            alive = mbar_wait_bounded(q_full, 0) && kv_landed(0);
+            alive = mbar_wait_bounded(FP8 ? q_ready : q_full, 0) && kv_landed(0);
             if (alive)
                 for (int t = 0; t < kTcQT; ++t)
                     if (ntq[t] > 0) issue_s(t, 0);
@@ -361,6 +523,30 @@ __global__ void __launch_bounds__(320, 1)
         float m_ref = -INFINITY, l = 0.f;
         bool alive = true;
         const int nt = ntq[t];
+        if constexpr (FP8) {
+            // the products run in f16 (an E4M3 code is exact there): this warpgroup turns
+            // its Q tile from bf16 into f16 in place
+            const bool landed = mbar_wait_bounded(q_full, 0);
+            if (__all_sync(0xffffffffu, landed)) {
+                const uint32_t qt = base + kTcQ + t * kTcQBytes;
+                for (int w = r; w < kTcQBytes / 16; w += kTcRows) {
+                    uint4 v;
+                    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                                 : "r"(qt + 16 * w));
+                    v.x = bf16x2_to_f16x2(v.x);
+                    v.y = bf16x2_to_f16x2(v.y);
+                    v.z = bf16x2_to_f16x2(v.z);
+                    v.w = bf16x2_to_f16x2(v.w);
+                    st_shared_v4(qt + 16 * w, v);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(q_ready);
+            } else {
+                alive = false;
+            }
+        }
         // validity of the blocks this CTA reads, once, into shared memory (both
         // warpgroups together; the named barrier counts their 256 threads only)
         const int nblk_cta = min(nblk_seq, (last_pos / kBlockSize) + 1);
@@ -374,7 +560,7 @@ __global__ void __launch_bounds__(320, 1)
             }
             asm volatile("bar.sync 1, 256;" ::: "memory");
         }
-        for (int j = 0; j < nt; ++j) {
+        for (int j = 0; j < nt && alive; ++j) {
             if (*abort_flag) {
                 alive = false;
                 break;
@@ -438,7 +624,7 @@ __global__ void __launch_bounds__(320, 1)
             for (int e = 0; e < kTcKeys / 2; ++e) {
                 const float p0 = fast_exp2(x[2 * e] - mu), p1 = fast_exp2(x[2 * e + 1] - mu);
                 sum8[e & 7] += p0 + p1;
-                pw[e] = pack_bf16x2(p0, p1);
+                pw[e] = FP8 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
             }
             const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
             // PV_{j-1} must be done before P is overwritten and before O is read
@@ -484,7 +670,7 @@ __global__ void __launch_bounds__(320, 1)
             const bool w3 = mbar_wait_bounded(pv_done + 8 * t, (nt - 1) & 1);
             if (__all_sync(0xffffffffu, w3)) {
                 tc_fence_after();
-                const float inv = l > 0.f ? 1.f / l : 0.f;
+                const float inv = l > 0.f ? p.out_scale / l : 0.f;
                 const bool store = qrow < nq;
                 __nv_bfloat16* out = p.out + ((size_t)(qs0 + (store ? qrow : 0)) * p.num_heads + h) * kTcD;
 #pragma unroll 1
@@ -521,12 +707,13 @@ __global__ void __launch_bounds__(320, 1)
 }
 
 cudaError_t launch_prefill_tc(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                              const PrefillParams& p, int max_query_len, cudaStream_t stream) {
-    const int smem = kTcSmem + 1024;
-    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+                              const PrefillParams& p, bool fp8, int max_query_len, cudaStream_t stream) {
+    const int smem = (fp8 ? kTcSmemFp8 : kTcSmem) + 1024;
+    auto kernel = fp8 ? prefill_tc_kernel<true> : prefill_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const int tiles = (max_query_len + kTcQT * kTcRows - 1) / (kTcQT * kTcRows);
-    return launch_pdl(prefill_tc_kernel, dim3(tiles, p.num_seqs, p.num_heads), dim3(320), smem, stream, tmQ, tmK,
+    return launch_pdl(kernel, dim3(tiles, p.num_seqs, p.num_heads), dim3(fp8 ? 448 : 320), smem, stream, tmQ, tmK,
                       tmV, p);
 }
 

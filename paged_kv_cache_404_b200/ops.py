@@ -126,9 +126,10 @@ def paged_attention_decode_shared(out, q, k_pool, v_pool, block_tables, context_
 
 
 def paged_attention_prefill(out, q, k_pool, v_pool, block_tables, context_lens, query_start, scale, max_query_len,
-                            err_count=None, stream=None):
+                            err_count=None, stream=None, k_scale=1.0, v_scale=1.0):
     """Causal attention of each sequence's new tokens (the last nq of its context)
-    over its whole context; q/out [total_q, Hq, D], query_start int32 [S + 1]."""
+    over its whole context; q/out [total_q, Hq, D], query_start int32 [S + 1].
+    k_scale / v_scale dequantise an FP8 E4M3 cache (ignored for bf16)."""
     T, Hq, D = q.shape
     NB, bs, Hkv, D2 = k_pool.shape
     S = int(context_lens.numel())
@@ -142,7 +143,7 @@ def paged_attention_prefill(out, q, k_pool, v_pool, block_tables, context_lens, 
     st = L.lib().pkv_paged_attention_prefill(
         _ptr(out), _ptr(q), _dtype_code(q), _ptr(k_pool), _ptr(v_pool), _dtype_code(k_pool), _ptr(block_tables),
         int(block_tables.shape[1]), _ptr(context_lens), _ptr(query_start), S, T, int(max_query_len), NB, bs, Hq,
-        Hkv, D, float(scale), _ptr(err_count), _stream(stream))
+        Hkv, D, float(scale), float(k_scale), float(v_scale), _ptr(err_count), _stream(stream))
     L.check("pkv_paged_attention_prefill", st)
     return out
 

@@ -3,8 +3,8 @@ block tables) against the oracle.
 
 Prompts are allocated through the block manager (allocate first, then fill the
 last block), their K/V written with paged_kv_write at the prompt's slots, into
-pools whose every other byte is NaN, so a read of a slot past a context or of a
-wrong block shows.  Small cases are compared on every element, the full-size
+pools whose every other byte is NaN (bf16 NaN, or the E4M3 NaN code for an FP8
+cache), so a read of a slot past a context or of a wrong block shows.  Small cases are compared on every element, the full-size
 workload on sampled rows, in the launch configuration the benchmark uses.
 """
 import numpy as np
@@ -28,9 +28,10 @@ def _built():
 class PrefillCase:
     """Sequences with context lengths `ctx` whose last `nq` tokens are queries."""
 
-    def __init__(self, Hq, Hkv, ctx, nq, seed, nan_pool=True):
+    def __init__(self, Hq, Hkv, ctx, nq, seed, nan_pool=True, cache="bf16"):
         import paged_kv_cache_404_b200 as pkv
-        self.w = W.Workload("pf", Hq, Hkv, 128, "bf16", "bf16", len(ctx), "uniform", 1, 1, seed=seed)
+        self.w = W.Workload("pf", Hq, Hkv, 128, cache, "bf16", len(ctx), "uniform", 1, 1, seed=seed)
+        self.cache = cache
         self.ctx = np.asarray(ctx, np.int32)
         self.nq = np.asarray(nq, np.int32)
         need = int(sum(-(-int(c) // 16) for c in ctx))
@@ -41,16 +42,23 @@ class PrefillCase:
         self.maxb = max(1, max(-(-int(c) // 16) for c in ctx))
         self.tables, _ = self.bm.tables(self.ids, self.maxb, pad=-1)
         shape = (self.NB, 16, Hkv, 128)
-        if nan_pool:
+        if nan_pool and cache == "fp8":
+            self.kp = torch.full(shape, 0x7F, dtype=torch.uint8, device="cuda")
+            self.vp = torch.full(shape, 0xFF, dtype=torch.uint8, device="cuda")
+        elif nan_pool:
             self.kp = torch.full(shape, float("nan"), dtype=torch.bfloat16, device="cuda")
             self.vp = torch.full(shape, float("nan"), dtype=torch.bfloat16, device="cuda")
         else:
             self.kp, self.vp, _, _ = W.random_pools(self.w, self.NB, "cuda")
         total = int(self.ctx.sum())
         k, v = W.logical_kv(self.w, total, "cuda", stream=80)
+        # per-tensor FP8 scales amax / 448 of the written tokens (1 for bf16)
+        self.k_scale = float(k.abs().max().float().item()) / 448.0 if cache == "fp8" and total else 1.0
+        self.v_scale = float(v.abs().max().float().item()) / 448.0 if cache == "fp8" and total else 1.0
         slots = np.concatenate([self.bm.slots(s, 0, int(c)) for s, c in zip(self.ids, ctx)]) if total else []
         if total:
-            pkv.paged_kv_write(k, v, torch.from_numpy(np.asarray(slots, np.int64)).cuda(), self.kp, self.vp)
+            pkv.paged_kv_write(k, v, torch.from_numpy(np.asarray(slots, np.int64)).cuda(), self.kp, self.vp,
+                               self.k_scale, self.v_scale)
         self.qs = np.concatenate([[0], np.cumsum(self.nq)]).astype(np.int32)
         self.q = W.queries(W.scaled(self.w, num_seqs=int(self.qs[-1])), int(self.qs[-1]), "cuda")
 
@@ -62,15 +70,17 @@ class PrefillCase:
         mq = int(self.nq.max()) if max_query_len is None else max_query_len
         pkv.paged_attention_prefill(self.out, self.q, self.kp, self.vp, torch.from_numpy(tabs).cuda(),
                                     torch.from_numpy(self.ctx).cuda(), torch.from_numpy(self.qs).cuda(),
-                                    self.w.scale, mq, err_count=self.err)
+                                    self.w.scale, mq, err_count=self.err, k_scale=self.k_scale,
+                                    v_scale=self.v_scale)
         torch.cuda.synchronize()
         return self.out
 
     def oracle(self, rows=None, tables=None):
         tabs = self.tables if tables is None else tables
+        cdt = oracle.FP8_E4M3 if self.cache == "fp8" else oracle.BF16
         return oracle.paged_attention_prefill(to_np_bits(self.q), oracle.BF16, to_np_bits(self.kp),
-                                              to_np_bits(self.vp), oracle.BF16, tabs, self.ctx, self.qs,
-                                              self.w.scale, rows=rows)
+                                              to_np_bits(self.vp), cdt, tabs, self.ctx, self.qs,
+                                              self.w.scale, self.k_scale, self.v_scale, rows=rows)
 
 
 RAGGED = ([1, 15, 16, 17, 64, 65, 200, 300, 100, 129, 33],
@@ -86,6 +96,42 @@ def test_ragged_prompts_every_element(Hq, Hkv):
     ref, bad = c.oracle()
     assert bad == 0 and int(c.err.item()) == 0
     assert_close(got, ref, "bf16", "prefill G=%d" % (Hq // Hkv))
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (64, 8)])
+def test_fp8_cache_ragged_prompts_every_element(Hq, Hkv):
+    """The same ragged prompts over an FP8 E4M3 cache (codes turned into f16 in
+    shared memory, per-tensor scales); unowned bytes hold the E4M3 NaN code."""
+    c = PrefillCase(Hq, Hkv, *RAGGED, seed=50 + Hq, cache="fp8")
+    got = out_to_f64(c.run())
+    ref, bad = c.oracle()
+    assert bad == 0 and int(c.err.item()) == 0
+    assert_close(got, ref, "fp8", "fp8 prefill G=%d" % (Hq // Hkv))
+
+
+def test_fp8_cache_long_prompts_sampled_rows():
+    """FP8 cache, prompts of 1,000..3,000 tokens (many KV tiles, both staging
+    slots reused), 32/8 heads; rows sampled, first and last of every prompt."""
+    lens = [3000, 1000, 2047, 1537]
+    c = PrefillCase(32, 8, lens, lens, seed=51, nan_pool=False, cache="fp8")
+    got = out_to_f64(c.run())
+    assert int(c.err.item()) == 0
+    rng = np.random.default_rng(52)
+    rows = np.sort(rng.choice(int(c.qs[-1]), 40, replace=False))
+    rows = np.unique(np.concatenate([rows, c.qs[1:] - 1, c.qs[:-1]]))
+    ref, _ = c.oracle(rows=rows)
+    assert_close(got[rows], ref[rows], "fp8", "fp8 long prompts")
+
+
+def test_fp8_cache_bad_ids_are_counted():
+    c = PrefillCase(16, 4, [90, 40], [90, 10], seed=53, nan_pool=False, cache="fp8")
+    tabs = c.tables.copy()
+    tabs[0, 2] = c.NB + 5
+    tabs[1, 0] = -3
+    got = out_to_f64(c.run(tables=tabs))
+    ref, bad = c.oracle(tables=tabs)
+    assert bad == 2 and int(c.err.item()) == bad
+    assert_close(got, ref, "fp8", "fp8 bad ids")
 
 
 def test_one_token_rows_equal_decode():
@@ -147,6 +193,9 @@ def test_warp_mma_kernel_agrees(tmp_path):
         "got = out_to_f64(c.run()); ref, bad = c.oracle()\n"
         "assert bad == 0 and int(c.err.item()) == 0\n"
         "assert_close(got, ref, 'bf16', 'mma.sync prefill')\n"
+        "import pytest, paged_kv_cache_404_b200 as pkv\n"
+        "f = PrefillCase(8, 8, [40], [40], seed=46, cache='fp8')\n"
+        "with pytest.raises(pkv.PagedKVError): f.run()\n"
         "print('ok')\n" % os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
     env = dict(os.environ, PKV_PREFILL_KERNEL="mma")
     r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=600)

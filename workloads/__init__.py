@@ -17,6 +17,8 @@ Workloads are shaped like the PagedAttention pages' examples:
 - "fp8_long": FP8 E4M3 cache, log-uniform context lengths 256..32,768.
 - "prefill70b": the prompt pass of the Llama-3.1-70B shape: 16 prompts of
   512..4,096 tokens written into blocks and attended causally.
+- "prefill70b_fp8": the same prompt pass over an FP8 E4M3 cache (per-tensor
+  scales amax/448 of the prompt's K and V).
 - "beam": beam search, 16 requests x 4 beams over a 1,000-token prompt; at
   every step each request keeps 4 beams drawn (seeded) from its current ones:
   forks, frees and copy-on-write at every step.
@@ -67,6 +69,7 @@ WORKLOADS = {
                               num_prompts=64, samples=3, prefix_len=1000),
     "fp8_long": Workload("fp8_long", 32, 8, 128, "fp8", "bf16", 128, "loguniform", 256, 32768, seed=5),
     "prefill70b": Workload("prefill70b", 64, 8, 128, "bf16", "bf16", 16, "uniform", 512, 4096, seed=6),
+    "prefill70b_fp8": Workload("prefill70b_fp8", 64, 8, 128, "fp8", "bf16", 16, "uniform", 512, 4096, seed=6),
     "beam": Workload("beam", 32, 8, 128, "bf16", "bf16", 64, "beam", 0, 48, seed=7,
                      num_prompts=16, samples=4, prefix_len=1000),
 }
