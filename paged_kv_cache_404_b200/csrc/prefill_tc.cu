@@ -11,30 +11,33 @@
 // warps for a bf16 cache:
 //  - warp 8 (producer): TMA-loads the two Q tiles once and, per 64-key tile, the
 //    K and V of 4 blocks of the table (16-slot x 1-head x 128-byte boxes,
-//    128-byte swizzle) into a 3-stage ring; V rows that hold no token of the context
+//    128-byte swizzle) into a 4-stage ring; V rows that hold no token of the context
 //    (past its end, or a block past the table or with a bad id) are zeroed in
 //    shared memory, so that a zero probability never meets a NaN there;
 //  - warp 9 (MMA): one thread issues tcgen05.mma: per Q tile t, S_t = Q_t K^T
-//    (M=128, N=64, K=128, bf16 -> fp32) into TMEM, then O_t += P_t V (P from
-//    shared memory, V MN-major) into a TMEM accumulator; tcgen05.commit signals
-//    mbarriers; the warp allocates and frees the 512 TMEM columns;
+//    (M=128, N=64, K=128, bf16 -> fp32; Q_t from TMEM, K from shared memory) into
+//    TMEM, then O_t += P_t V (P_t from TMEM, V MN-major from shared memory) into a
+//    TMEM accumulator; tcgen05.commit signals mbarriers; the warp allocates and
+//    frees the 512 TMEM columns;
 //  - warps 0-3 and 4-7 (softmax, one warpgroup per Q tile): thread r owns
-//    query row r of its tile (TMEM lane r): loads its 64 scores with
-//    tcgen05.ld, applies the causal mask, runs the online
-//    softmax in base 2 (the reference max moves only when a score exceeds it by
-//    more than 2^8, then O is rescaled in TMEM), writes P as bf16 into the
-//    swizzled K-major layout the PV MMA reads, and finally normalises O and
-//    stores the rows.
+//    query row r of its tile (TMEM lane r): first moves its row of Q from the
+//    TMA-landed tile into TMEM; then per KV tile loads its 64 scores with
+//    tcgen05.ld, applies the causal mask, runs the online softmax in base 2 (the
+//    reference max moves only when a score exceeds it by more than 2^8, then O is
+//    rescaled in TMEM), writes P as 16-bit pairs into TMEM over the scores it
+//    has read, and finally normalises O and stores the row.
 // The products are issued PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), ..., so that
 // each warpgroup's softmax runs while the tensor core works for the other.
+// Keeping Q and P in TMEM leaves shared memory only the K and V reads of the
+// products.
 //
 // FP8 E4M3 cache (14 warps): the products run in f16, which holds every E4M3
 // value exactly.  Warp 8 TMA-loads the codes (128-byte rows) into a 2-deep
 // staging ring; warps 10-13 each turn one 16-slot block of a tile into f16 in the
 // ring the tensor core reads (and zero V where no token is), then arrive on the
-// stage's barriers; the softmax warps first take their Q tile from bf16 into f16
-// in place and write P as f16.  k_scale folds into the score scale and v_scale
-// into the final normalisation.
+// stage's barriers; the softmax warps take Q into f16 on its way to TMEM and
+// write P as f16.  k_scale folds into the score scale and v_scale into the final
+// normalisation.
 #include "pkv_common.cuh"
 
 namespace pkv {
@@ -47,23 +50,22 @@ constexpr int kTcKeys = 64;                    // keys per KV tile (MMA N of S, 
 constexpr int kTcD = 128;                      // head_dim
 constexpr int kTcQChunk = kTcRows * 128;       // one 64-element column chunk of a 128-row operand: 16 KB
 constexpr int kTcQBytes = 2 * kTcQChunk;       // Q tile: 128 rows x 128 bf16
-constexpr int kTcPBytes = kTcRows * 128;       // P tile: 128 rows x 64 keys (one chunk)
 constexpr int kTcKVChunk = kTcKeys * 128;      // one 64-element column chunk of a 64-row operand: 8 KB
 constexpr int kTcKVBytes = 2 * kTcKVChunk;     // K (or V) tile: 64 keys x 128 bf16
-constexpr int kTcStages = 3;
+constexpr int kTcStages = 4;
 constexpr int kTcBlocks = kTcKeys / kBlockSize;  // table blocks per KV tile
 // shared memory layout (offsets from a 1024-aligned base)
-constexpr int kTcQ = 0;                                    // Q tile t at kTcQ + t * kTcQBytes
-constexpr int kTcP = kTcQ + kTcQT * kTcQBytes;             // P tile t at kTcP + t * kTcPBytes
-constexpr int kTcKV = kTcP + kTcQT * kTcPBytes;            // stage st: K, then V
+constexpr int kTcQ = 0;                                    // Q tile t at kTcQ + t * kTcQBytes (TMA landing)
+constexpr int kTcKV = kTcQ + kTcQT * kTcQBytes;            // stage st: K, then V
 constexpr int kTcSmem = kTcKV + kTcStages * 2 * kTcKVBytes;  // 192 KB
 // FP8 cache: E4M3 K and V tiles land in a 2-deep staging ring (64 rows x 128 bytes
 // each), then become f16 in the ring above
 constexpr int kTcStgBytes = kTcKeys * 128;
 constexpr int kTcStg = kTcSmem;
 constexpr int kTcSmemFp8 = kTcStg + 2 * 2 * kTcStgBytes;  // 224 KB
-// TMEM columns: S of Q tile t at t*64, O of Q tile t at 128 + t*128
-constexpr int kTcSCol = 0, kTcOCol = 128;
+// TMEM columns (512): S of Q tile t at t*64 (fp32; P as 16-bit pairs over its first
+// 32), O of Q tile t at 128 + t*128 (fp32), Q tile t at 384 + t*64 (16-bit pairs)
+constexpr int kTcSCol = 0, kTcOCol = 128, kTcQCol = 384;
 constexpr float kRescaleThreshold = 8.f;       // log2 of the largest factor p may exceed 1 by
 constexpr int kTcOkWords = 64;                 // validity bits kept in shared memory for 2048 blocks
 
@@ -111,12 +113,13 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
     return r;
 }
 
-__device__ __forceinline__ void umma_ss(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, bool accumulate) {
+// A from TMEM (lane = row, 16-bit pairs along K), B from shared memory.
+__device__ __forceinline__ void umma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t idesc, bool accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "l"(a), "l"(b), "r"(idesc), "r"((uint32_t)accumulate)
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(b), "r"(idesc), "r"((uint32_t)accumulate)
         : "memory");
 }
 
@@ -173,17 +176,18 @@ __global__ void __launch_bounds__(FP8 ? 448 : 320, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
-    // kv_full[3], kv_empty[3], v_ready[3], q_full, s_full[2], p_full[2], pv_done[2],
-    // FP8: stg_full[2], stg_empty[2], q_ready
-    __shared__ __align__(8) uint64_t bars[21];
+    // kv_full[S], kv_empty[S], v_ready[S] (S = kTcStages), q_full, s_full[2], p_full[2],
+    // pv_done[2], FP8: stg_full[2], stg_empty[2]; q_ready
+    __shared__ __align__(8) uint64_t bars[3 * kTcStages + 12];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
     __shared__ uint32_t ok_bits[kTcOkWords];  // block b of the sequence holds tokens (table, id in range)
     volatile int* abort_flag = &abort_sh;
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
     const uint32_t b0 = smem_u32(&bars[0]);
-    const uint32_t kv_full = b0, kv_empty = b0 + 24, v_ready = b0 + 48, q_full = b0 + 72, s_full = b0 + 80,
-                   p_full = b0 + 96, pv_done = b0 + 112, stg_full = b0 + 128, stg_empty = b0 + 144, q_ready = b0 + 160;
+    const uint32_t kv_full = b0, kv_empty = kv_full + 8 * kTcStages, v_ready = kv_empty + 8 * kTcStages,
+                   q_full = v_ready + 8 * kTcStages, s_full = q_full + 8, p_full = s_full + 16, pv_done = p_full + 16,
+                   stg_full = pv_done + 16, stg_empty = stg_full + 16, q_ready = stg_empty + 16;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int kProducer = 8, kMma = 9, kConv0 = 10;  // FP8: warps 10-13 convert
     constexpr int kConvWarps = kTcBlocks;
@@ -206,7 +210,7 @@ __global__ void __launch_bounds__(FP8 ? 448 : 320, 1)
             mbar_init(stg_full + 8 * i, 1);
             mbar_init(stg_empty + 8 * i, kConvWarps);
         }
-        mbar_init(q_ready, 8);  // FP8: each softmax warp has turned its rows of Q into f16
+        mbar_init(q_ready, 8);  // each softmax warp has put its 32 rows of Q into TMEM
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -459,17 +463,16 @@ __global__ void __launch_bounds__(FP8 ? 448 : 320, 1)
         bool alive = true;
         // descriptors of an operand's first k-step; a k-step adds its byte offset >> 4 to
         // the start-address field (all of shared memory is below 2^18 bytes: no carry)
-        const uint64_t dq0 = smem_desc(base + kTcQ, 16, 1024), dp0 = smem_desc(base + kTcP, 16, 1024);
         const uint64_t dkv0 = smem_desc(base + kTcKV, 16, 1024);
         const uint64_t dvv0 = smem_desc(base + kTcKV + kTcKVBytes, kTcKVChunk, 1024);
         auto kv_landed = [&](int j) { return mbar_wait_bounded(kv_full + 8 * (j % kTcStages), (j / kTcStages) & 1); };
         auto issue_s = [&](int t, int j) {
             tc_fence_after();
             const uint64_t dk = dkv0 + (uint64_t)(((j % kTcStages) * 2 * kTcKVBytes) >> 4);
-            const uint64_t dq = dq0 + (uint64_t)((t * kTcQBytes) >> 4);
+            // Q_t from TMEM: 16 head dims = 8 columns per k-step
 #pragma unroll
             for (int ks = 0; ks < kTcD / 16; ++ks) {
-                umma_ss(tmem + kTcSCol + t * kTcKeys, dq + (uint64_t)((((ks >> 2) * kTcQChunk) + (ks & 3) * 32) >> 4),
+                umma_ts(tmem + kTcSCol + t * kTcKeys, tmem + kTcQCol + t * (kTcD / 2) + ks * 8,
                         dk + (uint64_t)((((ks >> 2) * kTcKVChunk) + (ks & 3) * 32) >> 4), idesc_s, ks > 0);
             }
             umma_commit(s_full + 8 * t);
@@ -479,17 +482,19 @@ __global__ void __launch_bounds__(FP8 ? 448 : 320, 1)
             if (!mbar_wait_bounded(v_ready + 8 * (j % kTcStages), (j / kTcStages) & 1)) return false;
             tc_fence_after();
             const uint64_t dv = dvv0 + (uint64_t)(((j % kTcStages) * 2 * kTcKVBytes) >> 4);
-            const uint64_t dp = dp0 + (uint64_t)((t * kTcPBytes) >> 4);
+            // P_t from TMEM over S_t's columns: 16 keys = 8 columns per k-step.  The next
+            // S_t product, issued after this one, overwrites them: the tensor core runs
+            // one thread's products in issue order.
 #pragma unroll
             for (int ks = 0; ks < kTcKeys / 16; ++ks) {
-                umma_ss(tmem + kTcOCol + t * kTcD, dp + (uint64_t)((ks * 32) >> 4),
+                umma_ts(tmem + kTcOCol + t * kTcD, tmem + kTcSCol + t * kTcKeys + ks * 8,
                         dv + (uint64_t)((ks * 16 * 128) >> 4), idesc_o, j > 0 || ks > 0);
             }
             umma_commit(pv_done + 8 * t);
             return true;
         };
         if (lane == 0) {
-            alive = mbar_wait_bounded(FP8 ? q_ready : q_full, 0) && kv_landed(0);
+            alive = mbar_wait_bounded(q_ready, 0) && kv_landed(0);
             if (alive)
                 for (int t = 0; t < kTcQT; ++t)
                     if (ntq[t] > 0) issue_s(t, 0);
@@ -519,28 +524,39 @@ __global__ void __launch_bounds__(FP8 ? 448 : 320, 1)
         const int qpos = pos0 + qrow;
         const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const uint32_t s_addr = lane_addr + kTcSCol + t * kTcKeys, o_addr = lane_addr + kTcOCol + t * kTcD;
-        const uint32_t p_row = base + kTcP + t * kTcPBytes + r * 128;
         float m_ref = -INFINITY, l = 0.f;
         bool alive = true;
         const int nt = ntq[t];
-        if constexpr (FP8) {
-            // the products run in f16 (an E4M3 code is exact there): this warpgroup turns
-            // its Q tile from bf16 into f16 in place
+        {
+            // this thread's query row from the TMA-landed tile into TMEM lane r (head dims
+            // 2c, 2c+1 in column c), as f16 for an FP8 cache (whose codes are exact in f16)
             const bool landed = mbar_wait_bounded(q_full, 0);
             if (__all_sync(0xffffffffu, landed)) {
-                const uint32_t qt = base + kTcQ + t * kTcQBytes;
-                for (int w = r; w < kTcQBytes / 16; w += kTcRows) {
-                    uint4 v;
-                    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                                 : "r"(qt + 16 * w));
-                    v.x = bf16x2_to_f16x2(v.x);
-                    v.y = bf16x2_to_f16x2(v.y);
-                    v.z = bf16x2_to_f16x2(v.z);
-                    v.w = bf16x2_to_f16x2(v.w);
-                    st_shared_v4(qt + 16 * w, v);
+                const uint32_t q_row = base + kTcQ + t * kTcQBytes + r * 128;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    float qv[32];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        uint4 v;
+                        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                                     : "r"(q_row + hf * kTcQChunk + ((q ^ (r & 7)) << 4)));
+                        if constexpr (FP8) {
+                            v.x = bf16x2_to_f16x2(v.x);
+                            v.y = bf16x2_to_f16x2(v.y);
+                            v.z = bf16x2_to_f16x2(v.z);
+                            v.w = bf16x2_to_f16x2(v.w);
+                        }
+                        qv[4 * q] = __uint_as_float(v.x);
+                        qv[4 * q + 1] = __uint_as_float(v.y);
+                        qv[4 * q + 2] = __uint_as_float(v.z);
+                        qv[4 * q + 3] = __uint_as_float(v.w);
+                    }
+                    tmem_st32(lane_addr + kTcQCol + t * (kTcD / 2) + 32 * hf, qv);
                 }
-                fence_proxy_async_smem();
+                tmem_wait_st();
+                tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(q_ready);
             } else {
@@ -650,13 +666,14 @@ __global__ void __launch_bounds__(FP8 ? 448 : 320, 1)
             }
             l = l * alpha + sum;
             m_ref = m_new;
-            // P row into the K-major 128-byte-swizzled operand: 16-byte piece q at ((q ^ (r & 7)) << 4)
+            // P row into TMEM over the first 32 columns of the scores just read
+            {
+                float pf[kTcKeys / 2];
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(p_row + ((q ^ (r & 7)) << 4)),
-                             "r"(pw[4 * q]), "r"(pw[4 * q + 1]), "r"(pw[4 * q + 2]), "r"(pw[4 * q + 3])
-                             : "memory");
-            fence_proxy_async_smem();  // generic-proxy P stores -> read by the tensor core
+                for (int e = 0; e < kTcKeys / 2; ++e) pf[e] = __uint_as_float(pw[e]);
+                tmem_st32(s_addr, pf);
+                tmem_wait_st();
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(p_full + 8 * t);
