@@ -63,9 +63,9 @@ constexpr int kTcSmem = kTcKV + kTcStages * 2 * kTcKVBytes;  // 192 KB
 constexpr int kTcStgBytes = kTcKeys * 128;
 constexpr int kTcStg = kTcSmem;
 constexpr int kTcSmemFp8 = kTcStg + 2 * 2 * kTcStgBytes;  // 224 KB
-// TMEM columns (512): S of Q tile t at t*64 (fp32; P as 16-bit pairs over its first
-// 32), O of Q tile t at 128 + t*128 (fp32), Q tile t at 384 + t*64 (16-bit pairs)
-constexpr int kTcSCol = 0, kTcOCol = 128, kTcQCol = 384;
+// TMEM columns (512): O of Q tile t at t*128 (fp32); scores of Q tile t, KV tile j in
+// buffer 256 + (2t + (j & 1))*64 (fp32; P as 16-bit pairs over its first 32)
+constexpr int kTcOCol = 0, kTcSCol = 256;
 constexpr float kRescaleThreshold = 8.f;       // log2 of the largest factor p may exceed 1 by
 constexpr int kTcOkWords = 64;                 // validity bits kept in shared memory for 2048 blocks
 
@@ -111,6 +111,16 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
     asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(__uint_as_float(w & 0xFFFF0000u)),
         "f"(__uint_as_float(w << 16)));
     return r;
+}
+
+// A and B from shared memory.
+__device__ __forceinline__ void umma_ss(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(a), "l"(b), "r"(idesc), "r"((uint32_t)accumulate)
+        : "memory");
 }
 
 // A from TMEM (lane = row, 16-bit pairs along K), B from shared memory.
@@ -176,9 +186,12 @@ __global__ void __launch_bounds__(FP8 ? 448 : 320, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
-    // kv_full[S], kv_empty[S], v_ready[S] (S = kTcStages), q_full, s_full[2], p_full[2],
-    // pv_done[2], FP8: stg_full[2], stg_empty[2]; q_ready
-    __shared__ __align__(8) uint64_t bars[3 * kTcStages + 12];
+    // kv_full[S], kv_empty[S], v_ready[S] (S = kTcStages), q_full, s_full[2][2], p_full[2][2],
+    // pv_done[2][2], FP8: stg_full[2], stg_empty[2], q_ready.  Scores, P and PV completion
+    // have one barrier per (Q tile, buffer j & 1), so that no barrier is ever more than
+    // one phase ahead of a waiter: the softmax may finish tile j+1 before the MMA issuer
+    // takes P(j), and may skip PV waits while the reference max stays put.
+    __shared__ __align__(8) uint64_t bars[3 * kTcStages + 18];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
     __shared__ uint32_t ok_bits[kTcOkWords];  // block b of the sequence holds tokens (table, id in range)
@@ -186,8 +199,8 @@ __global__ void __launch_bounds__(FP8 ? 448 : 320, 1)
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
     const uint32_t b0 = smem_u32(&bars[0]);
     const uint32_t kv_full = b0, kv_empty = kv_full + 8 * kTcStages, v_ready = kv_empty + 8 * kTcStages,
-                   q_full = v_ready + 8 * kTcStages, s_full = q_full + 8, p_full = s_full + 16, pv_done = p_full + 16,
-                   stg_full = pv_done + 16, stg_empty = stg_full + 16, q_ready = stg_empty + 16;
+                   q_full = v_ready + 8 * kTcStages, s_full = q_full + 8, p_full = s_full + 32, pv_done = p_full + 32,
+                   stg_full = pv_done + 32, stg_empty = stg_full + 16, q_ready = stg_empty + 16;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int kProducer = 8, kMma = 9, kConv0 = 10;  // FP8: warps 10-13 convert
     constexpr int kConvWarps = kTcBlocks;
@@ -201,16 +214,16 @@ __global__ void __launch_bounds__(FP8 ? 448 : 320, 1)
             mbar_init(v_ready + 8 * i, FP8 ? kConvWarps : 1);
         }
         mbar_init(q_full, 1);
-        for (int t = 0; t < kTcQT; ++t) {
-            mbar_init(s_full + 8 * t, 1);
-            mbar_init(p_full + 8 * t, 4);
-            mbar_init(pv_done + 8 * t, 1);
+        for (int i = 0; i < 2 * kTcQT; ++i) {
+            mbar_init(s_full + 8 * i, 1);
+            mbar_init(p_full + 8 * i, 4);
+            mbar_init(pv_done + 8 * i, 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(stg_full + 8 * i, 1);
             mbar_init(stg_empty + 8 * i, kConvWarps);
         }
-        mbar_init(q_ready, 8);  // each softmax warp has put its 32 rows of Q into TMEM
+        mbar_init(q_ready, 8);  // FP8: each softmax warp has turned its share of Q into f16
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -456,58 +469,62 @@ __global__ void __launch_bounds__(FP8 ? 448 : 320, 1)
         }
     } else if (warp == kMma) {
         // ================= MMA issuer =================
-        // order per KV tile j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1): each Q tile's softmax
-        // overlaps the other tile's products
+        // S_t(0), S_t(1) first; then per KV tile j: PV_0(j), S_0(j+2), PV_1(j), S_1(j+2).
+        // The scores are double-buffered, so a Q tile's softmax of tile j+1 runs while
+        // the tensor core does PV(j) and S(j+2)
         const uint32_t idesc_s = instr_desc_16(kTcRows, kTcKeys, false, FP8);
         const uint32_t idesc_o = instr_desc_16(kTcRows, kTcD, true, FP8);
         bool alive = true;
         // descriptors of an operand's first k-step; a k-step adds its byte offset >> 4 to
         // the start-address field (all of shared memory is below 2^18 bytes: no carry)
+        const uint64_t dq0 = smem_desc(base + kTcQ, 16, 1024);
         const uint64_t dkv0 = smem_desc(base + kTcKV, 16, 1024);
         const uint64_t dvv0 = smem_desc(base + kTcKV + kTcKVBytes, kTcKVChunk, 1024);
         auto kv_landed = [&](int j) { return mbar_wait_bounded(kv_full + 8 * (j % kTcStages), (j / kTcStages) & 1); };
         auto issue_s = [&](int t, int j) {
             tc_fence_after();
             const uint64_t dk = dkv0 + (uint64_t)(((j % kTcStages) * 2 * kTcKVBytes) >> 4);
-            // Q_t from TMEM: 16 head dims = 8 columns per k-step
+            const uint64_t dq = dq0 + (uint64_t)((t * kTcQBytes) >> 4);
+            const int sb = 2 * t + (j & 1);
 #pragma unroll
             for (int ks = 0; ks < kTcD / 16; ++ks) {
-                umma_ts(tmem + kTcSCol + t * kTcKeys, tmem + kTcQCol + t * (kTcD / 2) + ks * 8,
+                umma_ss(tmem + kTcSCol + sb * kTcKeys, dq + (uint64_t)((((ks >> 2) * kTcQChunk) + (ks & 3) * 32) >> 4),
                         dk + (uint64_t)((((ks >> 2) * kTcKVChunk) + (ks & 3) * 32) >> 4), idesc_s, ks > 0);
             }
-            umma_commit(s_full + 8 * t);
+            umma_commit(s_full + 8 * sb);
         };
         auto issue_pv = [&](int t, int j) -> bool {
-            if (!mbar_wait_bounded(p_full + 8 * t, j & 1)) return false;
+            if (!mbar_wait_bounded(p_full + 8 * (2 * t + (j & 1)), (j >> 1) & 1)) return false;
             if (!mbar_wait_bounded(v_ready + 8 * (j % kTcStages), (j / kTcStages) & 1)) return false;
             tc_fence_after();
             const uint64_t dv = dvv0 + (uint64_t)(((j % kTcStages) * 2 * kTcKVBytes) >> 4);
-            // P_t from TMEM over S_t's columns: 16 keys = 8 columns per k-step.  The next
-            // S_t product, issued after this one, overwrites them: the tensor core runs
-            // one thread's products in issue order.
+            // P_t(j) from TMEM over its score buffer: 16 keys = 8 columns per k-step.  The
+            // S_t(j+2) product, issued after this one, overwrites them: the tensor core
+            // runs one thread's products in issue order.
+            const int sb = 2 * t + (j & 1);
 #pragma unroll
             for (int ks = 0; ks < kTcKeys / 16; ++ks) {
-                umma_ts(tmem + kTcOCol + t * kTcD, tmem + kTcSCol + t * kTcKeys + ks * 8,
+                umma_ts(tmem + kTcOCol + t * kTcD, tmem + kTcSCol + sb * kTcKeys + ks * 8,
                         dv + (uint64_t)((ks * 16 * 128) >> 4), idesc_o, j > 0 || ks > 0);
             }
-            umma_commit(pv_done + 8 * t);
+            umma_commit(pv_done + 8 * sb);
             return true;
         };
         if (lane == 0) {
-            alive = mbar_wait_bounded(q_ready, 0) && kv_landed(0);
-            if (alive)
-                for (int t = 0; t < kTcQT; ++t)
-                    if (ntq[t] > 0) issue_s(t, 0);
+            alive = mbar_wait_bounded(FP8 ? q_ready : q_full, 0);
+            for (int j = 0; j < 2 && j < ntiles && alive; ++j) {
+                alive = kv_landed(j);
+                for (int t = 0; t < kTcQT && alive; ++t)
+                    if (j < ntq[t]) issue_s(t, j);
+            }
             for (int j = 0; j < ntiles && alive && !*abort_flag; ++j) {
-                const bool next = j + 1 < ntiles;
                 for (int t = 0; t < kTcQT && alive; ++t) {
                     if (j < ntq[t]) alive = issue_pv(t, j);
-                    if (alive && j + 1 < ntq[t]) {
-                        alive = kv_landed(j + 1);
-                        if (alive) issue_s(t, j + 1);
+                    if (alive && j + 2 < ntq[t]) {
+                        alive = kv_landed(j + 2);
+                        if (alive) issue_s(t, j + 2);
                     }
                 }
-                (void)next;
                 if (alive) umma_commit(kv_empty + 8 * (j % kTcStages));
             }
             if (!alive) {
@@ -523,40 +540,28 @@ __global__ void __launch_bounds__(FP8 ? 448 : 320, 1)
         const int qrow = row0 + t * kTcRows + r;     // query row in the sequence
         const int qpos = pos0 + qrow;
         const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-        const uint32_t s_addr = lane_addr + kTcSCol + t * kTcKeys, o_addr = lane_addr + kTcOCol + t * kTcD;
+        const uint32_t o_addr = lane_addr + kTcOCol + t * kTcD;
         float m_ref = -INFINITY, l = 0.f;
         bool alive = true;
         const int nt = ntq[t];
-        {
-            // this thread's query row from the TMA-landed tile into TMEM lane r (head dims
-            // 2c, 2c+1 in column c), as f16 for an FP8 cache (whose codes are exact in f16)
+        if constexpr (FP8) {
+            // the products run in f16 (an E4M3 code is exact there): this warpgroup turns
+            // its Q tile from bf16 into f16 in place
             const bool landed = mbar_wait_bounded(q_full, 0);
             if (__all_sync(0xffffffffu, landed)) {
-                const uint32_t q_row = base + kTcQ + t * kTcQBytes + r * 128;
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    float qv[32];
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        uint4 v;
-                        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                                     : "r"(q_row + hf * kTcQChunk + ((q ^ (r & 7)) << 4)));
-                        if constexpr (FP8) {
-                            v.x = bf16x2_to_f16x2(v.x);
-                            v.y = bf16x2_to_f16x2(v.y);
-                            v.z = bf16x2_to_f16x2(v.z);
-                            v.w = bf16x2_to_f16x2(v.w);
-                        }
-                        qv[4 * q] = __uint_as_float(v.x);
-                        qv[4 * q + 1] = __uint_as_float(v.y);
-                        qv[4 * q + 2] = __uint_as_float(v.z);
-                        qv[4 * q + 3] = __uint_as_float(v.w);
-                    }
-                    tmem_st32(lane_addr + kTcQCol + t * (kTcD / 2) + 32 * hf, qv);
+                const uint32_t qt = base + kTcQ + t * kTcQBytes;
+                for (int w = r; w < kTcQBytes / 16; w += kTcRows) {
+                    uint4 v;
+                    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                                 : "r"(qt + 16 * w));
+                    v.x = bf16x2_to_f16x2(v.x);
+                    v.y = bf16x2_to_f16x2(v.y);
+                    v.z = bf16x2_to_f16x2(v.z);
+                    v.w = bf16x2_to_f16x2(v.w);
+                    st_shared_v4(qt + 16 * w, v);
                 }
-                tmem_wait_st();
-                tc_fence_before();
+                fence_proxy_async_smem();  // read by the tensor core
                 __syncwarp();
                 if (lane == 0) mbar_arrive(q_ready);
             } else {
@@ -593,7 +598,9 @@ __global__ void __launch_bounds__(FP8 ? 448 : 320, 1)
                     if (id >= 0 && id < p.num_blocks) okmask |= 1u << b;
                 }
             }
-            const bool w1 = mbar_wait_bounded(s_full + 8 * t, j & 1);
+            const int sb = 2 * t + (j & 1);
+            const uint32_t s_addr = lane_addr + kTcSCol + sb * kTcKeys;
+            const bool w1 = mbar_wait_bounded(s_full + 8 * sb, (j >> 1) & 1);
             if (!__all_sync(0xffffffffu, w1)) {
                 alive = false;
                 break;
@@ -633,7 +640,7 @@ __global__ void __launch_bounds__(FP8 ? 448 : 320, 1)
             const float m_new = move ? mx : m_ref;
             if (move && m_ref != -INFINITY) alpha = fast_exp2(m_ref - m_new);
             const float mu = m_new == -INFINITY ? 0.f : m_new;
-            // P row as bf16 (computed before waiting for the previous PV)
+            // P row as 16-bit pairs
             uint32_t pw[kTcKeys / 2];
             float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -643,26 +650,25 @@ __global__ void __launch_bounds__(FP8 ? 448 : 320, 1)
                 pw[e] = FP8 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
             }
             const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
-            // PV_{j-1} must be done before P is overwritten and before O is read
-            if (j > 0) {
-                const bool w2 = mbar_wait_bounded(pv_done + 8 * t, (j - 1) & 1);
+            // a moved reference max rescales O, once PV(j-1) has landed in it (PV(j+1), the
+            // next on that barrier, waits for P(j+1): the barrier is at most one phase on)
+            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                const bool w2 = mbar_wait_bounded(pv_done + 8 * (2 * t + ((j - 1) & 1)), ((j - 1) >> 1) & 1);
                 if (!__all_sync(0xffffffffu, w2)) {
                     alive = false;
                     break;
                 }
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-                    for (int c4 = 0; c4 < kTcD / 32; ++c4) {
-                        float v[32];
-                        tmem_ld32(o_addr + 32 * c4, v);
-                        tmem_wait_ld();
+                for (int c4 = 0; c4 < kTcD / 32; ++c4) {
+                    float v[32];
+                    tmem_ld32(o_addr + 32 * c4, v);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] *= alpha;
-                        tmem_st32(o_addr + 32 * c4, v);
-                    }
-                    tmem_wait_st();
+                    for (int i = 0; i < 32; ++i) v[i] *= alpha;
+                    tmem_st32(o_addr + 32 * c4, v);
                 }
+                tmem_wait_st();
             }
             l = l * alpha + sum;
             m_ref = m_new;
@@ -676,7 +682,7 @@ __global__ void __launch_bounds__(FP8 ? 448 : 320, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full + 8 * t);
+            if (lane == 0) mbar_arrive(p_full + 8 * sb);
         }
         if (!alive && lane == 0) {
             count_error(p.err);
@@ -684,7 +690,8 @@ __global__ void __launch_bounds__(FP8 ? 448 : 320, 1)
         }
         // epilogue: wait for the last PV, normalise and store the row
         if (alive && nt > 0 && !*abort_flag) {
-            const bool w3 = mbar_wait_bounded(pv_done + 8 * t, (nt - 1) & 1);
+            // PV(nt-1) is the last product into O; its commit covers every earlier one
+            const bool w3 = mbar_wait_bounded(pv_done + 8 * (2 * t + ((nt - 1) & 1)), ((nt - 1) >> 1) & 1);
             if (__all_sync(0xffffffffu, w3)) {
                 tc_fence_after();
                 const float inv = l > 0.f ? p.out_scale / l : 0.f;
