@@ -493,9 +493,9 @@ __global__ void __launch_bounds__(FP8 ? 448 : 320, 1)
             }
             umma_commit(s_full + 8 * sb);
         };
-        auto issue_pv = [&](int t, int j) -> bool {
-            if (!mbar_wait_bounded(p_full + 8 * (2 * t + (j & 1)), (j >> 1) & 1)) return false;
-            if (!mbar_wait_bounded(v_ready + 8 * (j % kTcStages), (j / kTcStages) & 1)) return false;
+        auto issue_pv = [&](int t, int j, bool pre) -> bool {
+            if (!pre && !mbar_wait_bounded(p_full + 8 * (2 * t + (j & 1)), (j >> 1) & 1)) return false;
+            if (!pre && !mbar_wait_bounded(v_ready + 8 * (j % kTcStages), (j / kTcStages) & 1)) return false;
             tc_fence_after();
             const uint64_t dv = dvv0 + (uint64_t)(((j % kTcStages) * 2 * kTcKVBytes) >> 4);
             // P_t(j) from TMEM over its score buffer: 16 keys = 8 columns per k-step.  The
@@ -518,10 +518,16 @@ __global__ void __launch_bounds__(FP8 ? 448 : 320, 1)
                     if (j < ntq[t]) issue_s(t, j);
             }
             for (int j = 0; j < ntiles && alive && !*abort_flag; ++j) {
+                // every condition of this tile tested at once (their latencies overlap);
+                // the ordered bounded waits only when one is not met yet
+                uint32_t pre = mbar_try_wait(v_ready + 8 * (j % kTcStages), (j / kTcStages) & 1) ? 1u : 0u;
+                if (j < ntq[0]) pre &= mbar_try_wait(p_full + 8 * (j & 1), (j >> 1) & 1) ? 1u : 0u;
+                if (j < ntq[1]) pre &= mbar_try_wait(p_full + 8 * (2 + (j & 1)), (j >> 1) & 1) ? 1u : 0u;
+                if (j + 2 < ntiles) pre &= mbar_try_wait(kv_full + 8 * ((j + 2) % kTcStages), ((j + 2) / kTcStages) & 1) ? 1u : 0u;
                 for (int t = 0; t < kTcQT && alive; ++t) {
-                    if (j < ntq[t]) alive = issue_pv(t, j);
+                    if (j < ntq[t]) alive = issue_pv(t, j, pre != 0u);
                     if (alive && j + 2 < ntq[t]) {
-                        alive = kv_landed(j + 2);
+                        alive = pre != 0u || kv_landed(j + 2);
                         if (alive) issue_s(t, j + 2);
                     }
                 }
