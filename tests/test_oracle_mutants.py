@@ -50,6 +50,8 @@ MUTANTS = {
          "(pos + 2 <= context_lens[s2] ? pos + 2 : pos + 1), block_size, num_blocks, num_kv_heads, h / group,")],
     "prefill_head_mapping": ("pos + 1, block_size, num_blocks, num_kv_heads, h / group,",
                              "pos + 1, block_size, num_blocks, num_kv_heads, h % num_kv_heads,"),
+    "prefill_k_with_v_scale": ("h / group, head_dim, scale, k_scale,\n                         v_scale, scores, &m, &l, o)",
+                               "h / group, head_dim, scale, v_scale,\n                         v_scale, scores, &m, &l, o)"),
     "gather_wrong_slot": ("((size_t)blk * block_size + (size_t)(t % block_size)) * row_bytes, row_bytes);",
                           "((size_t)blk * block_size + (size_t)(t / block_size)) * row_bytes, row_bytes);"),
 }
@@ -74,6 +76,7 @@ def _pins(golden):
         P.test_swap_blocks_between_pools_of_different_sizes,
         lambda: [P.test_prefill_equals_numpy_causal_attention(*a) for a in [(2, 2), (8, 2)]],
         P.test_prefill_first_position_returns_v0, P.test_prefill_bf16_and_row_subset,
+        P.test_prefill_fp8_equals_numpy_causal_of_library_decoded_codes,
     ]
     return fns
 

@@ -539,6 +539,22 @@ def test_prefill_row_equals_decode_of_its_prefix():
         np.testing.assert_allclose(got[i], dec[0], rtol=1e-13, atol=1e-13)
 
 
+def test_prefill_fp8_equals_numpy_causal_of_library_decoded_codes():
+    """FP8 cache in the prefill: E4M3 codes times per-tensor scales (distinct for K
+    and V), against the causal brute force on torch's decoding of the same codes."""
+    q, kp, vp, tabs, lens, qs = _prefill_case(35, [45, 70], [45, 23], 8, 2, 32)
+    ks, vs = 0.0123, 0.0371
+    kc = torch.from_numpy(kp / ks).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    vc = torch.from_numpy(vp / vs).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    bits = lambda a: torch.from_numpy(a).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)  # noqa: E731
+    qb = bits(q)
+    got, bad = oracle.paged_attention_prefill(qb, oracle.BF16, kc, vc, FP8, tabs, lens, qs, 0.2, ks, vs)
+    assert bad == 0
+    ref = _numpy_causal(_library_values(qb, "bf16"), _library_values(kc, "fp8") * ks,
+                        _library_values(vc, "fp8") * vs, tabs, lens, qs, 0.2)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
 def test_prefill_bf16_and_row_subset():
     q, kp, vp, tabs, lens, qs = _prefill_case(34, [33, 70], [33, 40], 4, 2, 32)
     bits = lambda a: torch.from_numpy(a).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)  # noqa: E731
