@@ -373,25 +373,48 @@ def divergence_step(w, device, args):
             "us_decode": round(1e3 * dec, 2), "device_errors": int(step.err.item())}
 
 
+def pack_inputs(tensors, device, copies=1):
+    """One pinned host buffer holding the bytes of `tensors` (name -> tensor), and
+    `copies` device buffers of the same layout with a view per name in each, so that
+    a step's inputs go up in one copy.  Offsets are 256-byte aligned.  Returns
+    (host buffer, [device buffers], [views per device buffer], input bytes)."""
+    offs, total = {}, 0
+    for n, v in tensors.items():
+        offs[n] = total
+        total += -(-v.numel() * v.element_size() // 256) * 256
+    host = torch.empty(max(total, 256), dtype=torch.uint8).pin_memory()
+    for n, v in tensors.items():
+        nb = v.numel() * v.element_size()
+        host[offs[n]:offs[n] + nb].copy_(v.detach().cpu().contiguous().view(-1).view(torch.uint8))
+    devs, views = [], []
+    for _ in range(copies):
+        d = torch.empty(max(total, 256), dtype=torch.uint8, device=device)
+        devs.append(d)
+        views.append({n: d[offs[n]:offs[n] + v.numel() * v.element_size()].view(v.dtype).view(v.shape)
+                      for n, v in tensors.items()})
+    return host, devs, views, sum(v.numel() * v.element_size() for v in tensors.values())
+
+
 def time_e2e(step: Step, steps: int, warmup: int, world: int):
     """The same step through the public API from pinned HOST buffers.  Every
     step copies its inputs (q, new K/V, slots, tables, lengths, copy pairs)
     host->device and reads its output back device->host inside the timed
-    region.  The copies run on a second stream with two device input sets, so
-    step i+1's uploads and step i-1's download overlap step i's kernels, as in
-    a serving loop; the KV pools stay resident (they are the cache, not a
-    per-step input).  Uploads and downloads use separate streams."""
+    region.  The inputs are packed into one pinned buffer and go up in one copy
+    (per-copy overhead, not bytes, dominates a step's uploads); the copies run
+    on a second stream with two device input sets, so step i+1's uploads and
+    step i-1's download overlap step i's kernels, as in a serving loop; the KV
+    pools stay resident (they are the cache, not a per-step input).  Uploads
+    and downloads use separate streams."""
     compute = torch.cuda.current_stream()
     up = torch.cuda.Stream(device=step.device)
     down = torch.cuda.Stream(device=step.device)
     names = ["q", "k_new", "v_new", "g_slots", "g_tables", "g_lens"] + (["g_pairs"] if step.g_pairs is not None else [])
     if step.groups is not None:
         names += ["g_offs", "g_mem", "g_sh"]
-    host = {n: getattr(step, n).cpu().pin_memory() for n in names}
-    dev = [{n: getattr(step, n) for n in names}, {n: torch.empty_like(getattr(step, n)) for n in names}]
+    saved = {n: getattr(step, n) for n in names}
+    host, dev_bufs, dev, h2d = pack_inputs(saved, step.device, copies=2)
     outs = [step.out, torch.empty_like(step.out)]
     out_host = [torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory() for _ in range(2)]
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = out_host[0].numel() * out_host[0].element_size()
     uploaded = [torch.cuda.Event() for _ in range(2)]
     computed = [torch.cuda.Event() for _ in range(2)]
@@ -404,8 +427,7 @@ def time_e2e(step: Step, steps: int, warmup: int, world: int):
             with torch.cuda.stream(up):
                 if i >= 2:
                     up.wait_event(consumed[b])
-                for n in names:
-                    dev[b][n].copy_(host[n], non_blocking=True)
+                dev_bufs[b].copy_(host, non_blocking=True)
                 uploaded[b].record(up)
             compute.wait_event(uploaded[b])
             if i >= 2:
@@ -437,7 +459,7 @@ def time_e2e(step: Step, steps: int, warmup: int, world: int):
     z.record(compute)
     torch.cuda.synchronize()
     for n in names:
-        setattr(step, n, dev[0][n])
+        setattr(step, n, saved[n])
     step.out = outs[0]
     return a.elapsed_time(z), h2d, d2h
 
@@ -804,6 +826,83 @@ class BeamStep:
                                                err_count=self.err)
 
 
+def time_beam_e2e(step, idx, world):
+    """Beam steps `idx` through the public API from pinned HOST buffers: every step
+    uploads its inputs (slots, copy pairs, tables, lengths, prefix groups, new K/V,
+    q) and reads its output back.  A step's inputs are packed into one pinned buffer
+    and go up in one copy into a device buffer the step's tensors view; uploads run
+    on one stream and downloads on another, overlapping the neighbouring steps'
+    kernels; the output alternates between two buffers, with events ordering every
+    reuse.  The host block-manager decisions are reported apart
+    (host_block_manager_us_per_step).  Replaying a step is idempotent (same slots,
+    same data, same copies).  Returns (ms, h2d bytes per step, d2h bytes per step)."""
+    compute = torch.cuda.current_stream()
+    up = torch.cuda.Stream(device=step.device)
+    down = torch.cuda.Stream(device=step.device)
+    common = ["q", "k_new", "v_new"]
+    saved = {n: getattr(step, n) for n in common}
+    packed = {}
+    for t in set(idx):
+        parts = {k: v for k, v in step.steps[t].items() if isinstance(v, torch.Tensor)}
+        parts.update(saved)
+        host, devs, views, nbytes = pack_inputs(parts, step.device)
+        packed[t] = (host, devs[0], views[0], nbytes)
+    originals = {t: dict(step.steps[t]) for t in packed}
+    outs = [step.out, torch.empty_like(step.out)]
+    out_host = [torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory() for _ in range(2)]
+    h2d = sum(packed[t][3] for t in idx) // len(idx)
+    d2h = out_host[0].numel() * out_host[0].element_size()
+    uploaded = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    downloaded = [torch.cuda.Event() for _ in range(2)]
+
+    def run(ts):
+        for i, t in enumerate(ts):
+            b = i & 1
+            host, dev, views, _ = packed[t]
+            with torch.cuda.stream(up):
+                dev.copy_(host, non_blocking=True)
+                uploaded[b].record(up)
+            compute.wait_event(uploaded[b])
+            if i >= 2:
+                compute.wait_event(downloaded[b])
+            for k, v in views.items():
+                if k in common:
+                    setattr(step, k, v)
+                else:
+                    step.steps[t][k] = v
+            step.out = outs[b]
+            step.copy_and_write(t)
+            step.decode(t)
+            computed[b].record(compute)
+            with torch.cuda.stream(down):
+                down.wait_event(computed[b])
+                out_host[b].copy_(outs[b], non_blocking=True)
+                downloaded[b].record(down)
+        compute.wait_stream(up)
+        compute.wait_stream(down)
+
+    run(idx[:2])
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    z = torch.cuda.Event(enable_timing=True)
+    a.record(compute)
+    up.wait_event(a)
+    down.wait_event(a)
+    run(idx)
+    z.record(compute)
+    torch.cuda.synchronize()
+    for n in common:
+        setattr(step, n, saved[n])
+    for t, d in originals.items():
+        step.steps[t] = d
+    step.out = outs[0]
+    return reduce_max(a.elapsed_time(z), world, step.device), h2d, d2h
+
+
 def run_beam(args, w0, device, rank, world):
     w = rank_workload(w0, rank)
     step = BeamStep(w, device, args.warmup + args.steps)
@@ -838,6 +937,14 @@ def run_beam(args, w0, device, rank, world):
     value = kv * world / (total_ms / 1e3) / 1e9
     dec_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
     cw_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
+    e2e = None
+    if not args.no_e2e:
+        n_e = max(3, args.steps // 4)
+        idx = [args.warmup + i % args.steps for i in range(n_e)]
+        e_ms, h2d, d2h = time_beam_e2e(step, idx, world)
+        e_kv = sum(step.steps[t]["kv_bytes"] for t in idx)
+        e2e = {"value": round(e_kv * world / (e_ms / 1e3) / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms / n_e, 4)}
     peak, peak_kind = measured_peak_hbm()
     achieved = kv / args.steps / (dec_ms / 1e3) / 1e9
     if rank == 0:
@@ -859,7 +966,7 @@ def run_beam(args, w0, device, rank, world):
                          "frac": round(achieved / peak, 4), "traffic": None,
                          "kernel": "paged_attention_decode_shared call (logical bytes; shared prompt read once per "
                                    "request)", "peak_source": peak_kind},
-            "cpu_baseline": cpu, "e2e": None, "gpu_launches": sum(4 + (st["npairs"] > 0) for st in timed),
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": sum(4 + (st["npairs"] > 0) for st in timed),
             "device_errors": int(step.err.item()), "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)
