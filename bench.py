@@ -395,7 +395,7 @@ def pack_inputs(tensors, device, copies=1):
     return host, devs, views, sum(v.numel() * v.element_size() for v in tensors.values())
 
 
-def time_e2e(step: Step, steps: int, warmup: int, world: int):
+def time_e2e(step, steps: int, warmup: int, world: int, names=None):
     """The same step through the public API from pinned HOST buffers.  Every
     step copies its inputs (q, new K/V, slots, tables, lengths, copy pairs)
     host->device and reads its output back device->host inside the timed
@@ -408,9 +408,11 @@ def time_e2e(step: Step, steps: int, warmup: int, world: int):
     compute = torch.cuda.current_stream()
     up = torch.cuda.Stream(device=step.device)
     down = torch.cuda.Stream(device=step.device)
-    names = ["q", "k_new", "v_new", "g_slots", "g_tables", "g_lens"] + (["g_pairs"] if step.g_pairs is not None else [])
-    if step.groups is not None:
-        names += ["g_offs", "g_mem", "g_sh"]
+    if names is None:   # a decode Step
+        names = ["q", "k_new", "v_new", "g_slots", "g_tables", "g_lens"] + (
+            ["g_pairs"] if step.g_pairs is not None else [])
+        if step.groups is not None:
+            names += ["g_offs", "g_mem", "g_sh"]
     saved = {n: getattr(step, n) for n in names}
     host, dev_bufs, dev, h2d = pack_inputs(saved, step.device, copies=2)
     outs = [step.out, torch.empty_like(step.out)]
@@ -629,6 +631,10 @@ class PrefillStep:
         self.pkv.paged_kv_write(self.k_new, self.v_new, self.g_slots, self.k_pool, self.v_pool, self.k_scale,
                                 self.v_scale, err_count=self.err)
 
+    def run(self):
+        self.write()
+        self.attend()
+
     def attend(self):
         self.pkv.paged_attention_prefill(self.out, self.q, self.k_pool, self.v_pool, self.g_tables, self.g_lens,
                                          self.g_qs, self.w.scale, self.max_q, err_count=self.err,
@@ -707,31 +713,12 @@ def run_prefill(args, w0, device, rank, world):
 
     e2e = None
     if not args.no_e2e:
-        # through the public API from pinned host buffers: inputs up, output down, every step
-        names = ["q", "k_new", "v_new", "g_slots", "g_tables", "g_lens", "g_qs"]
-        host = {n: getattr(step, n).cpu().pin_memory() for n in names}
-        out_host = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in host.values())
-        d2h = out_host.numel() * out_host.element_size()
+        # through the public API from pinned host buffers: inputs up, output down, every
+        # step, pipelined as the decode lines are (time_e2e)
         n_e = max(3, args.steps // 4)
-
-        def e2e_step():
-            for n in names:
-                getattr(step, n).copy_(host[n], non_blocking=True)
-            step.write()
-            step.attend()
-            out_host.copy_(step.out, non_blocking=True)
-
-        for _ in range(2):
-            e2e_step()
-        torch.cuda.synchronize()
-        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(n_e):
-            e2e_step()
-        z.record(stream)
-        torch.cuda.synchronize()
-        e_ms = reduce_max(a.elapsed_time(z), world, device)
+        e_ms, h2d, d2h = time_e2e(step, n_e, 2, world,
+                                  names=["q", "k_new", "v_new", "g_slots", "g_tables", "g_lens", "g_qs"])
+        e_ms = reduce_max(e_ms, world, device)
         e2e = {"value": round(step.flops * world * n_e / (e_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms / n_e, 4)}
 

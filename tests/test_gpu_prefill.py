@@ -179,6 +179,21 @@ def test_full_size_prefill_sampled_rows():
     assert_close(got[rows], ref[rows], "bf16", "prefill70b")
 
 
+def test_full_size_fp8_prefill_sampled_rows():
+    """The FP8-cache prompt pass as bench.py times it (16 prompts of 512..4,096
+    tokens, 64/8 heads, scales amax/448 of the prompts' K and V); rows sampled."""
+    w = W.WORKLOADS["prefill70b_fp8"]
+    lens = W.context_lens(w)
+    c = PrefillCase(w.num_heads, w.num_kv_heads, lens, lens, seed=w.seed, nan_pool=False, cache="fp8")
+    got = out_to_f64(c.run())
+    assert int(c.err.item()) == 0
+    rng = np.random.default_rng(47)
+    rows = np.sort(rng.choice(int(c.qs[-1]), 48, replace=False))
+    rows = np.unique(np.concatenate([rows, c.qs[1:] - 1, c.qs[:-1]]))
+    ref, _ = c.oracle(rows=rows)
+    assert_close(got[rows], ref[rows], "fp8", "prefill70b_fp8")
+
+
 def test_warp_mma_kernel_agrees(tmp_path):
     """The mma.sync prefill kernel (PKV_PREFILL_KERNEL=mma, a separate process)
     gives the oracle's result on the ragged case too."""
