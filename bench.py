@@ -97,6 +97,14 @@ def reduce_max(value: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def spread_us(ms_list):
+    """p10 / median / p90 of per-step times (ms in, us out)."""
+    ys = sorted(ms_list)
+    at = lambda f: ys[min(len(ys) - 1, int(round(f * (len(ys) - 1))))]  # noqa: E731
+    return {"p10": round(1e3 * at(0.1), 2), "median": round(1e3 * statistics.median(ys), 2),
+            "p90": round(1e3 * at(0.9), 2)}
+
+
 def rank_workload(w: W.Workload, rank: int) -> W.Workload:
     """Weak scaling: each rank gets an independent batch of the same shape (its own seed)."""
     return W.scaled(w, seed=w.seed + 1000 * rank) if rank else w
@@ -742,6 +750,7 @@ def run_prefill(args, w0, device, rank, world):
                            step.q.numel() * 2 / 1e6, 2 * step.k_pool.numel() * step.k_pool.element_size() / 1e6)},
             "prompt_tokens_per_s": round(step.total * world * args.steps / (total_ms / 1e3), 1),
             "us_attention": round(1e3 * att_ms, 2), "us_write": round(1e3 * wr_ms, 2),
+            "us_attention_spread": spread_us([b.elapsed_time(c) for _, b, c in ev]),
             "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(achieved / peak, 4), "traffic": ncu_traffic(w0.name),
                          "kernel": "prefill_tc_kernel (tcgen05.mma, TMEM accumulators)" if os.environ.get("PKV_PREFILL_KERNEL", "")[:1] != "m" else "prefill_kernel (mma.sync m16n8k16)", "peak_source": peak_kind},
@@ -947,6 +956,7 @@ def run_beam(args, w0, device, rank, world):
                        "seq_len": step.max_len, "parallelism": "replicas: requests sharded by rank, no collective",
                        "l2": "logical KV bytes counted (the prompt is shared by the 4 beams of a request)"},
             "us_decode": round(1e3 * dec_ms, 2), "us_copy_and_write": round(1e3 * cw_ms, 2),
+            "us_decode_spread": spread_us([b.elapsed_time(c) for _, b, c in ev]),
             "copy_pairs_per_step": round(sum(st["npairs"] for st in timed) / args.steps, 2),
             "host_block_manager_us_per_step": round(step.host_us_per_step, 1),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
@@ -1159,6 +1169,7 @@ def main(argv=None):
             "seq_tokens_per_s": round(step.seq_tokens * world * args.steps / (max_ms / 1e3), 1),
             "us_per_step_per_layer": round(1e3 * ms_per_step, 2),
             "us_decode": round(1e3 * dec_ms, 2), "us_write": round(1e3 * statistics.mean(write_ms), 2),
+            "us_decode_spread": spread_us(decode_ms),
             "pct_of_8tbps": round(100 * value / world / NOMINAL_HBM_GBS, 2),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": step.launches * args.steps, "device_errors": err,
