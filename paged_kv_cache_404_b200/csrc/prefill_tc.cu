@@ -15,29 +15,29 @@
 //    (past its end, or a block past the table or with a bad id) are zeroed in
 //    shared memory, so that a zero probability never meets a NaN there;
 //  - warp 9 (MMA): one thread issues tcgen05.mma: per Q tile t, S_t = Q_t K^T
-//    (M=128, N=64, K=128, bf16 -> fp32; Q_t from TMEM, K from shared memory) into
-//    TMEM, then O_t += P_t V (P_t from TMEM, V MN-major from shared memory) into a
-//    TMEM accumulator; tcgen05.commit signals mbarriers; the warp allocates and
-//    frees the 512 TMEM columns;
+//    (M=128, N=64, K=128, bf16 -> fp32; Q_t and K from shared memory) into one of
+//    two TMEM score buffers, then O_t += P_t V (P_t from TMEM, V MN-major from
+//    shared memory) into a TMEM accumulator; tcgen05.commit signals mbarriers; the
+//    warp allocates and frees the 512 TMEM columns;
 //  - warps 0-3 and 4-7 (softmax, one warpgroup per Q tile): thread r owns
-//    query row r of its tile (TMEM lane r): first moves its row of Q from the
-//    TMA-landed tile into TMEM; then per KV tile loads its 64 scores with
+//    query row r of its tile (TMEM lane r): per KV tile loads its 64 scores with
 //    tcgen05.ld, applies the causal mask, runs the online softmax in base 2 (the
 //    reference max moves only when a score exceeds it by more than 2^8, then O is
 //    rescaled in TMEM), writes P as 16-bit pairs into TMEM over the scores it
 //    has read, and finally normalises O and stores the row.
-// The products are issued PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), ..., so that
-// each warpgroup's softmax runs while the tensor core works for the other.
-// Keeping Q and P in TMEM leaves shared memory only the K and V reads of the
-// products.
+// Each Q tile's scores alternate between two TMEM buffers: S_t(j+2) is issued right
+// after PV_t(j) (which reads P_t(j) from the buffer it then overwrites; the tensor
+// core runs one thread's products in issue order), so the softmax of tile j+1 runs
+// while the tensor core does PV_t(j) and S_t(j+2), and each warpgroup's softmax
+// overlaps the other's products.
 //
 // FP8 E4M3 cache (14 warps): the products run in f16, which holds every E4M3
 // value exactly.  Warp 8 TMA-loads the codes (128-byte rows) into a 2-deep
 // staging ring; warps 10-13 each turn one 16-slot block of a tile into f16 in the
 // ring the tensor core reads (and zero V where no token is), then arrive on the
-// stage's barriers; the softmax warps take Q into f16 on its way to TMEM and
-// write P as f16.  k_scale folds into the score scale and v_scale into the final
-// normalisation.
+// stage's barriers; the softmax warps first turn their Q tile from bf16 into f16
+// in place and write P as f16.  k_scale folds into the score scale and v_scale
+// into the final normalisation.
 #include "pkv_common.cuh"
 
 namespace pkv {
