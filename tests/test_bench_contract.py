@@ -1,0 +1,64 @@
+"""The benchmark's one-line JSON report: the keys and invariants its readers rely on.
+
+The reference arm (the fp64 oracle on the host cores) runs here on the CPU; the
+device arm runs a short default step on the GPU.
+"""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+COMMON = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+          "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"}
+
+
+def _run(args, timeout):
+    env = dict(os.environ)
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        env.pop(k, None)
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py")] + args, cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=timeout)
+    assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout[-2000:]       # exactly one JSON line
+    return json.loads(lines[0])
+
+
+def _check_common(d):
+    missing = COMMON - set(d)
+    assert not missing, missing
+    assert d["n_gpus"] == 1 and d["scaling"] == "weak" and d["higher_is_better"] is True
+    assert d["value"] > 0 and d["ms_per_step"] > 0 and d["warmup"] >= 3
+    assert isinstance(d["config"], dict) and d["config"]["workload"].startswith("gqa70b")
+    e = d["e2e"]
+    assert {"value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"} <= set(e) and e["unit"] == d["unit"]
+
+
+def test_reference_arm_line():
+    d = _run(["--impl", "reference", "--steps", "1", "--warmup", "3"], timeout=600)
+    _check_common(d)
+    assert d["impl"] == "reference" and d["dtype"] == "f64"
+    c = d["cpu_baseline"]
+    assert c["kind"] == "oracle" and c["cores"] >= 1 and c["sample"] and c["value"] == d["value"]
+    assert d["e2e"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+@pytest.mark.gpu
+def test_device_arm_line():
+    d = _run(["--steps", "5", "--warmup", "3", "--no-cpu-baseline"], timeout=900)
+    _check_common(d)
+    assert "impl" not in d or d["impl"] != "reference"
+    r = d["roofline"]
+    assert {"bound", "achieved", "peak", "unit", "frac", "traffic"} <= set(r)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-3
+    assert 0.3 < r["frac"] < 1.3                       # above 1 a little is possible; far above is a bug
+    assert d["gpu_launches"] > 0 and d["device_errors"] == 0
+    assert d["e2e"]["h2d_bytes_per_step"] > 0 and d["e2e"]["d2h_bytes_per_step"] > 0
+    c = d["clocks"]
+    assert {"sm_mhz", "sm_max_mhz", "reasons"} <= set(c)
+    s = d["us_decode_spread"]
+    assert s["p10"] <= s["median"] <= s["p90"]
