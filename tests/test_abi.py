@@ -117,3 +117,31 @@ def test_python_binding_refuses_cpu_tensors():
     pool = torch.zeros(4, 16, 8, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         pkv.paged_kv_write(k, k, torch.zeros(1, dtype=torch.int64), pool, pool)
+
+
+def _prefill(L, **kw):
+    a = dict(out=FAKE, q=FAKE, qdt=L.PKV_BF16, kp=FAKE, vp=FAKE, cdt=L.PKV_BF16, bt=FAKE, mb=256, cl=FAKE, qs=FAKE,
+             S=4, T=4096, mq=1024, nb=1024, bs=16, hq=64, hkv=8, d=128, ks=1.0, vs=1.0, err=None)
+    a.update(kw)
+    return L.lib().pkv_paged_attention_prefill(
+        a["out"], a["q"], a["qdt"], a["kp"], a["vp"], a["cdt"], a["bt"], a["mb"], a["cl"], a["qs"], a["S"], a["T"],
+        a["mq"], a["nb"], a["bs"], a["hq"], a["hkv"], a["d"], 0.088, a["ks"], a["vs"], a["err"], None)
+
+
+def test_prefill_validation(L):
+    assert _prefill(L, S=0) == L.PKV_OK                     # nothing to do, no CUDA call
+    assert _prefill(L, mq=0) == L.PKV_OK
+    assert _prefill(L, S=-1) == L.PKV_EINVAL
+    assert _prefill(L, mb=0) == L.PKV_EINVAL
+    assert _prefill(L, hq=60) == L.PKV_EINVAL               # 60 % 8 != 0
+    assert _prefill(L, bs=32) == L.PKV_EUNSUPPORTED
+    assert _prefill(L, qdt=L.PKV_F32) == L.PKV_EUNSUPPORTED
+    assert _prefill(L, cdt=L.PKV_F32) == L.PKV_EUNSUPPORTED
+    assert _prefill(L, d=64) == L.PKV_EUNSUPPORTED
+    assert _prefill(L, cdt=L.PKV_FP8_E4M3, ks=float("nan")) == L.PKV_EINVAL
+    assert _prefill(L, cdt=L.PKV_FP8_E4M3, vs=float("inf")) == L.PKV_EINVAL
+    assert _prefill(L, S=70000) == L.PKV_EUNSUPPORTED       # grid y limit
+    assert _prefill(L, out=None) == L.PKV_EINVAL
+    assert _prefill(L, qs=None) == L.PKV_EINVAL
+    assert _prefill(L, q=ODD) == L.PKV_EINVAL
+    assert _prefill(L, cl=C.c_void_p(0x10002)) == L.PKV_EINVAL   # int32 arrays must be 4-byte aligned
