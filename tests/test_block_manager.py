@@ -351,3 +351,106 @@ def test_fork_many_and_free_many_equal_single_calls(BM):
     with pytest.raises(PagedKVError):
         a.fork_many([1, 99])           # unknown parent: nothing forked
     assert a.fork_many([1]).tolist() == [6]
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2, 3])
+def test_mixed_feature_traces_match_reference(BM, seed):
+    """Every feature at once: prefix caching (hits on live and on free cached
+    blocks), plain allocation, fork, release, single and batched appends with
+    copy-on-write, swap out / in (whose fresh blocks may evict cached keys) and
+    prefix groups of resident batches.  Same results and state as the reference."""
+    from paged_kv_cache_404_b200 import PagedKVError
+    rng = np.random.default_rng(700 + seed)
+    NB, NH = 200, 120
+    order = rng.permutation(NB)
+    bm, ref = BM(NB, 16, free_order=order), RefBlockManager(NB, 16, free_order=order)
+    for m in (bm, ref):
+        m.set_prefix_cache(True)
+        m.set_host_pool(NH)
+    systems = [rng.integers(0, 40, size=int(rng.integers(16, 80))).tolist() for _ in range(3)]
+    live = []
+
+    def resident():
+        return [s for s in live if s not in ref.swapped]
+
+    for step in range(3000):
+        op = int(rng.integers(0, 14))
+        if op <= 2 or not live:
+            toks = systems[int(rng.integers(len(systems)))] + rng.integers(0, 3, size=int(rng.integers(0, 30))).tolist()
+            try:
+                exp = ref.alloc_seq_tokens(toks)
+            except MemoryError:
+                with pytest.raises(PagedKVError):
+                    bm.alloc_seq_tokens(toks)
+                continue
+            assert bm.alloc_seq_tokens(toks) == exp
+            live.append(exp[0])
+        elif op == 3:
+            n = int(rng.integers(0, 50))
+            try:
+                r = ref.alloc_seq(n)
+            except MemoryError:
+                with pytest.raises(PagedKVError):
+                    bm.alloc_seq(n)
+                continue
+            assert bm.alloc_seq(n) == r
+            live.append(r)
+        elif op == 4 and len(live) > 1:
+            s = live.pop(int(rng.integers(len(live))))
+            ref.free_seq(s)
+            bm.free_seq(s)
+        elif op == 5:
+            res = resident()
+            if not res:
+                continue
+            s = res[int(rng.integers(len(res)))]
+            r = ref.fork(s)
+            assert bm.fork(s) == r
+            live.append(r)
+        elif op == 6:
+            s = live[int(rng.integers(len(live)))]
+            swap = ref.swap_in if s in ref.swapped else ref.swap_out
+            native = bm.swap_in if s in ref.swapped else bm.swap_out
+            try:
+                exp = swap(s)
+            except MemoryError:
+                with pytest.raises(PagedKVError):
+                    native(s)
+                continue
+            assert [tuple(p) for p in native(s).tolist()] == exp
+        elif op == 7:
+            res = resident()
+            if len(res) < 2:
+                continue
+            batch = [res[int(i)] for i in rng.choice(len(res), size=int(rng.integers(2, len(res) + 1)), replace=False)]
+            offs, mem, sh = bm.prefix_groups(batch)
+            assert (offs.tolist(), mem.tolist(), sh.tolist()) == tuple(ref.prefix_groups(batch))
+        elif op <= 10:
+            res = resident()
+            if not res:
+                continue
+            batch = [res[int(i)] for i in rng.choice(len(res), size=min(len(res), int(rng.integers(1, 6))),
+                                                       replace=False)]
+            if len(batch) > ref.num_free():
+                continue                       # a batch that cannot fail part-way
+            exp = [ref.append_token(s) for s in batch]
+            slots, pairs = bm.append_tokens(batch)
+            assert slots.tolist() == [e[0] for e in exp]
+            assert [tuple(p) for p in pairs.tolist()] == [e[1] for e in exp if e[1] is not None]
+        else:
+            res = resident()
+            if not res:
+                continue
+            s = res[int(rng.integers(len(res)))]
+            try:
+                exp = ref.append_token(s)
+            except MemoryError:
+                with pytest.raises(PagedKVError):
+                    bm.append_token(s)
+                continue
+            assert bm.append_token(s) == exp
+        if step % 150 == 0:
+            _same_state(bm, ref, live)
+            assert bm.num_cached_blocks() == len(ref.cache)
+    _same_state(bm, ref, live)
+    assert bm.num_cached_blocks() == len(ref.cache)
