@@ -454,3 +454,45 @@ def test_mixed_feature_traces_match_reference(BM, seed):
             assert bm.num_cached_blocks() == len(ref.cache)
     _same_state(bm, ref, live)
     assert bm.num_cached_blocks() == len(ref.cache)
+
+
+def test_batched_append_stops_at_the_first_sequence_out_of_blocks(BM):
+    """One pkv_bm_append_tokens call that runs out of blocks part-way: it returns
+    PKV_ENOMEM, reports how many sequences got their slot, those keep it (with
+    their copy-on-write pairs), the failing sequence and the rest are unchanged."""
+    import ctypes as C
+    from paged_kv_cache_404_b200 import _lib as L
+    order = list(range(12))
+    bm, ref = BM(12, 16, free_order=order), RefBlockManager(12, 16, free_order=order)
+    # a: 3 full blocks (its next token needs a block); b: a fork of c (copy-on-write);
+    # c: 2 blocks with room; d: 1 full block
+    seqs = []
+    for m in (bm, ref):
+        a = m.alloc_seq(48)
+        c = m.alloc_seq(20)
+        b = m.fork(c)
+        d = m.alloc_seq(16)
+        seqs = [a, b, c, d]
+    assert ref.num_free() == 12 - 3 - 2 - 1
+    # use up all but 2 free blocks
+    for m in (bm, ref):
+        m.alloc_seq(16 * 4)
+    batch = seqs                      # a takes 1 block, b 1 (copy-on-write), c writes in place, d finds none
+    exp = []
+    for s in batch:
+        try:
+            exp.append(ref.append_token(s))
+        except MemoryError:
+            break
+    assert len(exp) == 3 and ref.num_free() == 0
+    arr = np.asarray(batch, dtype=np.int32)
+    slots = np.empty(4, dtype=np.int64)
+    pairs = np.empty((4, 2), dtype=np.int64)
+    npairs, ndone = C.c_int(), C.c_int()
+    st = bm._lib.pkv_bm_append_tokens(bm._h, arr.ctypes.data, 4, slots.ctypes.data, pairs.ctypes.data,
+                                      C.byref(npairs), C.byref(ndone))
+    assert st == L.PKV_ENOMEM and ndone.value == 3
+    assert slots[:3].tolist() == [e[0] for e in exp]
+    assert [tuple(p) for p in pairs[:npairs.value].tolist()] == [e[1] for e in exp if e[1] is not None]
+    _same_state(bm, ref, seqs)        # d unchanged on both sides
+    assert bm.seq_len(seqs[3]) == 16
