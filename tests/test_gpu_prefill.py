@@ -194,6 +194,20 @@ def test_full_size_fp8_prefill_sampled_rows():
     assert_close(got[rows], ref[rows], "fp8", "prefill70b_fp8")
 
 
+@pytest.mark.parametrize("cache", ["bf16", "fp8"])
+def test_context_past_the_shared_memory_validity_bits(cache):
+    """A 33,000-token context (2,063 blocks): past the 2,048 blocks whose validity
+    the kernel keeps in shared memory, block ids are checked per tile from the
+    table; a bad id there is skipped and counted once."""
+    c = PrefillCase(8, 8, [33000], [200], seed=48, nan_pool=False, cache=cache)
+    tabs = c.tables.copy()
+    tabs[0, 2055] = -1
+    got = out_to_f64(c.run(tables=tabs))
+    ref, bad = c.oracle(tables=tabs)
+    assert bad == 1 and int(c.err.item()) == 1
+    assert_close(got, ref, cache, "33k context %s" % cache)
+
+
 def test_warp_mma_kernel_agrees(tmp_path):
     """The mma.sync prefill kernel (PKV_PREFILL_KERNEL=mma, a separate process)
     gives the oracle's result on the ragged case too."""
