@@ -851,12 +851,16 @@ def time_beam_e2e(step, idx, world):
     uploaded = [torch.cuda.Event() for _ in range(2)]
     computed = [torch.cuda.Event() for _ in range(2)]
     downloaded = [torch.cuda.Event() for _ in range(2)]
+    consumed = {t: torch.cuda.Event() for t in packed}   # step t's device inputs read: free to refill
+    used = set()                                          # steps whose `consumed` has been recorded
 
     def run(ts):
         for i, t in enumerate(ts):
             b = i & 1
             host, dev, views, _ = packed[t]
             with torch.cuda.stream(up):
+                if t in used:                              # a repeated step index (fewer steps than uploads)
+                    up.wait_event(consumed[t])
                 dev.copy_(host, non_blocking=True)
                 uploaded[b].record(up)
             compute.wait_event(uploaded[b])
@@ -871,6 +875,8 @@ def time_beam_e2e(step, idx, world):
             step.copy_and_write(t)
             step.decode(t)
             computed[b].record(compute)
+            consumed[t].record(compute)
+            used.add(t)
             with torch.cuda.stream(down):
                 down.wait_event(computed[b])
                 out_host[b].copy_(outs[b], non_blocking=True)
