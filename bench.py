@@ -753,7 +753,7 @@ def run_prefill(args, w0, device, rank, world):
             "us_attention_spread": spread_us([b.elapsed_time(c) for _, b, c in ev]),
             "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(achieved / peak, 4), "traffic": ncu_traffic(w0.name),
-                         "kernel": "prefill_tc_kernel (tcgen05.mma, TMEM accumulators)" if os.environ.get("PKV_PREFILL_KERNEL", "")[:1] != "m" else "prefill_kernel (mma.sync m16n8k16)", "peak_source": peak_kind},
+                         "kernel": "prefill_tc_kernel (tcgen05.mma, TMEM accumulators)", "peak_source": peak_kind},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps, "device_errors": int(step.err.item()),
             "clocks": clk.summary(),
         }

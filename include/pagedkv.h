@@ -184,13 +184,18 @@ int pkv_paged_attention_decode(void* out, const void* q, int q_dtype,
  * scratch is a device array of PKV_NOALLOC_SCRATCH_BYTES that the library
  * declares at file scope.  Every GPU that loads the library's kernels holds
  * that array until the process exits.
- *  - Limit: returns PKV_EINVAL, before any CUDA call, when the scratch these
- *    bounds need (pkv_decode_workspace_bytes(num_seqs, num_heads, head_dim,
- *    max_context_len, partition_tokens)) exceeds PKV_NOALLOC_SCRATCH_BYTES;
- *    a larger partition_tokens lowers the need.
- *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress, with that device current) and caches it; make that
- *    first call before any stream capture.
+ *  - Checks: first every argument check of pkv_paged_attention_decode (same
+ *    statuses: PKV_EUNSUPPORTED for an unsupported configuration whatever its
+ *    size), then the limit: PKV_EINVAL, before any CUDA call, when the scratch
+ *    these bounds need (pkv_decode_workspace_bytes(num_seqs, num_heads,
+ *    head_dim, max_context_len, partition_tokens)) exceeds
+ *    PKV_NOALLOC_SCRATCH_BYTES; a need of exactly that size is accepted.  A
+ *    larger partition_tokens lowers the need.
+ *  - The first call in a device's context looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current) and keeps it for later
+ *    calls in the same context; a context that was destroyed and created again
+ *    (cudaDeviceReset) is recognised by its driver context id and gets a new
+ *    lookup.  Make the first call on each device before any stream capture.
  *  - All calls share the one array and it keeps the last call's contents;
  *    nothing in it needs clearing (each call's first kernel rewrites what the
  *    others read).  Calls whose GPU work overlaps (different streams without
@@ -276,9 +281,6 @@ int pkv_paged_attention_decode_shared(void* out, const void* q, int q_dtype,
  * accumulators).  With an FP8 cache the codes become f16 in shared memory
  * (exactly) and q is taken into f16 (exact inside the f16 range; entries past
  * +-65504 saturate there), so both operands of every product are f16.
- * Setting the environment variable PKV_PREFILL_KERNEL=mma before the first
- * call selects the warp-level mma.sync kernel instead (same results, bf16
- * cache only: an FP8 cache then returns PKV_EUNSUPPORTED; for comparison).
  * Host errors, returned before any CUDA call: PKV_EINVAL for negative sizes,
  * max_blocks_per_seq <= 0, num_heads not a multiple of num_kv_heads, a null
  * pointer, a pointer not 16-byte (out, q, pools) or 4-byte (int32 arrays)

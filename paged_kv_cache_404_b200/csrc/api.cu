@@ -4,7 +4,6 @@
 #include <cudaTypedefs.h>
 
 #include <cmath>
-#include <cstdlib>
 
 #include "pagedkv.h"
 #include "pkv_common.cuh"
@@ -24,8 +23,6 @@ cudaError_t launch_decode_f32(const DecodeParams& p, int num_sms, cudaStream_t s
 int decode_tc_warps(bool fp8, int head_dim, bool grouped);
 bool decode_tc_groupable(bool fp8, int head_dim, int group);
 cudaError_t launch_decode_merge(const DecodeParams& p, int out_dtype, cudaStream_t stream);
-cudaError_t launch_prefill(const CUtensorMap& tmK, const CUtensorMap& tmV, const PrefillParams& p, int max_query_len,
-                           cudaStream_t stream);
 cudaError_t launch_prefill_tc(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                               const PrefillParams& p, bool fp8, int max_query_len, cudaStream_t stream);
 }  // namespace pkv
@@ -36,11 +33,8 @@ namespace {
 
 // Smallest partition the automatic plan considers, and how many units per
 // warp it aims for before it stops halving the partition.
-#ifndef PKV_UNITS_PER_WORKER
-#define PKV_UNITS_PER_WORKER 3
-#endif
 constexpr int kMinAutoPartition = 256;
-constexpr int kUnitsPerWorker = PKV_UNITS_PER_WORKER;
+constexpr int kUnitsPerWorker = 3;
 constexpr int kMaxCandidates = 12;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -98,16 +92,6 @@ bool rows_tensor_map(CUtensorMap* map, const void* base, int head_dim, int heads
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
-}
-
-// Prefill kernel: 0 = tcgen05 (default), 1 = mma.sync (PKV_PREFILL_KERNEL=mma, for comparison).
-int prefill_kernel_choice() {
-    static int choice = -1;
-    if (choice < 0) {
-        const char* v = getenv("PKV_PREFILL_KERNEL");
-        choice = (v != nullptr && v[0] == 'm') ? 1 : 0;
-    }
-    return choice;
 }
 
 int min_partition_of(int partition_tokens) {
@@ -236,13 +220,15 @@ int pkv_paged_attention_decode_shared(void* out, const void* q, int q_dtype, con
 
 }  // extern "C"
 
-namespace {
+namespace pkv {
 
-int decode_impl(void* out, const void* q, int q_dtype, const void* k_pool, const void* v_pool, int cache_dtype,
-                const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
-                int max_context_len, int num_blocks, int block_size, int num_heads, int num_kv_heads, int head_dim,
-                float scale, float k_scale, float v_scale, int partition_tokens, const PrefixGroups& pg,
-                void* workspace, size_t workspace_bytes, int32_t* err_count, void* stream) {
+// Every host-side check of the decode except those of its workspace; PKV_OK
+// with num_seqs == 0 means there is nothing to launch.
+int decode_check_args(const void* out, const void* q, int q_dtype, const void* k_pool, const void* v_pool,
+                      int cache_dtype, const int32_t* block_tables, int max_blocks_per_seq,
+                      const int32_t* context_lens, int num_seqs, int max_context_len, int num_blocks, int block_size,
+                      int num_heads, int num_kv_heads, int head_dim, float k_scale, float v_scale,
+                      int partition_tokens, const int32_t* err_count) {
     if (num_seqs < 0 || max_blocks_per_seq <= 0 || max_context_len < 0 || num_blocks <= 0 || block_size <= 0 ||
         num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || partition_tokens < 0)
         return PKV_EINVAL;
@@ -254,16 +240,35 @@ int decode_impl(void* out, const void* q, int q_dtype, const void* k_pool, const
     const bool bf16 = q_dtype == PKV_BF16 && cache_dtype == PKV_BF16;
     const bool fp8 = q_dtype == PKV_BF16 && cache_dtype == PKV_FP8_E4M3;
     if (!f32 && !bf16 && !fp8) return PKV_EUNSUPPORTED;
-    const int group = num_heads / num_kv_heads;
-    if (!f32 && group > 16) return PKV_EUNSUPPORTED;
+    if (!f32 && num_heads / num_kv_heads > 16) return PKV_EUNSUPPORTED;
     if (fp8 && head_dim != 128) return PKV_EUNSUPPORTED;
     if (fp8 && !(k_scale > 0.f && v_scale > 0.f)) return PKV_EINVAL;
     if (num_seqs == 0) return PKV_OK;
-    if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens || !workspace) return PKV_EINVAL;
+    if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens) return PKV_EINVAL;
     if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) ||
-        !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(workspace, 256) ||
-        !aligned(err_count, 4))
+        !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(err_count, 4))
         return PKV_EINVAL;
+    return PKV_OK;
+}
+
+}  // namespace pkv
+
+namespace {
+
+int decode_impl(void* out, const void* q, int q_dtype, const void* k_pool, const void* v_pool, int cache_dtype,
+                const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
+                int max_context_len, int num_blocks, int block_size, int num_heads, int num_kv_heads, int head_dim,
+                float scale, float k_scale, float v_scale, int partition_tokens, const PrefixGroups& pg,
+                void* workspace, size_t workspace_bytes, int32_t* err_count, void* stream) {
+    const int status = decode_check_args(out, q, q_dtype, k_pool, v_pool, cache_dtype, block_tables,
+                                         max_blocks_per_seq, context_lens, num_seqs, max_context_len, num_blocks,
+                                         block_size, num_heads, num_kv_heads, head_dim, k_scale, v_scale,
+                                         partition_tokens, err_count);
+    if (status != PKV_OK || num_seqs == 0) return status;
+    if (!workspace || !aligned(workspace, 256)) return PKV_EINVAL;
+    const bool f32 = q_dtype == PKV_F32;
+    const bool fp8 = cache_dtype == PKV_FP8_E4M3;
+    const int group = num_heads / num_kv_heads;
     const int max_parts = max_parts_of(max_context_len, partition_tokens);
     const WsLayout ws = pg.layout ? ws_layout_shared(num_seqs, num_heads, head_dim, max_parts)
                                   : ws_layout(num_seqs, num_heads, head_dim, max_parts);
@@ -361,7 +366,6 @@ int pkv_paged_attention_prefill(void* out, const void* q, int q_dtype, const voi
     if (block_size != kBlockSize) return PKV_EUNSUPPORTED;
     const bool fp8 = cache_dtype == PKV_FP8_E4M3;
     if (q_dtype != PKV_BF16 || (cache_dtype != PKV_BF16 && !fp8) || head_dim != 128) return PKV_EUNSUPPORTED;
-    if (fp8 && prefill_kernel_choice() == 1) return PKV_EUNSUPPORTED;  // the mma.sync kernel reads bf16 only
     if (fp8 && !(std::isfinite(k_scale) && std::isfinite(v_scale))) return PKV_EINVAL;
     if (num_seqs == 0 || max_query_len == 0 || total_query_tokens == 0) return PKV_OK;
     if (num_seqs > 65535 || num_heads > 65535) return PKV_EUNSUPPORTED;
@@ -388,15 +392,10 @@ int pkv_paged_attention_prefill(void* out, const void* q, int q_dtype, const voi
     if (!pool_tensor_map(&tmK, k_pool, cache_dtype, head_dim, num_kv_heads, slots) ||
         !pool_tensor_map(&tmV, v_pool, cache_dtype, head_dim, num_kv_heads, slots))
         return PKV_ECUDA;
-    cudaError_t e;
-    if (prefill_kernel_choice() == 1) {
-        e = launch_prefill(tmK, tmV, p, max_query_len, static_cast<cudaStream_t>(stream));
-    } else {
-        // q viewed as [total_q][heads][head_dim]; boxes of 128 rows x 1 head x 128 bytes
-        CUtensorMap tmQ;
-        if (!rows_tensor_map(&tmQ, q, head_dim, num_heads, total_query_tokens, 128)) return PKV_ECUDA;
-        e = launch_prefill_tc(tmQ, tmK, tmV, p, fp8, max_query_len, static_cast<cudaStream_t>(stream));
-    }
+    // q viewed as [total_q][heads][head_dim]; boxes of 128 rows x 1 head x 128 bytes
+    CUtensorMap tmQ;
+    if (!rows_tensor_map(&tmQ, q, head_dim, num_heads, total_query_tokens, 128)) return PKV_ECUDA;
+    const cudaError_t e = launch_prefill_tc(tmQ, tmK, tmV, p, fp8, max_query_len, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PKV_OK : PKV_ECUDA;
 }
 

@@ -22,10 +22,6 @@ constexpr int kPlanThreads = 1024;
 constexpr int kMaxBuckets = 1024;
 constexpr int kMaxCandidates = 12;
 
-// Automatic partitioning ends each context with geometrically shrinking pieces.
-#ifndef PKV_PLAN_GEOMETRIC
-#define PKV_PLAN_GEOMETRIC 1
-#endif
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
@@ -182,7 +178,8 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
     __shared__ int chosen;
     __shared__ int n_subs, n_members;
     const int tid = threadIdx.x;
-    const bool geometric = fixed_partition == 0 && PKV_PLAN_GEOMETRIC;
+    // automatic partitioning ends each context with geometrically shrinking pieces
+    const bool geometric = fixed_partition == 0;
     const int mb = min_partition / kBlockSize;
 
     // The workspace and the output may still be in use by the previous kernel.

@@ -33,20 +33,6 @@
 
 namespace pkv {
 
-// FP8 scores: 1 = E4M3 tensor-core MMA on the stored codes with q split into
-// E4M3 hi + lo parts; 0 = codes converted to f16 and an f16 MMA.
-#ifndef PKV_FP8_QK_E4M3
-#define PKV_FP8_QK_E4M3 0
-#endif
-#if PKV_DEBUG_TIMELINE
-// Per-warp timeline for experiments: start, end (ns), units, merges, merge ns, blocks.
-__device__ unsigned long long g_timeline[4096][7];
-__device__ __forceinline__ unsigned long long now_ns() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    return t;
-}
-#endif
 
 template <bool FP8, int D>
 struct TileCfg {
@@ -73,9 +59,6 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
-#if PKV_DEBUG_TIMELINE
-    const unsigned long long dbg_entry = now_ns();
-#endif
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
     const uint32_t ring = base + warp * STAGES * C::kStageBytes;
     const uint32_t bar0 = smem_u32(&bars[warp][0]);  // K barrier of stage st at bar0 + 8*st, V at + 8*(STAGES+st)
@@ -119,10 +102,6 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
     const int num_units = p.hdr->num_units;
     const int G = p.group;
     uint32_t seqno = 0;  // blocks this warp has consumed so far (stage = seqno % STAGES)
-#if PKV_DEBUG_TIMELINE
-    const unsigned long long dbg_t0 = now_ns();
-    unsigned long long dbg_units = 0, dbg_merges = 0, dbg_merge_ns = 0;
-#endif
 
     for (;;) {
         int u = 0;
@@ -183,8 +162,16 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
         int chunk_cur = 0;
         unsigned long long okmask = 0;  // bit (j & 63): block j's id was in range
 
-        // Q^T fragments (B operand): n = query head of the group, k = head_dim.
+        // Q^T fragments (B operand): n = query head of the group, k = head_dim,
+        // and the score scale of this thread's two score columns (heads 2t, 2t+1).
+        // FP8 cache: the products run in f16, where every E4M3 code is exact, but
+        // f16 does not span bf16's range.  So each head's q is first multiplied
+        // by a power of two 2^e that brings its largest magnitude into
+        // [2^14, 2^15): exact, no entry can overflow, and every entry down to
+        // 2^-28 of that maximum keeps all of its bf16 bits in f16.  The head's
+        // score column then takes 2^-e along with the score scale.
         uint32_t qf[NT][KS][2];
+        float cs[NT][2];
         const int hq0 = kvh * G;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -199,69 +186,47 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
             }
             const __nv_bfloat16* qrow =
                 static_cast<const __nv_bfloat16*>(p.q) + ((size_t)sq * p.num_heads + hq0 + (hv ? hh : 0)) * D;
+            if constexpr (!FP8) {
 #pragma unroll
-            for (int ks = 0; ks < KS; ++ks) {
-                if constexpr (!FP8) {
+                for (int ks = 0; ks < KS; ++ks) {
                     const int d0 = ks * 16 + 2 * t;
                     qf[nt][ks][0] = hv ? *reinterpret_cast<const uint32_t*>(qrow + d0) : 0u;
                     qf[nt][ks][1] = hv ? *reinterpret_cast<const uint32_t*>(qrow + d0 + 8) : 0u;
-                } else {
-                    // k positions {2t, 2t+1, 2t+8, 2t+9} of step ks hold head_dim 16ks+4t+{0,1,2,3}
-                    const int d0 = ks * 16 + 4 * t;
-                    uint2 w = hv ? *reinterpret_cast<const uint2*>(qrow + d0) : make_uint2(0u, 0u);
-                    qf[nt][ks][0] = pack_f16x2(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u));
-                    qf[nt][ks][1] = pack_f16x2(__uint_as_float(w.y << 16), __uint_as_float(w.y & 0xFFFF0000u));
                 }
+                cs[nt][0] = cs[nt][1] = p.score_scale;
+            } else {
+                // k positions {2t, 2t+1, 2t+8, 2t+9} of step ks hold head_dim 16ks+4t+{0,1,2,3};
+                // the four lanes t = 0..3 of group g hold the whole row of head g
+                uint2 w[KS];
+                uint32_t amax_bits = 0;
+#pragma unroll
+                for (int ks = 0; ks < KS; ++ks) {
+                    w[ks] = hv ? *reinterpret_cast<const uint2*>(qrow + ks * 16 + 4 * t) : make_uint2(0u, 0u);
+                    // |x| of a bf16 orders like its bits with the sign cleared
+                    amax_bits = max(amax_bits, max(max(w[ks].x & 0x7FFFu, (w[ks].x >> 16) & 0x7FFFu),
+                                                   max(w[ks].y & 0x7FFFu, (w[ks].y >> 16) & 0x7FFFu)));
+                }
+                amax_bits = max(amax_bits, __shfl_xor_sync(0xffffffffu, amax_bits, 1));
+                amax_bits = max(amax_bits, __shfl_xor_sync(0xffffffffu, amax_bits, 2));
+                // e = 14 - floor(log2 max|q|), kept in [-126, 126] so that 2^e and
+                // 2^-e are normal floats (a bf16 subnormal maximum then still lands
+                // at or above 2^-7); an all-zero head keeps e = 0
+                const int ex = amax_bits != 0 ? (int)(amax_bits >> 7) - 127 : 14;
+                const int e = min(max(14 - ex, -126), 126);
+                const float up = __uint_as_float((uint32_t)(127 + e) << 23);
+                const float down = __uint_as_float((uint32_t)(127 - e) << 23) * p.score_scale;
+#pragma unroll
+                for (int ks = 0; ks < KS; ++ks) {
+                    qf[nt][ks][0] = pack_f16x2(__uint_as_float(w[ks].x << 16) * up,
+                                               __uint_as_float(w[ks].x & 0xFFFF0000u) * up);
+                    qf[nt][ks][1] = pack_f16x2(__uint_as_float(w[ks].y << 16) * up,
+                                               __uint_as_float(w[ks].y & 0xFFFF0000u) * up);
+                }
+                // score column c is head c of this n-tile, held by lanes 4c .. 4c+3
+                cs[nt][0] = __shfl_sync(0xffffffffu, down, 8 * t);
+                cs[nt][1] = __shfl_sync(0xffffffffu, down, 8 * t + 4);
             }
         }
-
-#if PKV_FP8_QK_E4M3
-        // FP8 scores on the FP8 tensor path: q of head g scaled by a power of two
-        // s_g (max |q| s_g in [128, 256)) and split into E4M3 hi + lo words in
-        // the m16n8k32 B layout (k = head_dim 32kk + 4t..4t+3 and +16); the
-        // score columns are divided by s back in the softmax.
-        uint32_t qhi[NT][D / 32][2], qlo[NT][D / 32][2];
-        float col_scale[NT][2];
-        if constexpr (FP8) {
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const int hh = nt * 8 + g;
-                const bool hv = hh < G;
-                const __nv_bfloat16* qrow =
-                    static_cast<const __nv_bfloat16*>(p.q) + ((size_t)s * p.num_heads + hq0 + (hv ? hh : 0)) * D;
-                float x[D / 32][2][4];
-                float amax = 0.f;
-#pragma unroll
-                for (int kk = 0; kk < D / 32; ++kk)
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const uint2 w = hv ? *reinterpret_cast<const uint2*>(qrow + 32 * kk + 16 * h + 4 * t)
-                                           : make_uint2(0u, 0u);
-                        x[kk][h][0] = __uint_as_float(w.x << 16);
-                        x[kk][h][1] = __uint_as_float(w.x & 0xFFFF0000u);
-                        x[kk][h][2] = __uint_as_float(w.y << 16);
-                        x[kk][h][3] = __uint_as_float(w.y & 0xFFFF0000u);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(x[kk][h][e]));
-                    }
-                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-                // s = 2^(7 - floor(log2 amax)); 1 for an all-zero (or padding) head
-                const int ex = amax > 0.f ? (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127 : 7;
-                const float sq = __uint_as_float((uint32_t)(127 + 7 - ex) << 23);
-#pragma unroll
-                for (int kk = 0; kk < D / 32; ++kk)
-#pragma unroll
-                    for (int h = 0; h < 2; ++h)
-                        split_e4m3x4(x[kk][h][0] * sq, x[kk][h][1] * sq, x[kk][h][2] * sq, x[kk][h][3] * sq,
-                                     qhi[nt][kk][h], qlo[nt][kk][h]);
-                // this thread's score columns are heads 2t and 2t+1 (held by lanes 8t and 8t+4)
-                const float inv = 1.f / sq;
-                col_scale[nt][0] = __shfl_sync(0xffffffffu, inv, 8 * t);
-                col_scale[nt][1] = __shfl_sync(0xffffffffu, inv, 8 * t + 4);
-            }
-        }
-#endif
 
         // Issue the TMA loads of block j of this unit into its stage (all lanes
         // call it: the block id is broadcast with a shuffle).
@@ -326,26 +291,6 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
                             mma_bf16((ks & 1) ? sc2[nt] : sc[nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
                 }
             } else {
-#if PKV_FP8_QK_E4M3
-                // ldmatrix of 16 rows x 32 codes is exactly the m16n8k32 A fragment
-#pragma unroll
-                for (int kk = 0; kk < D / 32; ++kk) {
-                    uint32_t r0, r1, r2, r3;
-                    ldmatrix_x4(kt + koff[kk], r0, r1, r2, r3);
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        mma_e4m3(sc[nt], r0, r1, r2, r3, qhi[nt][kk][0], qhi[nt][kk][1]);
-                        mma_e4m3(sc2[nt], r0, r1, r2, r3, qlo[nt][kk][0], qlo[nt][kk][1]);
-                    }
-                }
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        sc[nt][e] *= col_scale[nt][e & 1];
-                        sc2[nt][e] *= col_scale[nt][e & 1];
-                    }
-#else
 #pragma unroll
                 for (int kp = 0; kp < KS / 2; ++kp) {
                     uint32_t r0, r1, r2, r3;
@@ -359,7 +304,6 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
                                 e4m3x2_to_f16x2(r3 >> 16), qf[nt][2 * kp + 1][0], qf[nt][2 * kp + 1][1]);
                     }
                 }
-#endif
             }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
@@ -461,10 +405,10 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
 #pragma unroll
                     for (int b = 0; b < BPS; ++b) {
                         const bool vlo = okb[b] && g < nvalid[b], vhi = okb[b] && g + 8 < nvalid[b];
-                        x[b][0] = vlo ? sc[b][nt][0] * p.score_scale : -INFINITY;
-                        x[b][1] = vlo ? sc[b][nt][1] * p.score_scale : -INFINITY;
-                        x[b][2] = vhi ? sc[b][nt][2] * p.score_scale : -INFINITY;
-                        x[b][3] = vhi ? sc[b][nt][3] * p.score_scale : -INFINITY;
+                        x[b][0] = vlo ? sc[b][nt][0] * cs[nt][0] : -INFINITY;
+                        x[b][1] = vlo ? sc[b][nt][1] * cs[nt][1] : -INFINITY;
+                        x[b][2] = vhi ? sc[b][nt][2] * cs[nt][0] : -INFINITY;
+                        x[b][3] = vhi ? sc[b][nt][3] * cs[nt][1] : -INFINITY;
                         b0 = fmaxf(b0, fmaxf(x[b][0], x[b][2]));
                         b1 = fmaxf(b1, fmaxf(x[b][1], x[b][3]));
                     }
@@ -629,24 +573,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
                 }
             }
         }  // pass
-#if PKV_DEBUG_TIMELINE
-        ++dbg_units;
-#endif
     }
-#if PKV_DEBUG_TIMELINE
-    if (lane == 0) {
-        const int w = blockIdx.x * WARPS + warp;
-        if (w < 4096) {
-            g_timeline[w][0] = dbg_t0;
-            g_timeline[w][1] = now_ns();
-            g_timeline[w][2] = dbg_units;
-            g_timeline[w][3] = dbg_merges;
-            g_timeline[w][4] = dbg_merge_ns;
-            g_timeline[w][5] = seqno;
-            g_timeline[w][6] = dbg_entry;
-        }
-    }
-#endif
 }
 
 template <bool FP8, int D, int NT, int WARPS, int STAGES, int BPS, bool GROUPED = false>
@@ -660,53 +587,21 @@ static cudaError_t launch_tc(const CUtensorMap& tmK, const CUtensorMap& tmV, con
     return launch_pdl(kern, dim3(num_sms), dim3(WARPS * 32), smem, stream, tmK, tmV, p);
 }
 
-#if PKV_DEBUG_TIMELINE
-extern "C" int pkv_debug_timeline(void* host, int rows) {
-    return cudaMemcpyFromSymbol(host, g_timeline, sizeof(unsigned long long) * 7 * rows) == cudaSuccess ? 0 : 3;
-}
-#endif
-
-// Warps per CTA (one CTA per SM) and ring depth per warp, per cache type.
-// Shared memory per CTA = warps * stages * 2 tiles (+1 KB alignment slack).
-#ifndef PKV_TC_WARPS_BF16
-#define PKV_TC_WARPS_BF16 12
-#endif
-#ifndef PKV_TC_STAGES_BF16
-#define PKV_TC_STAGES_BF16 2
-#endif
-#ifndef PKV_TC_WARPS_BF16_D64
-#define PKV_TC_WARPS_BF16_D64 8
-#endif
-#ifndef PKV_TC_STAGES_BF16_D64
-#define PKV_TC_STAGES_BF16_D64 6
-#endif
-#ifndef PKV_TC_WARPS_FP8
-#define PKV_TC_WARPS_FP8 16
-#endif
-#ifndef PKV_TC_STAGES_FP8
-#define PKV_TC_STAGES_FP8 3
-#endif
-// Blocks per step of the main loop (one softmax reduction per step).
-#ifndef PKV_TC_BPS_BF16
-#define PKV_TC_BPS_BF16 1
-#endif
-#ifndef PKV_TC_BPS_FP8
-#define PKV_TC_BPS_FP8 2
-#endif
-
-
-// The shared-prefix variant (bf16, head_dim 128) holds 16 score columns.
-#ifndef PKV_TC_WARPS_GROUPED
-#define PKV_TC_WARPS_GROUPED 12
-#endif
-#ifndef PKV_TC_STAGES_GROUPED
-#define PKV_TC_STAGES_GROUPED 2
-#endif
+// Launch shapes, chosen by measurement on B200: warps per CTA (one CTA per SM),
+// ring stages per warp and blocks per main-loop step (one softmax reduction per
+// step).  Shared memory per CTA = warps * stages * 2 tiles (+1 KB alignment slack).
+struct Shape {
+    int warps, stages, bps;
+};
+constexpr Shape kBf16D128{12, 2, 1};
+constexpr Shape kBf16D64{8, 6, 1};
+constexpr Shape kFp8{16, 3, 2};
+constexpr Shape kGrouped{12, 2, 1};  // shared-prefix variant (bf16, head_dim 128, 16 score columns)
 
 int decode_tc_warps(bool fp8, int head_dim, bool grouped) {
-    if (grouped) return PKV_TC_WARPS_GROUPED;
-    if (fp8) return PKV_TC_WARPS_FP8;
-    return head_dim == 128 ? PKV_TC_WARPS_BF16 : PKV_TC_WARPS_BF16_D64;
+    if (grouped) return kGrouped.warps;
+    if (fp8) return kFp8.warps;
+    return head_dim == 128 ? kBf16D128.warps : kBf16D64.warps;
 }
 
 bool decode_tc_groupable(bool fp8, int head_dim, int group) { return !fp8 && head_dim == 128 && group <= 8; }
@@ -716,21 +611,21 @@ cudaError_t launch_decode_tc(const CUtensorMap& tmK, const CUtensorMap& tmV, con
     const int nt = (p.group + 7) / 8;
     if (p.num_groups > 0) {
         if (!decode_tc_groupable(fp8, p.head_dim, p.group)) return cudaErrorInvalidValue;
-        return launch_tc<false, 128, 2, PKV_TC_WARPS_GROUPED, PKV_TC_STAGES_GROUPED, PKV_TC_BPS_BF16, true>(
+        return launch_tc<false, 128, 2, kGrouped.warps, kGrouped.stages, kGrouped.bps, true>(
             tmK, tmV, p, num_sms, stream);
     }
     if (fp8) {
         if (p.head_dim != 128) return cudaErrorInvalidValue;
-        return nt == 1 ? launch_tc<true, 128, 1, PKV_TC_WARPS_FP8, PKV_TC_STAGES_FP8, PKV_TC_BPS_FP8>(tmK, tmV, p, num_sms, stream)
-                       : launch_tc<true, 128, 2, PKV_TC_WARPS_FP8, PKV_TC_STAGES_FP8, PKV_TC_BPS_FP8>(tmK, tmV, p, num_sms, stream);
+        return nt == 1 ? launch_tc<true, 128, 1, kFp8.warps, kFp8.stages, kFp8.bps>(tmK, tmV, p, num_sms, stream)
+                       : launch_tc<true, 128, 2, kFp8.warps, kFp8.stages, kFp8.bps>(tmK, tmV, p, num_sms, stream);
     }
     if (p.head_dim == 128)
         return nt == 1
-                   ? launch_tc<false, 128, 1, PKV_TC_WARPS_BF16, PKV_TC_STAGES_BF16, PKV_TC_BPS_BF16>(tmK, tmV, p, num_sms, stream)
-                   : launch_tc<false, 128, 2, PKV_TC_WARPS_BF16, PKV_TC_STAGES_BF16, PKV_TC_BPS_BF16>(tmK, tmV, p, num_sms, stream);
+                   ? launch_tc<false, 128, 1, kBf16D128.warps, kBf16D128.stages, kBf16D128.bps>(tmK, tmV, p, num_sms, stream)
+                   : launch_tc<false, 128, 2, kBf16D128.warps, kBf16D128.stages, kBf16D128.bps>(tmK, tmV, p, num_sms, stream);
     return nt == 1
-               ? launch_tc<false, 64, 1, PKV_TC_WARPS_BF16_D64, PKV_TC_STAGES_BF16_D64, PKV_TC_BPS_BF16>(tmK, tmV, p, num_sms, stream)
-               : launch_tc<false, 64, 2, PKV_TC_WARPS_BF16_D64, PKV_TC_STAGES_BF16_D64, PKV_TC_BPS_BF16>(tmK, tmV, p, num_sms, stream);
+               ? launch_tc<false, 64, 1, kBf16D64.warps, kBf16D64.stages, kBf16D64.bps>(tmK, tmV, p, num_sms, stream)
+               : launch_tc<false, 64, 2, kBf16D64.warps, kBf16D64.stages, kBf16D64.bps>(tmK, tmV, p, num_sms, stream);
 }
 
 }  // namespace pkv

@@ -306,32 +306,6 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1,
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// D(16x8, f32) += A(16x32, e4m3, row) * B(32x8, e4m3, col); products are exact
-// in fp32 (3-bit mantissas).
-__device__ __forceinline__ void mma_e4m3(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-    asm("mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 "
-        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// Four floats (already scaled into E4M3 range) as an E4M3 "hi" word and the
-// E4M3 word of their residuals ("lo"): x ~= value(hi) + value(lo), relative
-// error about 2^-8 for |x| >= 2^-2 (round to nearest even, saturating).
-__device__ __forceinline__ void split_e4m3x4(float x0, float x1, float x2, float x3, uint32_t& hi, uint32_t& lo) {
-    const uint32_t h01 = __nv_cvt_float2_to_fp8x2(make_float2(x0, x1), __NV_SATFINITE, __NV_E4M3);
-    const uint32_t h23 = __nv_cvt_float2_to_fp8x2(make_float2(x2, x3), __NV_SATFINITE, __NV_E4M3);
-    const __half2_raw b01 = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(h01), __NV_E4M3);
-    const __half2_raw b23 = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(h23), __NV_E4M3);
-    const float r0 = x0 - __half2float(__ushort_as_half(b01.x)), r1 = x1 - __half2float(__ushort_as_half(b01.y));
-    const float r2 = x2 - __half2float(__ushort_as_half(b23.x)), r3 = x3 - __half2float(__ushort_as_half(b23.y));
-    const uint32_t l01 = __nv_cvt_float2_to_fp8x2(make_float2(r0, r1), __NV_SATFINITE, __NV_E4M3);
-    const uint32_t l23 = __nv_cvt_float2_to_fp8x2(make_float2(r2, r3), __NV_SATFINITE, __NV_E4M3);
-    hi = (h01 & 0xFFFFu) | (h23 << 16);
-    lo = (l01 & 0xFFFFu) | (l23 << 16);
-}
-
 // Two E4M3 codes (low byte -> low half) to two f16 values; exact (every E4M3
 // value is representable in f16).
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {

@@ -1,5 +1,5 @@
-// prefill_tc.cu -- causal multi-token paged attention on the 5th-generation
-// tensor cores (tcgen05): same result as prefill.cu's kernel.
+// prefill_tc.cu -- causal multi-token paged attention (the prompt pass) on the
+// 5th-generation tensor cores (tcgen05).
 //
 // What it computes: sequence s has nq new query tokens, the last nq of its
 // context_len tokens (K/V already in the pool); query i at position
@@ -105,12 +105,15 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4 v) {
                  : "memory");
 }
 
-// two bf16 (one word) -> two f16, saturating at +-65504 (exact inside the f16 normal range)
-__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
-    uint32_t r;
-    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(__uint_as_float(w & 0xFFFF0000u)),
-        "f"(__uint_as_float(w << 16)));
-    return r;
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
+// two bf16 (one word) times a power of two `up` -> two f16 (round to nearest)
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_scaled(uint32_t w, float up) {
+    return pack_f16x2(__uint_as_float(w << 16) * up, __uint_as_float(w & 0xFFFF0000u) * up);
 }
 
 // A and B from shared memory.
@@ -550,22 +553,43 @@ __global__ void __launch_bounds__(FP8 ? 448 : 320, 1)
         float m_ref = -INFINITY, l = 0.f;
         bool alive = true;
         const int nt = ntq[t];
+        float row_scale = p.score_scale;  // this row's scores -> base-2 units
         if constexpr (FP8) {
-            // the products run in f16 (an E4M3 code is exact there): this warpgroup turns
-            // its Q tile from bf16 into f16 in place
+            // The products run in f16 (an E4M3 code is exact there), and f16 does not
+            // span bf16's range: each thread turns its own query row of the Q tile
+            // into f16 in place after multiplying it by a power of two 2^e that puts
+            // the row's largest magnitude in [2^14, 2^15) (exact; entries down to
+            // 2^-28 of it keep all their bf16 bits), and takes 2^-e into its score
+            // scale.  Row r of the tile is 128 bytes in each 64-column half, its
+            // 16-byte chunks permuted by (r & 7): 8 consecutive rows touch 8
+            // distinct bank groups.
             const bool landed = mbar_wait_bounded(q_full, 0);
             if (__all_sync(0xffffffffu, landed)) {
                 const uint32_t qt = base + kTcQ + t * kTcQBytes;
-                for (int w = r; w < kTcQBytes / 16; w += kTcRows) {
-                    uint4 v;
-                    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                                 : "r"(qt + 16 * w));
-                    v.x = bf16x2_to_f16x2(v.x);
-                    v.y = bf16x2_to_f16x2(v.y);
-                    v.z = bf16x2_to_f16x2(v.z);
-                    v.w = bf16x2_to_f16x2(v.w);
-                    st_shared_v4(qt + 16 * w, v);
+                auto chunk_addr = [&](int c) {  // c = 0..15: half c / 8, chunk c % 8 of row r
+                    return qt + (c >> 3) * (kTcRows * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+                };
+                uint32_t amax_bits = 0;
+#pragma unroll 4
+                for (int c = 0; c < 16; ++c) {
+                    const uint4 v = ld_shared_v4(chunk_addr(c));
+                    const uint32_t m01 = max(max(v.x & 0x7FFFu, (v.x >> 16) & 0x7FFFu), max(v.y & 0x7FFFu, (v.y >> 16) & 0x7FFFu));
+                    const uint32_t m23 = max(max(v.z & 0x7FFFu, (v.z >> 16) & 0x7FFFu), max(v.w & 0x7FFFu, (v.w >> 16) & 0x7FFFu));
+                    amax_bits = max(amax_bits, max(m01, m23));
+                }
+                // e = 14 - floor(log2 max|q|) within [-126, 126]; an all-zero row keeps e = 0
+                const int ex = amax_bits != 0 ? (int)(amax_bits >> 7) - 127 : 14;
+                const int e = min(max(14 - ex, -126), 126);
+                const float up = __uint_as_float((uint32_t)(127 + e) << 23);
+                row_scale = __uint_as_float((uint32_t)(127 - e) << 23) * p.score_scale;
+#pragma unroll 4
+                for (int c = 0; c < 16; ++c) {
+                    uint4 v = ld_shared_v4(chunk_addr(c));
+                    v.x = bf16x2_to_f16x2_scaled(v.x, up);
+                    v.y = bf16x2_to_f16x2_scaled(v.y, up);
+                    v.z = bf16x2_to_f16x2_scaled(v.z, up);
+                    v.w = bf16x2_to_f16x2_scaled(v.w, up);
+                    st_shared_v4(chunk_addr(c), v);
                 }
                 fence_proxy_async_smem();  // read by the tensor core
                 __syncwarp();
@@ -624,12 +648,12 @@ __global__ void __launch_bounds__(FP8 ? 448 : 320, 1)
             const int k0 = j * kTcKeys;
             if (k0 + kTcKeys - 1 <= qpos && okmask == (1u << kTcBlocks) - 1u) {
 #pragma unroll
-                for (int c = 0; c < kTcKeys; ++c) x[c] *= p.score_scale;
+                for (int c = 0; c < kTcKeys; ++c) x[c] *= row_scale;
             } else {
 #pragma unroll
                 for (int c = 0; c < kTcKeys; ++c) {
                     const bool valid = k0 + c <= qpos && ((okmask >> (c >> 4)) & 1u);
-                    x[c] = valid ? x[c] * p.score_scale : -INFINITY;
+                    x[c] = valid ? x[c] * row_scale : -INFINITY;
                 }
             }
             // max as 8 independent chains, then a tree (short dependency chains)

@@ -1,8 +1,8 @@
 """GPU parity of paged_attention_decode (+ the step's KV write) against the oracle.
 
-Small cases are compared on every output element; the full-size workloads on
-sampled sequences (the oracle computes those one by one), in the launch
-configuration the benchmark uses (automatic partitioning).
+Small cases and the full-size workloads are compared on every output element,
+the full-size ones in the launch configuration the benchmark uses (automatic
+partitioning).
 """
 import numpy as np
 import pytest
@@ -119,7 +119,7 @@ def test_fp8_group_sizes(G):
     _run(DecodeCase(w, lens=np.array([1, 17, 250, 1000], np.int32)), 0)
 
 
-# ------------------------------------------------------------------ full-size workloads (sampled)
+# ------------------------------------------------------------------ full-size workloads (every element)
 
 def test_full_mha13b_every_element():
     w = W.WORKLOADS["mha13b"]
@@ -127,21 +127,57 @@ def test_full_mha13b_every_element():
     _run(case, 0)
 
 
-def test_full_gqa70b_sampled():
-    w = W.WORKLOADS["gqa70b"]
-    rng = np.random.default_rng(7)
-    case = DecodeCase(w, sample=np.sort(rng.choice(w.num_seqs, 10, replace=False)))
-    _run(case, 0)
+def test_full_gqa70b_every_element():
+    """The benchmark's headline batch (256 x 4,096 tokens, 64/8 heads, 4 GiB of
+    K/V) in its launch configuration, every output element against the oracle."""
+    _run(DecodeCase(W.WORKLOADS["gqa70b"]), 0)
 
 
-def test_full_fp8_long_sampled():
-    w = W.WORKLOADS["fp8_long"]
-    lens = W.context_lens(w)
-    pick = {int(np.argmax(lens)), int(np.argmin(lens))}
-    rng = np.random.default_rng(8)
-    pick |= set(int(x) for x in rng.choice(w.num_seqs, 8, replace=False))
-    case = DecodeCase(w, sample=np.array(sorted(pick)))
-    _run(case, 0)
+def test_full_fp8_long_every_element():
+    """All 128 sequences of the FP8 workload (contexts 256..32,768, split
+    partitions and their merge), every output element against the oracle."""
+    _run(DecodeCase(W.WORKLOADS["fp8_long"]), 0)
+
+
+# ------------------------------------------------------------------ FP8 cache: q of any finite bf16 magnitude
+
+# Powers of two per query head (exact in bf16): far above and far below 1.
+HEAD_EXP = (17, -20, 8, 0, -8, 12, 3, -14)
+
+
+def scale_q_magnitudes(q, mode):
+    """q (bf16, [..., heads, head_dim]) rescaled by powers of two; returns the new
+    tensor and the factor for k_scale that keeps scores in a useful range.
+      big:   every entry x 2^12, and one entry of head 1 set to 70,000 (past f16's 65,504)
+      tiny:  every entry x 2^-20, the K cache x 2^20 (scores unchanged, q below f16's normal range)
+      mixed: head h x 2^HEAD_EXP[h % 8], one entry of head 0 set to -70,000"""
+    x = q.float()
+    H = x.shape[-2]
+    if mode == "big":
+        x = x * 2.0 ** 12
+        x[..., 1 % H, 5] = 70000.0
+        return x.to(torch.bfloat16), 1.0
+    if mode == "tiny":
+        return (x * 2.0 ** -20).to(torch.bfloat16), 2.0 ** 20
+    f = torch.tensor([2.0 ** HEAD_EXP[h % 8] for h in range(H)], device=x.device)
+    x = x * f[:, None]
+    x[..., 0, 7] = -70000.0
+    return x.to(torch.bfloat16), 1.0
+
+
+@pytest.mark.parametrize("mode", ["big", "tiny", "mixed"])
+@pytest.mark.parametrize("G", [4, 8, 16])
+def test_fp8_q_beyond_f16_range(mode, G):
+    """The FP8 decode multiplies in f16; q is bf16, whose range f16 does not
+    span.  Every finite bf16 q must still give the oracle's result: entries past
+    65,504, entries below f16's normal range, and heads of very different
+    magnitudes in one group (each head's scaling lands on its own score column)."""
+    w = W.scaled(W.WORKLOADS["fp8_long"], num_heads=2 * G, num_kv_heads=2, num_seqs=4)
+    for P in (0, 64):
+        case = DecodeCase(w, lens=np.array([1, 17, 250, 1000], np.int32))
+        case.q, kf = scale_q_magnitudes(case.q, mode)
+        case.k_scale *= kf
+        _run(case, P)
 
 
 # ------------------------------------------------------------------ edge cases

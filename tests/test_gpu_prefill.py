@@ -109,6 +109,23 @@ def test_fp8_cache_ragged_prompts_every_element(Hq, Hkv):
     assert_close(got, ref, "fp8", "fp8 prefill G=%d" % (Hq // Hkv))
 
 
+@pytest.mark.parametrize("mode", ["big", "tiny", "mixed"])
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (64, 8)])
+def test_fp8_cache_q_beyond_f16_range(mode, Hq, Hkv):
+    """The FP8-cache prompt pass multiplies in f16; every finite bf16 q must
+    still give the oracle's result (entries past 65,504, entries below f16's
+    normal range, heads of very different magnitudes)."""
+    from tests.test_gpu_decode import scale_q_magnitudes
+    c = PrefillCase(Hq, Hkv, *RAGGED, seed=60 + Hq, cache="fp8")
+    q, kf = scale_q_magnitudes(c.q, mode)
+    c.q = q
+    c.k_scale *= kf
+    got = out_to_f64(c.run())
+    ref, bad = c.oracle()
+    assert bad == 0 and int(c.err.item()) == 0
+    assert_close(got, ref, "fp8", "fp8 prefill q %s G=%d" % (mode, Hq // Hkv))
+
+
 def test_fp8_cache_long_prompts_sampled_rows():
     """FP8 cache, prompts of 1,000..3,000 tokens (many KV tiles, both staging
     slots reused), 32/8 heads; rows sampled, first and last of every prompt."""
@@ -206,29 +223,6 @@ def test_context_past_the_shared_memory_validity_bits(cache):
     ref, bad = c.oracle(tables=tabs)
     assert bad == 1 and int(c.err.item()) == 1
     assert_close(got, ref, cache, "33k context %s" % cache)
-
-
-def test_warp_mma_kernel_agrees(tmp_path):
-    """The mma.sync prefill kernel (PKV_PREFILL_KERNEL=mma, a separate process)
-    gives the oracle's result on the ragged case too."""
-    import os
-    import subprocess
-    import sys
-    code = (
-        "import numpy as np, sys; sys.path.insert(0, %r)\n"
-        "from tests.test_gpu_prefill import PrefillCase, RAGGED\n"
-        "from tests.helpers import assert_close, out_to_f64\n"
-        "c = PrefillCase(16, 4, *RAGGED, seed=44)\n"
-        "got = out_to_f64(c.run()); ref, bad = c.oracle()\n"
-        "assert bad == 0 and int(c.err.item()) == 0\n"
-        "assert_close(got, ref, 'bf16', 'mma.sync prefill')\n"
-        "import pytest, paged_kv_cache_404_b200 as pkv\n"
-        "f = PrefillCase(8, 8, [40], [40], seed=46, cache='fp8')\n"
-        "with pytest.raises(pkv.PagedKVError): f.run()\n"
-        "print('ok')\n" % os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
-    env = dict(os.environ, PKV_PREFILL_KERNEL="mma")
-    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=600)
-    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout[-2000:] + r.stderr[-2000:]
 
 
 def test_sequences_without_queries_and_oversized_launch():
