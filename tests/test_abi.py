@@ -89,6 +89,34 @@ def test_decode_validation(L):
     assert _decode(L, mb=0) == L.PKV_EINVAL
 
 
+def _noalloc(L, **kw):
+    a = dict(out=FAKE, q=FAKE, qdt=L.PKV_BF16, kp=FAKE, vp=FAKE, cdt=L.PKV_BF16, bt=FAKE, mb=256, cl=FAKE, S=256,
+             maxlen=4096, nb=1024, bs=16, hq=64, hkv=8, d=128, P=0, err=None)
+    a.update(kw)
+    return L.lib().pkv_paged_attention_decode_noalloc(
+        a["out"], a["q"], a["qdt"], a["kp"], a["vp"], a["cdt"], a["bt"], a["mb"], a["cl"], a["S"], a["maxlen"],
+        a["nb"], a["bs"], a["hq"], a["hkv"], a["d"], 0.088, 1.0, 1.0, a["P"], a["err"], None)
+
+
+def test_noalloc_validation_order(L):
+    """The no-alloc decode runs the decode's own checks before its scratch limit,
+    so an unsupported configuration reports PKV_EUNSUPPORTED whatever its size;
+    only a supported one that needs more than the fixed scratch gets PKV_EINVAL.
+    Every case here returns before any CUDA call."""
+    f = L.lib().pkv_decode_workspace_bytes
+    assert f(256, 64, 128, 4096, 0) > (32 << 20)           # the default case is over the limit
+    assert _noalloc(L) == L.PKV_EINVAL
+    assert _noalloc(L, S=0) == L.PKV_OK                     # nothing to do
+    assert _noalloc(L, d=256) == L.PKV_EUNSUPPORTED         # big and unsupported: the configuration decides
+    assert _noalloc(L, hq=256, hkv=8) == L.PKV_EUNSUPPORTED  # group 32 > 16 with a bf16 cache
+    assert _noalloc(L, cdt=L.PKV_FP8_E4M3, d=64) == L.PKV_EUNSUPPORTED
+    assert _noalloc(L, bs=8) == L.PKV_EUNSUPPORTED
+    assert _noalloc(L, hq=60) == L.PKV_EINVAL
+    assert _noalloc(L, P=24) == L.PKV_EINVAL
+    assert _noalloc(L, out=None) == L.PKV_EINVAL
+    assert _noalloc(L, q=ODD) == L.PKV_EINVAL
+
+
 def test_workspace_bytes(L):
     f = L.lib().pkv_decode_workspace_bytes
     a = f(256, 64, 128, 4096, 0)
