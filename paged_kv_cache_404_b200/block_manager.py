@@ -3,10 +3,12 @@
 The manager itself is C++ (csrc/block_manager.cpp); this class only marshals
 numpy arrays.  It runs on the CPU and needs no GPU.
 
-Optional event trace (JSON lines), for the record a paged cache is best kept
-with (iplexlaw.co.kr recommends logging when blocks are allocated, the tables,
-when blocks are shared, copied and freed, the sequence lengths and how many
-requests run at once): every allocation, fork, append, release and swap writes
+Optional event trace (JSON lines).  The iplexlaw.co.kr blog post on
+PagedAttention and the vLLM KV cache, section "Memory management and the
+technical differences", advises recording when blocks are allocated, the block
+tables, the conditions of sharing, copies and releases, sequence lengths and
+the number of concurrent requests; this trace keeps that record: every
+allocation, fork, append, release and swap writes
 one line with a monotonic timestamp (t_ns), the operation's inputs and results
 (tables, slots, copy-on-write pairs, blocks actually freed, swap pairs, tokens
 reused from the prefix cache), and the live-sequence and free-block counts after

@@ -301,6 +301,40 @@ def test_same_system_prompt_reuses_full_blocks():
     _check_invariants(bm)
 
 
+def test_two_requests_share_their_common_system_prompt_block():
+    """Worked by hand from the glossary entry's sharing section: requests that
+    start with the same system prompt reuse one copy of it, each block counted
+    by a reference counter, and hashing whole blocks is what carries the sharing
+    from one request to the next.  Free list as in the worked example:
+    [41, 7, 19, 2, 33], then 11 and 5 (no other block of the 64 is free).
+      A = S + U1 + 5 tokens   -> no hit, blocks [41, 7, 19]
+      B = S + U2 + 3 tokens   -> S hits 41 (16 tokens), U2 misses: [41, 2, 33]
+      D = U1 + S              -> no hit: U1 at the start is not A's second block
+                                 (its keys and values follow S there): [11, 5]
+      A freed                 -> 41 keeps B's reference; 7 (full, keyed) and 19
+                                 go to the back of the free list: [7, 19]
+      E = S + U1 + 1 token    -> hits 41 and 7 (taken back out of the free
+                                 list), 32 tokens; its tail gets 19: [41, 7, 19]"""
+    S, U1, U2 = list(range(100, 116)), list(range(200, 216)), list(range(300, 316))
+    bm = RefBlockManager(64, 16, free_order=[41, 7, 19, 2, 33, 11, 5])
+    bm.set_prefix_cache(True)
+    a, ca = bm.alloc_seq_tokens(S + U1 + [1] * 5)
+    assert (bm.tables[a], ca) == ([41, 7, 19], 0)
+    b, cb = bm.alloc_seq_tokens(S + U2 + [2] * 3)
+    assert (bm.tables[b], cb) == ([41, 2, 33], 16)
+    assert [bm.ref[x] for x in (41, 7, 19, 2, 33)] == [2, 1, 1, 1, 1]
+    d, cd = bm.alloc_seq_tokens(U1 + S)
+    assert (bm.tables[d], cd) == ([11, 5], 0)
+    assert bm.ref[7] == 1 and list(bm.free) == []
+    bm.free_seq(a)
+    assert list(bm.free) == [7, 19] and [bm.ref[x] for x in (41, 7, 19)] == [1, 0, 0]
+    e, ce = bm.alloc_seq_tokens(S + U1 + [3])
+    assert (bm.tables[e], ce) == ([41, 7, 19], 32)
+    assert [bm.ref[x] for x in (41, 7, 19, 2, 33, 11, 5)] == [2, 1, 1, 1, 1, 1, 1]
+    assert list(bm.free) == []
+    _check_invariants(bm)
+
+
 def test_a_block_is_keyed_by_its_whole_prefix():
     """The same 16 tokens after a different first block are a different block."""
     bm = _cached_bm()

@@ -496,3 +496,26 @@ def test_batched_append_stops_at_the_first_sequence_out_of_blocks(BM):
     assert [tuple(p) for p in pairs[:npairs.value].tolist()] == [e[1] for e in exp if e[1] is not None]
     _same_state(bm, ref, seqs)        # d unchanged on both sides
     assert bm.seq_len(seqs[3]) == 16
+
+
+def test_native_manager_on_the_hand_worked_system_prompt_case(BM):
+    """The hand-worked system-prompt sharing case of the reference manager's pins
+    (worked example's free list; two requests share their first block, a request
+    that starts with another's second block gets no hit, a freed keyed block is
+    taken back out of the free list), on the native manager."""
+    S, U1, U2 = list(range(100, 116)), list(range(200, 216)), list(range(300, 316))
+    bm = BM(64, 16, free_order=[41, 7, 19, 2, 33, 11, 5])
+    bm.set_prefix_cache(True)
+    a, ca = bm.alloc_seq_tokens(S + U1 + [1] * 5)
+    assert (bm.block_table(a).tolist(), ca) == ([41, 7, 19], 0)
+    b, cb = bm.alloc_seq_tokens(S + U2 + [2] * 3)
+    assert (bm.block_table(b).tolist(), cb) == ([41, 2, 33], 16)
+    assert [bm.refcount(x) for x in (41, 7, 19, 2, 33)] == [2, 1, 1, 1, 1]
+    d, cd = bm.alloc_seq_tokens(U1 + S)
+    assert (bm.block_table(d).tolist(), cd) == ([11, 5], 0)
+    bm.free_seq(a)
+    assert bm.free_list().tolist() == [7, 19]
+    e, ce = bm.alloc_seq_tokens(S + U1 + [3])
+    assert (bm.block_table(e).tolist(), ce) == ([41, 7, 19], 32)
+    assert [bm.refcount(x) for x in (41, 7, 19, 2, 33, 11, 5)] == [2, 1, 1, 1, 1, 1, 1]
+    assert bm.num_free() == 0

@@ -201,9 +201,12 @@ def test_pins_reject_swap_in_that_restores_old_block_ids(monkeypatch):
         A.test_swap_round_trip_restores_every_token()
 
 
-def test_pins_reject_prefix_cache_keyed_by_tokens_only(monkeypatch):
+@pytest.mark.parametrize("pin", ["test_a_block_is_keyed_by_its_whole_prefix",
+                                 "test_two_requests_share_their_common_system_prompt_block"])
+def test_pins_reject_prefix_cache_keyed_by_tokens_only(monkeypatch, pin):
     """Planted mistake: a full block is keyed by its own 16 tokens only, not by
-    its prefix, so the same tokens after a different start alias one block."""
+    its prefix, so the same tokens after a different start alias one block.
+    Both the synthetic pin and the hand-worked system-prompt case reject it."""
     from oracle import allocator
     real = allocator.RefBlockManager.alloc_seq_tokens
 
@@ -220,7 +223,7 @@ def test_pins_reject_prefix_cache_keyed_by_tokens_only(monkeypatch):
 
     monkeypatch.setattr(allocator.RefBlockManager, "alloc_seq_tokens", bad)
     with pytest.raises(AssertionError):
-        A.test_a_block_is_keyed_by_its_whole_prefix()
+        getattr(A, pin)()
 
 
 def test_pins_reject_prefix_cache_that_keeps_keys_of_reused_blocks(monkeypatch):
