@@ -325,8 +325,12 @@ class Step:
 
 
 def time_steps(step: Step, steps: int, warmup: int, world: int, device):
-    """K timed steps between a barrier + synchronize on both sides; the step and
-    the decode call inside it are timed with CUDA events on the launching stream."""
+    """K timed steps between a barrier + synchronize on both sides, timed with CUDA
+    events on the launching stream at the start and the end only (an event between
+    two kernels keeps the second from starting before the first has finished, so
+    per-step events would hide the overlap of a step's kernels).  A second pass
+    over the same steps records events around the write and the decode call of
+    each step, for their split and spread."""
     stream = torch.cuda.current_stream()
     for _ in range(warmup):
         step.run()
@@ -335,23 +339,26 @@ def time_steps(step: Step, steps: int, warmup: int, world: int, device):
         import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     start.record(stream)
-    for a, b, c in ev:
-        a.record(stream)
-        step.copy_and_write()
-        b.record(stream)
-        step.decode()
-        c.record(stream)
+    for _ in range(steps):
+        step.run()
     end.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
     total_ms = start.elapsed_time(end)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b, c in ev:
+        a.record(stream)
+        step.copy_and_write()
+        b.record(stream)
+        step.decode()
+        c.record(stream)
+    torch.cuda.synchronize()
     decode_ms = [b.elapsed_time(c) for _, b, c in ev]
     write_ms = [a.elapsed_time(b) for a, b, _ in ev]
     return total_ms, decode_ms, write_ms
@@ -735,7 +742,7 @@ def run_prefill(args, w0, device, rank, world):
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            cpu = prefill_cpu_baseline(w)
+            cpu = prefill_cpu_baseline(w, target_s=args.cpu_seconds)
         line = {
             "metric": "causal paged prefill attention TFLOP/s (4*Hq*D*keys attended per query row)",
             "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -757,7 +764,8 @@ def run_prefill(args, w0, device, rank, world):
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps, "device_errors": int(step.err.item()),
             "clocks": clk.summary(),
         }
-        print(json.dumps(line), flush=True)
+        return line
+    return None
 
 
 class BeamStep:
@@ -797,10 +805,11 @@ class BeamStep:
             offs, mem, sh = bm.prefix_groups(flat)
             host_s += time.perf_counter() - t0
             g = lambda a, dt=torch.int32: torch.from_numpy(np.asarray(a)).to(device=device, dtype=dt)  # noqa: E731
+            per_tok = w.num_kv_heads * w.head_dim * 2 * 2
             self.steps.append(dict(slots=g(slots, torch.int64), pairs=g(pairs, torch.int64) if len(pairs) else None,
                                    tables=g(tabs), lens=g(lens), offs=g(offs), mem=g(mem), sh=g(sh),
-                                   kv_bytes=int(lens.astype(np.int64).sum()) * w.num_kv_heads * w.head_dim * 2 * 2,
-                                   npairs=len(pairs)))
+                                   kv_bytes=int(lens.astype(np.int64).sum()) * per_tok,
+                                   unique_kv_bytes=unique_kv_bytes(tabs, lens, per_tok), npairs=len(pairs)))
             self.pairs_total += len(pairs)
         self.host_us_per_step = 1e6 * host_s / total_steps
         self.k_new, self.v_new = W.new_tokens(w, self.S, device)
@@ -905,11 +914,44 @@ def time_beam_e2e(step, idx, world):
     return reduce_max(a.elapsed_time(z), world, step.device), h2d, d2h
 
 
+def unique_kv_bytes(tables, lens, per_token):
+    """KV bytes of the distinct (physical block, slot) pairs a decode step reads:
+    a block shared by several sequences counts once, with the most tokens any of
+    them reads from it."""
+    tables = np.asarray(tables)
+    lens = np.asarray(lens).astype(np.int64)
+    nblk = -(-lens // 16)
+    j = np.arange(tables.shape[1])[None, :]
+    used = j < nblk[:, None]
+    valid = np.minimum(16, lens[:, None] - 16 * j)
+    blk = tables[used].astype(np.int64)
+    cnt = valid[used]
+    best = np.zeros(int(blk.max()) + 1 if blk.size else 1, dtype=np.int64)
+    np.maximum.at(best, blk, cnt)
+    return int(best.sum()) * per_token
+
+
+class L2Flush:
+    """A device buffer twice the 126 MB L2, written between timed steps so that no
+    step finds the previous step's data in L2."""
+
+    def __init__(self, device):
+        self.buf = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+
+    def __call__(self):
+        self.buf.fill_(1)
+
+
 def run_beam(args, w0, device, rank, world):
+    """Beam-search steps, each timed on its own with L2 flushed before it (the
+    beams' KV, about 70 MB, would otherwise stay in the 126 MB L2 from one step
+    to the next)."""
     w = rank_workload(w0, rank)
     step = BeamStep(w, device, args.warmup + args.steps)
     stream = torch.cuda.current_stream()
+    flush = L2Flush(device)
     for t in range(args.warmup):
+        flush()
         step.copy_and_write(t)
         step.decode(t)
     torch.cuda.synchronize()
@@ -918,24 +960,22 @@ def run_beam(args, w0, device, rank, world):
         dist.barrier()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     with ClockSampler(device) as clk:
-        a0 = torch.cuda.Event(enable_timing=True)
-        z0 = torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
         for i, (a, b, c) in enumerate(ev):
             t = args.warmup + i
+            flush()
             a.record(stream)
             step.copy_and_write(t)
             b.record(stream)
             step.decode(t)
             c.record(stream)
-        z0.record(stream)
         torch.cuda.synchronize()
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    total_ms = reduce_max(a0.elapsed_time(z0), world, device)
+    total_ms = reduce_max(sum(a.elapsed_time(c) for a, _, c in ev), world, device)
     timed = step.steps[args.warmup:]
     kv = sum(st["kv_bytes"] for st in timed)
+    ukv = sum(st["unique_kv_bytes"] for st in timed)
     value = kv * world / (total_ms / 1e3) / 1e9
     dec_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
     cw_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
@@ -948,11 +988,11 @@ def run_beam(args, w0, device, rank, world):
         e2e = {"value": round(e_kv * world / (e_ms / 1e3) / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms / n_e, 4)}
     peak, peak_kind = measured_peak_hbm()
-    achieved = kv / args.steps / (dec_ms / 1e3) / 1e9
+    achieved = ukv / args.steps / (dec_ms / 1e3) / 1e9
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            cpu = cpu_baseline(w0)
+            cpu = cpu_baseline(w0, target_s=args.cpu_seconds)
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
@@ -960,19 +1000,23 @@ def run_beam(args, w0, device, rank, world):
             "data": "synthetic (seeded N(0,1) K/V/q, seeded beam choices and block placement)",
             "config": {"workload": "beam: " + DESCR["beam"], "global_batch": step.S * world,
                        "seq_len": step.max_len, "parallelism": "replicas: requests sharded by rank, no collective",
-                       "l2": "logical KV bytes counted (the prompt is shared by the 4 beams of a request)"},
+                       "l2": "flushed before every timed step (256 MB write, outside the timed region); value "
+                             "counts logical KV bytes (the prompt once per beam)"},
             "us_decode": round(1e3 * dec_ms, 2), "us_copy_and_write": round(1e3 * cw_ms, 2),
             "us_decode_spread": spread_us([b.elapsed_time(c) for _, b, c in ev]),
+            "logical_kv_bytes_per_step": kv // args.steps, "unique_kv_bytes_per_step": ukv // args.steps,
+            "decode_call_logical_gbs": round(kv / args.steps / (dec_ms / 1e3) / 1e9, 1),
             "copy_pairs_per_step": round(sum(st["npairs"] for st in timed) / args.steps, 2),
             "host_block_manager_us_per_step": round(step.host_us_per_step, 1),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "traffic": None,
-                         "kernel": "paged_attention_decode_shared call (logical bytes; shared prompt read once per "
-                                   "request)", "peak_source": peak_kind},
+                         "frac": round(achieved / peak, 4), "traffic": ncu_traffic("beam"),
+                         "kernel": "paged_attention_decode_shared call (plan + grouped decode + merge); achieved "
+                                   "counts unique KV bytes (a shared block once)", "peak_source": peak_kind},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": sum(4 + (st["npairs"] > 0) for st in timed),
             "device_errors": int(step.err.item()), "clocks": clk.summary(),
         }
-        print(json.dumps(line), flush=True)
+        return line
+    return None
 
 
 def run_swap(args, device):
@@ -1069,6 +1113,114 @@ def run_swap(args, device):
     print(json.dumps(line), flush=True)
 
 
+def run_decode(args, w0, device, rank, world):
+    """The decode step (write + copy-on-write copies + decode) of a flat or
+    shared-prefix workload: K timed steps, e2e, roofline, CPU baseline."""
+    w = rank_workload(w0, rank)
+    step = Step(w, device, partition=args.partition, prefix_groups=not args.no_prefix_groups)
+    torch.cuda.synchronize()
+
+    with ClockSampler(device) as clk:
+        total_ms, decode_ms, write_ms = time_steps(step, args.steps, args.warmup, world, device)
+    err = int(step.err.item())
+    max_ms = reduce_max(total_ms, world, device)
+    ms_per_step = max_ms / args.steps
+    bytes_all = step.kv_bytes * world
+    value = bytes_all * args.steps / (max_ms / 1e3) / 1e9
+
+    e2e = None
+    if not args.no_e2e:
+        e_steps = max(5, args.steps // 2)
+        e_ms, h2d, d2h = time_e2e(step, e_steps, 3, world)
+        e_ms = reduce_max(e_ms, world, device)
+        e2e = {"value": round(bytes_all * e_steps / (e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": round(e_ms / e_steps, 4)}
+
+    peak, peak_kind = measured_peak_hbm()
+    dec_ms = statistics.mean(decode_ms)
+    elem = 1 if w.cache_dtype == "fp8" else 2
+    ukv = unique_kv_bytes(step.tables, step.lens, w.num_kv_heads * w.head_dim * 2 * elem)
+    shared = step.groups is not None
+    # a shared-prefix decode reads a shared block once: its roofline counts unique bytes
+    achieved = (ukv if shared else step.kv_bytes) / (dec_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": ncu_traffic(w0.name),
+                "kernel": ("paged_attention_decode_shared call (plan + grouped decode + merge); achieved counts "
+                           "unique KV bytes (a shared block once)") if shared else
+                          "paged_attention_decode call (plan + decode + merge launches)",
+                "peak_source": peak_kind, "frac_of_nominal_8tbps": round(achieved / NOMINAL_HBM_GBS, 4)}
+    if rank != 0:
+        return None
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w0, target_s=args.cpu_seconds)
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8-e4m3 cache, bf16 q/out, fp32 accumulate" if w.cache_dtype == "fp8" else w.cache_dtype,
+        "data": "synthetic (seeded N(0,1) K/V/q, seeded block placement)",
+        "config": {"workload": w0.name + ": " + DESCR[w0.name], "global_batch": step.S * world,
+                   "seq_len": step.max_len, "parallelism": "replicas: sequences sharded by rank, no collective",
+                   "l2": "inputs larger than L2 (pools %.1f GiB per GPU vs 126 MB L2)" % (
+                       2 * step.k_pool.numel() * step.k_pool.element_size() / 2**30),
+                   "partition_tokens": args.partition or "auto",
+                   "prefix_groups": shared},
+        "seq_tokens_per_s": round(step.seq_tokens * world * args.steps / (max_ms / 1e3), 1),
+        "us_per_step_per_layer": round(1e3 * ms_per_step, 2),
+        "us_decode": round(1e3 * dec_ms, 2), "us_write": round(1e3 * statistics.mean(write_ms), 2),
+        "us_decode_spread": spread_us(decode_ms),
+        "pct_of_8tbps": round(100 * value / world / NOMINAL_HBM_GBS, 2),
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": step.launches * args.steps, "device_errors": err,
+        "clocks": clk.summary(),
+    }
+    if w.lens == "shared":
+        line["logical_kv_bytes_per_step"] = step.kv_bytes
+        line["unique_kv_bytes_per_step"] = ukv
+        line["decode_call_logical_gbs"] = round(step.kv_bytes / (dec_ms / 1e3) / 1e9, 1)
+        line["memory_saving_by_sharing"] = round(step.mem_saving, 4)
+        line["divergence_step"] = divergence_step(w, device, args)
+    return line
+
+
+# The default run's other configurations (every workload the benchmark's
+# configuration list names besides the headline), each reported with the
+# fields of its own line; the tiny workload is a correctness case, not timed.
+CONFIG_KEYS = ("value", "unit", "ms_per_step", "steps", "warmup", "dtype", "seq_tokens_per_s",
+               "prompt_tokens_per_s", "us_decode", "us_write", "us_copy_and_write", "us_attention",
+               "us_decode_spread", "us_attention_spread", "logical_kv_bytes_per_step", "unique_kv_bytes_per_step",
+               "decode_call_logical_gbs", "memory_saving_by_sharing", "divergence_step", "copy_pairs_per_step",
+               "roofline", "cpu_baseline", "gpu_launches", "device_errors", "clocks")
+
+
+def run_configs(args, device, rank, world):
+    import copy
+    sub = copy.copy(args)
+    sub.steps = max(5, min(args.steps, 30))
+    sub.warmup = max(3, min(args.warmup, 5))
+    sub.no_e2e = True
+    sub.partition = 0
+    sub.no_prefix_groups = False
+    sub.cpu_seconds = min(args.cpu_seconds, 4.0)
+    out = {}
+    for name in ("mha13b", "shared_prefix", "fp8_long", "beam", "prefill70b"):
+        w0 = W.WORKLOADS[name]
+        if name == "beam":
+            line = run_beam(sub, w0, device, rank, world)
+        elif name.startswith("prefill"):
+            line = run_prefill(sub, w0, device, rank, world)
+        else:
+            line = run_decode(sub, w0, device, rank, world)
+        torch.cuda.empty_cache()
+        if line is not None:
+            entry = {"workload": line["config"]["workload"], "metric": line["metric"]}
+            entry.update({k: line[k] for k in CONFIG_KEYS if k in line})
+            out[name] = entry
+    return out
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -1080,7 +1232,10 @@ def main(argv=None):
     ap.add_argument("--num-seqs", type=int, default=0,
                     help="fewer sequences of the same shape (small cases for profiling; not a bench line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle work per CPU baseline (about)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="default run: skip the other configurations (the 'configs' object)")
     ap.add_argument("--swap", action="store_true", help="measure block swap to a host pool instead")
     ap.add_argument("--no-prefix-groups", action="store_true",
                     help="shared_prefix: plain decode (each sample reads the prompt's blocks itself)")
@@ -1099,27 +1254,10 @@ def main(argv=None):
     if rank == 0:
         pkv_build.build()
     torch.cuda.set_device(local)
-    if args.swap:
-        run_swap(args, torch.device("cuda", local))
-        return
-    if args.workload.startswith("prefill") or args.workload == "beam":
-        if world > 1:
-            import datetime
-            import torch.distributed as dist
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                    device_id=torch.device("cuda", local))
-            dist.barrier()
-            pkv_build.build()
-        if args.workload.startswith("prefill"):
-            run_prefill(args, w0, torch.device("cuda", local), rank, world)
-        else:
-            run_beam(args, w0, torch.device("cuda", local), rank, world)
-        if world > 1:
-            import torch.distributed as dist
-            dist.barrier()
-            dist.destroy_process_group()
-        return
     device = torch.device("cuda", local)
+    if args.swap:
+        run_swap(args, device)
+        return
     if world > 1:
         import datetime
         import torch.distributed as dist
@@ -1127,63 +1265,17 @@ def main(argv=None):
         dist.barrier()
         pkv_build.build()
 
-    w = rank_workload(w0, rank)
-    step = Step(w, device, partition=args.partition, prefix_groups=not args.no_prefix_groups)
-    torch.cuda.synchronize()
-
-    with ClockSampler(device) as clk:
-        total_ms, decode_ms, write_ms = time_steps(step, args.steps, args.warmup, world, device)
-    err = int(step.err.item())
-    max_ms = reduce_max(total_ms, world, device)
-    ms_per_step = max_ms / args.steps
-    bytes_all = step.kv_bytes * world
-    value = bytes_all * args.steps / (max_ms / 1e3) / 1e9
-
-    e2e = None
-    if not args.no_e2e:
-        e_ms, h2d, d2h = time_e2e(step, max(5, args.steps // 2), 3, world)
-        e_ms = reduce_max(e_ms, world, device)
-        e_steps = max(5, args.steps // 2)
-        e2e = {"value": round(bytes_all * e_steps / (e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": round(e_ms / e_steps, 4)}
-
-    peak, peak_kind = measured_peak_hbm()
-    dec_ms = statistics.mean(decode_ms)
-    achieved = step.kv_bytes / (dec_ms / 1e3) / 1e9
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": ncu_traffic(args.workload),
-                "kernel": "paged_attention_decode call (plan + decode + merge launches)",
-                "peak_source": peak_kind, "frac_of_nominal_8tbps": round(achieved / NOMINAL_HBM_GBS, 4)}
-
-    if rank == 0:
-        cpu = None
-        if world == 1 and not args.no_cpu_baseline:
-            cpu = cpu_baseline(w0)
-        line = {
-            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None,
-            "dtype": "fp8-e4m3 cache, bf16 q/out, fp32 accumulate" if w.cache_dtype == "fp8" else w.cache_dtype,
-            "data": "synthetic (seeded N(0,1) K/V/q, seeded block placement)",
-            "config": {"workload": args.workload + ": " + DESCR[args.workload], "global_batch": step.S * world,
-                       "seq_len": step.max_len, "parallelism": "replicas: sequences sharded by rank, no collective",
-                       "l2": "inputs larger than L2 (pools %.1f GiB per GPU vs 126 MB L2)" % (
-                           2 * step.k_pool.numel() * step.k_pool.element_size() / 2**30),
-                       "partition_tokens": args.partition or "auto",
-                       "prefix_groups": step.groups is not None},
-            "seq_tokens_per_s": round(step.seq_tokens * world * args.steps / (max_ms / 1e3), 1),
-            "us_per_step_per_layer": round(1e3 * ms_per_step, 2),
-            "us_decode": round(1e3 * dec_ms, 2), "us_write": round(1e3 * statistics.mean(write_ms), 2),
-            "us_decode_spread": spread_us(decode_ms),
-            "pct_of_8tbps": round(100 * value / world / NOMINAL_HBM_GBS, 2),
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": step.launches * args.steps, "device_errors": err,
-            "clocks": clk.summary(),
-        }
-        if w.lens == "shared":
-            line["memory_saving_by_sharing"] = round(step.mem_saving, 4)
-            line["divergence_step"] = divergence_step(w, device, args)
+    if args.workload.startswith("prefill"):
+        line = run_prefill(args, w0, device, rank, world)
+    elif args.workload == "beam":
+        line = run_beam(args, w0, device, rank, world)
+    else:
+        line = run_decode(args, w0, device, rank, world)
+    if args.workload == "gqa70b" and not args.num_seqs and not args.no_configs:
+        configs = run_configs(args, device, rank, world)
+        if line is not None:
+            line["configs"] = configs
+    if rank == 0 and line is not None:
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

@@ -175,23 +175,32 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
     __shared__ int hist[kMaxBuckets];
     __shared__ int own_blocks[kSmemSeqs];  // blocks of sequence s outside its shared prefix
     __shared__ unsigned long long units_of[kMaxCandidates];
-    __shared__ int chosen;
+    __shared__ int chosen, total_items;
     __shared__ int n_subs, n_members;
     const int tid = threadIdx.x;
     // automatic partitioning ends each context with geometrically shrinking pieces
     const bool geometric = fixed_partition == 0;
     const int mb = min_partition / kBlockSize;
+    const bool grouped = p.num_groups > 0;
 
-    // The workspace and the output may still be in use by the previous kernel.
-    pdl_wait();
+    // The plan reads caller inputs no kernel of this library writes (lengths,
+    // tables, group hints) and works in shared memory up to its scan; only its
+    // global writes (header, work list, partition counts, zero rows) must wait for
+    // the previous kernel on the stream, whose predecessors may still read this
+    // workspace and output.  So without prefix groups the wait comes after the
+    // scan, and the plan's work overlaps that kernel (the step's KV write).  The
+    // grouped plan claims members in the workspace itself: it waits first.  Either
+    // way the wait comes before the plan ends, so the decode that waits for the
+    // plan also finds the KV write done.
     pdl_trigger();
+    if (grouped) pdl_wait();
 
     // 0. shared-prefix subgroups: sequence s then owns blocks [seq_k[s], B) and
     //    its subgroup computes blocks [0, seq_k[s]) once for all its members
     if (tid == 0) n_subs = n_members = 0;
     if (tid < kMaxCandidates) units_of[tid] = 0;
+    for (int b = tid; b < kMaxBuckets; b += kPlanThreads) hist[b] = 0;
     __syncthreads();
-    const bool grouped = p.num_groups > 0;
     if (grouped) build_groups(p, &n_subs, &n_members);
     const int num_subs = n_subs;
     // blocks of s after its shared prefix (the length is clamped and counted once, here)
@@ -229,31 +238,15 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
             chosen = P;
         }
     }
-    for (int b = tid; b < kMaxBuckets; b += kPlanThreads) hist[b] = 0;
     __syncthreads();
     const int P = chosen;
     const int nb_top = P / kBlockSize;
     const int nbuckets = nb_top < kMaxBuckets ? nb_top : kMaxBuckets;
 
-    // 2. histogram of item sizes; partitions per sequence (shared ones first)
-    for (int s = tid; s < p.num_seqs; s += kPlanThreads) {
-        const int k = grouped ? p.seq_k[s] : 0;
-        const int B = own(s);
-        p.nparts[s] = count_pieces(k, nb_top, mb, geometric) +
-                      for_each_piece(B, nb_top, mb, geometric,
-                                     [&](int, int n) { atomicAdd(&hist[bucket_of(n, nb_top, nbuckets)], 1); });
-        if (B + k == 0) {
-            // an empty context produces a zero output row (nothing else writes it)
-            const size_t row = (size_t)s * p.num_heads * p.head_dim;
-            const int n = p.num_heads * p.head_dim;
-            for (int e = 0; e < n; ++e) {
-                if (zero_out_dtype == 0)
-                    static_cast<float*>(p.out)[row + e] = 0.f;
-                else
-                    static_cast<__nv_bfloat16*>(p.out)[row + e] = __float2bfloat16(0.f);
-            }
-        }
-    }
+    // 2. histogram of item sizes
+    for (int s = tid; s < p.num_seqs; s += kPlanThreads)
+        for_each_piece(own(s), nb_top, mb, geometric,
+                       [&](int, int n) { atomicAdd(&hist[bucket_of(n, nb_top, nbuckets)], 1); });
     for (int q = tid; q < num_subs; q += kPlanThreads)
         for_each_piece(p.sub_info[q].z, nb_top, mb, geometric,
                        [&](int, int n) { atomicAdd(&hist[bucket_of(n, nb_top, nbuckets)], 1); });
@@ -274,24 +267,41 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
             if (b >= 0) hist[b] = running + incl - v;
             running += __shfl_sync(0xffffffffu, incl, 31);
         }
-        if (tid == 0) {
-            p.hdr->num_items = running;
-            p.hdr->num_units = running * p.num_kv_heads;
-            p.hdr->partition = P;
-            p.hdr->counter = 0;
-            p.hdr->timeout = 0;
-            p.hdr->num_subs = num_subs;
-            p.hdr->num_members = n_members;
-        }
+        if (tid == 0) total_items = running;
     }
+    if (!grouped) pdl_wait();
     __syncthreads();
 
-    // 4. scatter the items (order inside a bucket does not affect results);
-    //    a sequence's shared partitions come first, then its own
+    // 4. global writes: header, partitions per sequence (shared ones first), zero
+    //    rows of empty contexts, and the items scattered into the work list (order
+    //    inside a bucket does not affect results; a sequence's shared partitions
+    //    come first, then its own)
+    if (tid == 0) {
+        p.hdr->num_items = total_items;
+        p.hdr->num_units = total_items * p.num_kv_heads;
+        p.hdr->partition = P;
+        p.hdr->counter = 0;
+        p.hdr->timeout = 0;
+        p.hdr->num_subs = num_subs;
+        p.hdr->num_members = n_members;
+    }
     for (int s = tid; s < p.num_seqs; s += kPlanThreads) {
         const int k = grouped ? p.seq_k[s] : 0;
+        const int B = own(s);
         int part = count_pieces(k, nb_top, mb, geometric);
-        for_each_piece(own(s), nb_top, mb, geometric, [&](int first, int n) {
+        p.nparts[s] = part + count_pieces(B, nb_top, mb, geometric);
+        if (B + k == 0) {
+            // an empty context produces a zero output row (nothing else writes it)
+            const size_t row = (size_t)s * p.num_heads * p.head_dim;
+            const int n = p.num_heads * p.head_dim;
+            for (int e = 0; e < n; ++e) {
+                if (zero_out_dtype == 0)
+                    static_cast<float*>(p.out)[row + e] = 0.f;
+                else
+                    static_cast<__nv_bfloat16*>(p.out)[row + e] = __float2bfloat16(0.f);
+            }
+        }
+        for_each_piece(B, nb_top, mb, geometric, [&](int first, int n) {
             const int pos = atomicAdd(&hist[bucket_of(n, nb_top, nbuckets)], 1);
             p.items[pos] = make_int4(s, part++, k + first, n);
         });

@@ -62,3 +62,27 @@ def test_device_arm_line():
     assert {"sm_mhz", "sm_max_mhz", "reasons"} <= set(c)
     s = d["us_decode_spread"]
     assert s["p10"] <= s["median"] <= s["p90"]
+    # the other configurations of the benchmark, each with its own roofline and errors
+    cf = d["configs"]
+    assert set(cf) == {"mha13b", "shared_prefix", "fp8_long", "beam", "prefill70b"}
+    for name, e in cf.items():
+        assert e["value"] > 0 and e["device_errors"] == 0, name
+        assert {"bound", "achieved", "peak", "unit", "frac", "traffic"} <= set(e["roofline"]), name
+        # the beam step (68 MB of unique KV, few long work units) is latency-bound well below
+        # the copy bandwidth; far above 1 would mean the timed kernel skipped work
+        assert 0.05 < e["roofline"]["frac"] < 1.3, (name, e["roofline"])
+    assert cf["shared_prefix"]["unique_kv_bytes_per_step"] < cf["shared_prefix"]["logical_kv_bytes_per_step"]
+    assert cf["beam"]["unique_kv_bytes_per_step"] < cf["beam"]["logical_kv_bytes_per_step"]
+
+
+def test_unique_kv_bytes_counts_a_shared_block_once():
+    """Two sequences sharing their first two blocks: 16 + 16 shared tokens, then
+    8 and 3 tokens in their own last blocks; a block's count is the most tokens
+    any sequence reads from it."""
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import bench
+    tables = np.array([[5, 6, 7], [5, 6, 9]], np.int32)
+    assert bench.unique_kv_bytes(tables, np.array([40, 35]), 10) == (16 + 16 + 8 + 3) * 10
+    assert bench.unique_kv_bytes(tables, np.array([20, 40]), 1) == 16 + 16 + 8      # block 6: 4 vs 16 tokens
+    assert bench.unique_kv_bytes(tables, np.array([0, 0]), 1) == 0
