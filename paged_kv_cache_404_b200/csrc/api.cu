@@ -31,8 +31,9 @@ using namespace pkv;
 
 namespace {
 
-// Smallest partition the automatic plan considers, and how many units per
-// warp it aims for before it stops halving the partition.
+// Smallest partition the automatic plan considers for a batch whose workspace
+// is large (see min_partition_of), and how many units per warp it aims for
+// before it stops halving the partition.
 constexpr int kMinAutoPartition = 256;
 constexpr int kUnitsPerWorker = 3;
 constexpr int kMaxCandidates = 12;
@@ -94,14 +95,36 @@ bool rows_tensor_map(CUtensorMap* map, const void* base, int head_dim, int heads
     return r == CUDA_SUCCESS;
 }
 
-int min_partition_of(int partition_tokens) {
-    return partition_tokens > 0 ? partition_tokens : kMinAutoPartition;
-}
+// Workspace within which automatic partitioning may cut below kMinAutoPartition
+// tokens (at most the no-alloc decode's scratch, so that whatever that entry point
+// accepted with 256-token pieces it still accepts).
+constexpr size_t kSmallBatchWorkspace = PKV_NOALLOC_SCRATCH_BYTES;
 
-int max_parts_of(int max_context_len, int partition_tokens) {
-    const int P = min_partition_of(partition_tokens);
+int parts_for(int max_context_len, int P) {
     const int n = (max_context_len + P - 1) / P;
     return n > 0 ? n : 1;
+}
+
+// Smallest partition the plan may use.  A fixed partition is the caller's.
+// Automatic: 256 tokens, or 128 / 64 when the workspace for pieces that small
+// stays within kSmallBatchWorkspace -- a small batch then gets enough pieces to
+// keep every warp busy (few sequences would otherwise leave most warps idle
+// while each walks a long piece); large batches have the work already.
+int min_partition_of(int partition_tokens, int num_seqs, int num_heads, int head_dim, int max_context_len,
+                     bool shared) {
+    if (partition_tokens > 0) return partition_tokens;
+    for (int P = kMinAutoPartition / 4; P < kMinAutoPartition; P <<= 1) {
+        const int parts = parts_for(max_context_len, P);
+        const size_t bytes = shared ? ws_layout_shared(num_seqs, num_heads, head_dim, parts).total
+                                    : ws_layout(num_seqs, num_heads, head_dim, parts).total;
+        if (bytes <= kSmallBatchWorkspace) return P;
+    }
+    return kMinAutoPartition;
+}
+
+int max_parts_of(int partition_tokens, int num_seqs, int num_heads, int head_dim, int max_context_len, bool shared) {
+    return parts_for(max_context_len,
+                     min_partition_of(partition_tokens, num_seqs, num_heads, head_dim, max_context_len, shared));
 }
 
 // Optional shared-prefix hints of pkv_paged_attention_decode_shared.
@@ -169,7 +192,9 @@ size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim, int
     if (num_seqs < 0 || num_heads <= 0 || head_dim <= 0 || max_context_len < 0 || partition_tokens < 0 ||
         partition_tokens % kBlockSize != 0)
         return 0;
-    return ws_layout(num_seqs, num_heads, head_dim, max_parts_of(max_context_len, partition_tokens)).total;
+    return ws_layout(num_seqs, num_heads, head_dim,
+                     max_parts_of(partition_tokens, num_seqs, num_heads, head_dim, max_context_len, false))
+        .total;
 }
 
 int pkv_paged_attention_decode(void* out, const void* q, int q_dtype, const void* k_pool, const void* v_pool,
@@ -189,7 +214,9 @@ size_t pkv_decode_workspace_bytes_shared(int num_seqs, int num_heads, int head_d
     if (num_seqs < 0 || num_heads <= 0 || head_dim <= 0 || max_context_len < 0 || partition_tokens < 0 ||
         partition_tokens % kBlockSize != 0)
         return 0;
-    return ws_layout_shared(num_seqs, num_heads, head_dim, max_parts_of(max_context_len, partition_tokens)).total;
+    return ws_layout_shared(num_seqs, num_heads, head_dim,
+                            max_parts_of(partition_tokens, num_seqs, num_heads, head_dim, max_context_len, true))
+        .total;
 }
 
 int pkv_paged_attention_decode_shared(void* out, const void* q, int q_dtype, const void* k_pool, const void* v_pool,
@@ -269,7 +296,8 @@ int decode_impl(void* out, const void* q, int q_dtype, const void* k_pool, const
     const bool f32 = q_dtype == PKV_F32;
     const bool fp8 = cache_dtype == PKV_FP8_E4M3;
     const int group = num_heads / num_kv_heads;
-    const int max_parts = max_parts_of(max_context_len, partition_tokens);
+    const int max_parts =
+        max_parts_of(partition_tokens, num_seqs, num_heads, head_dim, max_context_len, pg.layout);
     const WsLayout ws = pg.layout ? ws_layout_shared(num_seqs, num_heads, head_dim, max_parts)
                                   : ws_layout(num_seqs, num_heads, head_dim, max_parts);
     if (workspace_bytes < ws.total) return PKV_EINVAL;
@@ -318,7 +346,7 @@ int decode_impl(void* out, const void* q, int q_dtype, const void* k_pool, const
     p.sub_members = pg.layout ? reinterpret_cast<int*>(w + ws.sub_members) : nullptr;
 
     // Partition candidates: min_partition << c, up to the first that covers max_context_len.
-    const int min_p = min_partition_of(partition_tokens);
+    const int min_p = min_partition_of(partition_tokens, num_seqs, num_heads, head_dim, max_context_len, pg.layout);
     int ncand = 1;
     if (partition_tokens == 0)
         while (ncand < kMaxCandidates && ((long long)min_p << (ncand - 1)) < max_context_len) ++ncand;

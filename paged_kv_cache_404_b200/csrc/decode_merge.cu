@@ -9,10 +9,12 @@
 // and a sequence with a single partition was written by the decode kernel.
 //
 // One warp per (sequence, query head).  Lanes are 4 partition groups x 8
-// head_dim slices (16 elements each): group r takes partitions r, r+4, ...,
-// so a 60-partition context costs 15 dependent load rounds instead of 60; the
-// four groups are combined with shuffles at the end.  Deterministic: the order
-// of additions depends only on the partition count.
+// head_dim slices (16 elements each): group r takes partitions r, r+4, ...;
+// the first four partitions are loaded in one round (weights and outputs
+// together, before the max is known), so up to four partitions cost two
+// dependent rounds of loads (the partition count, then the partials); the four
+// groups are combined with shuffles at the end.  Deterministic: the order of additions
+// depends only on the partition count.
 #include "pkv_common.cuh"
 
 namespace pkv {
@@ -20,7 +22,8 @@ namespace pkv {
 template <int D, typename OutT>
 __global__ void __launch_bounds__(256) decode_merge_kernel(DecodeParams p) {
     pdl_wait();
-    constexpr int SL = D / 8;  // head_dim elements per lane
+    constexpr int SL = D / 8;   // head_dim elements per lane
+    constexpr int KR = 1;       // partitions per lane group loaded in the first round (4 per warp)
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (warp >= p.num_seqs * p.num_heads) return;
@@ -30,32 +33,61 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(DecodeParams p) {
     const size_t base = (size_t)warp * p.max_parts;
     const int grp = lane >> 3, slice = lane & 7;
 
+    // The first 4 partitions: each lane group loads its partition's (m, l) and its
+    // head_dim slice of its output in one round of loads, before the max is
+    // known.  Further partitions take further rounds.
     float M = -INFINITY;
-    for (int i = lane; i < n; i += 32) {
-        const float2 ml = p.part_ml[base + i];
-        if (ml.y > 0.f) M = fmaxf(M, ml.x);
-    }
+    float2 ml[KR];
+    float4 x[KR][SL / 4];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    for (int k = 0; k < KR; ++k) {
+        const int i = grp + 4 * k;
+        ml[k] = make_float2(-INFINITY, 0.f);
+        if (i < n) {
+            ml[k] = p.part_ml[base + i];
+            const float4* src = reinterpret_cast<const float4*>(p.part_o + (base + i) * D + slice * SL);
+#pragma unroll
+            for (int v = 0; v < SL / 4; ++v) x[k][v] = src[v];
+        }
+        if (ml[k].y > 0.f) M = fmaxf(M, ml[k].x);
+    }
+    for (int i = grp + 4 * KR; i < n; i += 4) {
+        const float2 m2 = p.part_ml[base + i];
+        if (m2.y > 0.f) M = fmaxf(M, m2.x);
+    }
+    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 8));
+    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 16));
 
     float acc[SL];
 #pragma unroll
     for (int e = 0; e < SL; ++e) acc[e] = 0.f;
     float W = 0.f;
     if (M != -INFINITY) {
-#pragma unroll 2
-        for (int i = grp; i < n; i += 4) {
-            const float2 ml = p.part_ml[base + i];
-            const float w = ml.y > 0.f ? ml.y * exp2f(ml.x - M) : 0.f;
+#pragma unroll
+        for (int k = 0; k < KR; ++k) {
+            if (grp + 4 * k >= n) continue;
+            const float w = ml[k].y > 0.f ? ml[k].y * exp2f(ml[k].x - M) : 0.f;
+            W += w;
+#pragma unroll
+            for (int v = 0; v < SL / 4; ++v) {
+                acc[4 * v] += w * x[k][v].x;
+                acc[4 * v + 1] += w * x[k][v].y;
+                acc[4 * v + 2] += w * x[k][v].z;
+                acc[4 * v + 3] += w * x[k][v].w;
+            }
+        }
+        for (int i = grp + 4 * KR; i < n; i += 4) {
+            const float2 m2 = p.part_ml[base + i];
+            const float w = m2.y > 0.f ? m2.y * exp2f(m2.x - M) : 0.f;
             W += w;
             const float4* src = reinterpret_cast<const float4*>(p.part_o + (base + i) * D + slice * SL);
 #pragma unroll
             for (int v = 0; v < SL / 4; ++v) {
-                const float4 x = src[v];
-                acc[4 * v] += w * x.x;
-                acc[4 * v + 1] += w * x.y;
-                acc[4 * v + 2] += w * x.z;
-                acc[4 * v + 3] += w * x.w;
+                const float4 y = src[v];
+                acc[4 * v] += w * y.x;
+                acc[4 * v + 1] += w * y.y;
+                acc[4 * v + 2] += w * y.z;
+                acc[4 * v + 3] += w * y.w;
             }
         }
     }
