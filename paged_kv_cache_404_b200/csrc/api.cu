@@ -97,8 +97,9 @@ bool rows_tensor_map(CUtensorMap* map, const void* base, int head_dim, int heads
 
 // Workspace within which automatic partitioning may cut below kMinAutoPartition
 // tokens (at most the no-alloc decode's scratch, so that whatever that entry point
-// accepted with 256-token pieces it still accepts).
+// accepted with 256-token pieces it still accepts), and the smaller partition.
 constexpr size_t kSmallBatchWorkspace = PKV_NOALLOC_SCRATCH_BYTES;
+constexpr int kSmallBatchPartition = 128;
 
 int parts_for(int max_context_len, int P) {
     const int n = (max_context_len + P - 1) / P;
@@ -106,20 +107,19 @@ int parts_for(int max_context_len, int P) {
 }
 
 // Smallest partition the plan may use.  A fixed partition is the caller's.
-// Automatic: 256 tokens, or 128 / 64 when the workspace for pieces that small
-// stays within kSmallBatchWorkspace -- a small batch then gets enough pieces to
-// keep every warp busy (few sequences would otherwise leave most warps idle
-// while each walks a long piece); large batches have the work already.
+// Automatic: 256 tokens, or 128 when the workspace for 128-token pieces stays
+// within kSmallBatchWorkspace -- a small batch then gets enough pieces to keep
+// the warps busy (few sequences would otherwise leave most warps idle while each
+// walks a long piece); large batches have the work already.  (64-token pieces
+// were measured too: the beam step's decode call took 61 us against 51 with
+// 128, the extra partitions costing the plan and the merge more than they gave.)
 int min_partition_of(int partition_tokens, int num_seqs, int num_heads, int head_dim, int max_context_len,
                      bool shared) {
     if (partition_tokens > 0) return partition_tokens;
-    for (int P = kMinAutoPartition / 4; P < kMinAutoPartition; P <<= 1) {
-        const int parts = parts_for(max_context_len, P);
-        const size_t bytes = shared ? ws_layout_shared(num_seqs, num_heads, head_dim, parts).total
-                                    : ws_layout(num_seqs, num_heads, head_dim, parts).total;
-        if (bytes <= kSmallBatchWorkspace) return P;
-    }
-    return kMinAutoPartition;
+    const int parts = parts_for(max_context_len, kSmallBatchPartition);
+    const size_t bytes = shared ? ws_layout_shared(num_seqs, num_heads, head_dim, parts).total
+                                : ws_layout(num_seqs, num_heads, head_dim, parts).total;
+    return bytes <= kSmallBatchWorkspace ? kSmallBatchPartition : kMinAutoPartition;
 }
 
 int max_parts_of(int partition_tokens, int num_seqs, int num_heads, int head_dim, int max_context_len, bool shared) {

@@ -130,17 +130,18 @@ def test_workspace_bytes(L):
 
 
 def test_automatic_partitions_of_small_batches(L):
-    """Automatic partitioning cuts below 256 tokens (128, then 64) only while the
+    """Automatic partitioning cuts 128-token pieces instead of 256 only while the
     workspace of the smaller pieces stays within the no-alloc scratch (32 MiB):
-    small batches get enough pieces to occupy every warp, large batches keep
+    small batches get enough pieces to occupy the warps, large batches keep
     their workspace, and anything the no-alloc decode accepted with 256-token
     pieces it still accepts."""
     f, g = L.lib().pkv_decode_workspace_bytes, L.lib().pkv_decode_workspace_bytes_shared
     lim = 32 << 20
-    assert f(4, 2, 64, 1024, 0) == f(4, 2, 64, 1024, 64)            # tiny: 64-token pieces
-    assert g(64, 32, 128, 1048, 0) == g(64, 32, 128, 1048, 64)      # 16 x 4 beams, 32 heads
-    assert f(64, 40, 128, 2048, 0) == f(64, 40, 128, 2048, 128)     # 64 x 40 heads: 128 fits, 64 does not
-    assert f(64, 40, 128, 2048, 64) > lim >= f(64, 40, 128, 2048, 128)
+    assert f(4, 2, 64, 1024, 0) == f(4, 2, 64, 1024, 128)          # tiny
+    assert g(64, 32, 128, 1048, 0) == g(64, 32, 128, 1048, 128)    # 16 x 4 beams, 32 heads
+    assert f(64, 40, 128, 2048, 0) == f(64, 40, 128, 2048, 128)    # 64 sequences x 40 heads
+    assert f(64, 64, 128, 2048, 128) > lim                          # 64 x 64 heads: 128 does not fit
+    assert f(64, 64, 128, 2048, 0) == f(64, 64, 128, 2048, 256)
     assert f(256, 64, 128, 4096, 0) == f(256, 64, 128, 4096, 256)  # large batches unchanged
     assert f(128, 32, 128, 32768, 0) == f(128, 32, 128, 32768, 256)
     for S, H, M in ((64, 64, 2048), (8, 1, 125200), (2, 64, 16384), (192, 32, 1513), (1, 8, 1 << 20)):
