@@ -569,27 +569,28 @@ __global__ void __launch_bounds__(FP8 ? 448 : 320, 1)
                 auto chunk_addr = [&](int c) {  // c = 0..15: half c / 8, chunk c % 8 of row r
                     return qt + (c >> 3) * (kTcRows * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4);
                 };
-                uint32_t amax_bits = 0;
-#pragma unroll 4
+                uint4 v[16];  // the row, one pass: loads, maximum, conversion, stores
+                uint32_t m2 = 0;  // two 16-bit maxima of |x| as bits (sign cleared)
+#pragma unroll
                 for (int c = 0; c < 16; ++c) {
-                    const uint4 v = ld_shared_v4(chunk_addr(c));
-                    const uint32_t m01 = max(max(v.x & 0x7FFFu, (v.x >> 16) & 0x7FFFu), max(v.y & 0x7FFFu, (v.y >> 16) & 0x7FFFu));
-                    const uint32_t m23 = max(max(v.z & 0x7FFFu, (v.z >> 16) & 0x7FFFu), max(v.w & 0x7FFFu, (v.w >> 16) & 0x7FFFu));
-                    amax_bits = max(amax_bits, max(m01, m23));
+                    v[c] = ld_shared_v4(chunk_addr(c));
+                    m2 = __vmaxu2(m2, __vmaxu2(__vmaxu2(v[c].x & 0x7FFF7FFFu, v[c].y & 0x7FFF7FFFu),
+                                               __vmaxu2(v[c].z & 0x7FFF7FFFu, v[c].w & 0x7FFF7FFFu)));
                 }
+                const uint32_t amax_bits = max(m2 & 0xFFFFu, m2 >> 16);
                 // e = 14 - floor(log2 max|q|) within [-126, 126]; an all-zero row keeps e = 0
                 const int ex = amax_bits != 0 ? (int)(amax_bits >> 7) - 127 : 14;
                 const int e = min(max(14 - ex, -126), 126);
                 const float up = __uint_as_float((uint32_t)(127 + e) << 23);
                 row_scale = __uint_as_float((uint32_t)(127 - e) << 23) * p.score_scale;
-#pragma unroll 4
+#pragma unroll
                 for (int c = 0; c < 16; ++c) {
-                    uint4 v = ld_shared_v4(chunk_addr(c));
-                    v.x = bf16x2_to_f16x2_scaled(v.x, up);
-                    v.y = bf16x2_to_f16x2_scaled(v.y, up);
-                    v.z = bf16x2_to_f16x2_scaled(v.z, up);
-                    v.w = bf16x2_to_f16x2_scaled(v.w, up);
-                    st_shared_v4(chunk_addr(c), v);
+                    uint4 w = v[c];
+                    w.x = bf16x2_to_f16x2_scaled(w.x, up);
+                    w.y = bf16x2_to_f16x2_scaled(w.y, up);
+                    w.z = bf16x2_to_f16x2_scaled(w.z, up);
+                    w.w = bf16x2_to_f16x2_scaled(w.w, up);
+                    st_shared_v4(chunk_addr(c), w);
                 }
                 fence_proxy_async_smem();  // read by the tensor core
                 __syncwarp();
