@@ -760,7 +760,8 @@ def run_prefill(args, w0, device, rank, world):
             "us_attention_spread": spread_us([b.elapsed_time(c) for _, b, c in ev]),
             "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(achieved / peak, 4), "traffic": ncu_traffic(w0.name),
-                         "kernel": "prefill_tc_kernel (tcgen05.mma, TMEM accumulators)", "peak_source": peak_kind},
+                         "kernel": ("prefill_fp8_kernel (64-key tiles" if step.fp8 else "prefill_bf16_kernel (128-key tiles")
+                         + "; tcgen05.mma, TMEM accumulators)", "peak_source": peak_kind},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps, "device_errors": int(step.err.item()),
             "clocks": clk.summary(),
         }
