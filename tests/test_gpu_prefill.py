@@ -28,7 +28,7 @@ def _built():
 class PrefillCase:
     """Sequences with context lengths `ctx` whose last `nq` tokens are queries."""
 
-    def __init__(self, Hq, Hkv, ctx, nq, seed, nan_pool=True, cache="bf16"):
+    def __init__(self, Hq, Hkv, ctx, nq, seed, nan_pool=True, cache="bf16", k_growth=None):
         import paged_kv_cache_404_b200 as pkv
         self.w = W.Workload("pf", Hq, Hkv, 128, cache, "bf16", len(ctx), "uniform", 1, 1, seed=seed)
         self.cache = cache
@@ -52,6 +52,10 @@ class PrefillCase:
             self.kp, self.vp, _, _ = W.random_pools(self.w, self.NB, "cuda")
         total = int(self.ctx.sum())
         k, v = W.logical_kv(self.w, total, "cuda", stream=80)
+        if k_growth and total:
+            # keys that grow along the sequence: token p of a prompt scaled by 1 + p / k_growth
+            pos = torch.from_numpy(np.concatenate([np.arange(int(c)) for c in ctx]).astype(np.float32)).cuda()
+            k = (k.float() * (1.0 + pos / k_growth).view(-1, *([1] * (k.dim() - 1)))).to(k.dtype)
         # per-tensor FP8 scales amax / 448 of the written tokens (1 for bf16)
         self.k_scale = float(k.abs().max().float().item()) / 448.0 if cache == "fp8" and total else 1.0
         self.v_scale = float(v.abs().max().float().item()) / 448.0 if cache == "fp8" and total else 1.0
@@ -85,6 +89,21 @@ class PrefillCase:
 
 RAGGED = ([1, 15, 16, 17, 64, 65, 200, 300, 100, 129, 33],
           [1, 15, 16, 17, 64, 65, 200, 37, 1, 128, 20])
+
+
+@pytest.mark.parametrize("cache", ["bf16", "fp8"])
+def test_growing_keys_move_the_reference_max(cache):
+    """Keys whose magnitude grows along the prompt (1 + p / 40): every KV tile's largest
+    score exceeds the previous tiles' by more than 2^8 in the exponent, so each row's
+    reference maximum moves tile after tile and O is rescaled in TMEM mid-row (the bf16
+    kernel computes a tile's probabilities before its maximum is known and redoes them
+    there).  Every element against the oracle."""
+    c = PrefillCase(16, 4, [700, 520, 300, 129], [700, 400, 300, 1], seed=77, cache=cache, k_growth=40.0)
+    got = out_to_f64(c.run())
+    ref, bad = c.oracle()
+    assert bad == 0 and int(c.err.item()) == 0
+    assert np.isfinite(got).all()
+    assert_close(got, ref, cache, "prefill growing keys")
 
 
 @pytest.mark.parametrize("Hq,Hkv", [(8, 8), (16, 4), (64, 8)])

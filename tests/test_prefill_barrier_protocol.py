@@ -299,6 +299,9 @@ def _run_bf16(nt, seed, kst=3, vst=2, plant=None):
     roles = {"producer": producer(), "issuer": issuer(), "softmax0": softmax(0), "softmax1": softmax(1)}
     cur = {k: next(g, None) for k, g in roles.items()}
     pv_done = {0: -1, 1: -1}
+    # how eagerly the tensor core and the copies progress, drawn per schedule, so that
+    # some schedules let products or copies lag far behind the threads
+    weight = {"tensor": rng.choice((0.05, 0.3, 1.0, 3.0)), "tma": rng.choice((0.05, 0.3, 1.0, 3.0))}
     for _ in range(400000):
         ready = [k for k, st in cur.items() if st is not None and
                  (st[0] != "wait" or (bars[st[1]].done & 1) != (st[2] & 1))]
@@ -310,7 +313,7 @@ def _run_bf16(nt, seed, kst=3, vst=2, plant=None):
             if any(v is not None for v in cur.values()):
                 issues.append("deadlock: " + ", ".join("%s waits %s" % (k, v[1:]) for k, v in cur.items() if v))
             return issues
-        k = rng.choice(ready)
+        k = rng.choices(ready, weights=[weight.get(r, 1.0) for r in ready])[0]
         if k == "tensor":
             op = tensor_q.pop(0)
             if op[0] == "commit":
@@ -345,8 +348,11 @@ def _run_bf16(nt, seed, kst=3, vst=2, plant=None):
 def _cases_bf16(n):
     rng = random.Random(4321)
     for i in range(n):
+        if rng.random() < 0.15:   # Q tile 1 past the last query row: it reads no KV tile
+            yield [rng.randint(1, 9), 0], i
+            continue
         n1 = rng.randint(1, 9)
-        n0 = rng.randint(0, n1)   # Q tile 0 never reads more KV tiles than Q tile 1
+        n0 = rng.randint(0, n1)   # otherwise Q tile 0 never reads more KV tiles than Q tile 1
         yield [n0, n1], i
 
 
@@ -357,7 +363,7 @@ def test_bf16_protocol_is_free_of_hazards_and_deadlock(kst, vst):
         assert not issues, (nt, seed, issues[:2])
 
 
-@pytest.mark.parametrize("plant,least", [("early_k_empty", 20), ("s_before_pv", 200), ("no_v_landing", 10)])
+@pytest.mark.parametrize("plant,least", [("early_k_empty", 10), ("s_before_pv", 200), ("no_v_landing", 20)])
 def test_bf16_protocol_mistakes_are_caught(plant, least):
     """Releasing a K slot before its products are issued lets the producer overwrite
     it under a queued product; issuing S_t(j+1) before PV_t(j) overwrites P_t(j); a PV
