@@ -185,15 +185,19 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
 
     // The plan reads caller inputs no kernel of this library writes (lengths,
     // tables, group hints) and works in shared memory up to its scan; only its
-    // global writes (header, work list, partition counts, zero rows) must wait for
-    // the previous kernel on the stream, whose predecessors may still read this
-    // workspace and output.  So without prefix groups the wait comes after the
-    // scan, and the plan's work overlaps that kernel (the step's KV write).  The
-    // grouped plan claims members in the workspace itself: it waits first.  Either
-    // way the wait comes before the plan ends, so the decode that waits for the
-    // plan also finds the KV write done.
+    // global writes of the header, work list, partition counts and zero rows must
+    // wait for the previous kernel on the stream, whose predecessors may still read
+    // this workspace and output.  So the wait comes after the scan, and the plan's
+    // work overlaps that kernel (the step's KV write).  The grouped plan's member
+    // claims and subgroup lists (seq_sub, seq_k, sub_info, sub_members) are written
+    // before the wait: the only kernels of this library that let a dependent start
+    // early (they signal it right after their own wait) are the KV write, the block
+    // copies, the prefill and the decode, and a decode that may still run then is one
+    // without prefix groups (a grouped call always ends with the merge, which does
+    // not signal early), which never reads those lists; the merge reads only the
+    // partition counts and partials.  The wait comes before the plan ends, so the
+    // decode that waits for the plan also finds the KV write done.
     pdl_trigger();
-    if (grouped) pdl_wait();
 
     // 0. shared-prefix subgroups: sequence s then owns blocks [seq_k[s], B) and
     //    its subgroup computes blocks [0, seq_k[s]) once for all its members
@@ -269,7 +273,7 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
         }
         if (tid == 0) total_items = running;
     }
-    if (!grouped) pdl_wait();
+    pdl_wait();
     __syncthreads();
 
     // 4. global writes: header, partitions per sequence (shared ones first), zero
