@@ -195,6 +195,18 @@ def test_empty_and_single_token_and_maximum():
     assert np.array_equal(got, np.broadcast_to(v_row[:, None, :], got.shape))
 
 
+def test_million_token_context_every_element():
+    """A context of 2^20 tokens (65,536 blocks, 4 GiB of K/V in the pool) beside a
+    5-token and a 70,001-token one: automatic partitions, then 64-token partitions
+    (16,384 partials merged per row of the long context); every element against
+    the oracle."""
+    w = W.scaled(W.WORKLOADS["gqa70b"], num_seqs=3)
+    case = DecodeCase(w, lens=np.array([1 << 20, 5, 70001], np.int32))
+    _run(case, 0)
+    _run(case, 64)
+    assert int(case.g_err.item()) == 0
+
+
 def test_maximum_table_width_is_respected():
     """A context that uses every table entry (len == max_blocks * 16)."""
     w = W.scaled(W.WORKLOADS["mha13b"], num_seqs=3, num_heads=4, num_kv_heads=4)
