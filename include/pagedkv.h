@@ -285,8 +285,9 @@ int pkv_paged_attention_decode_shared(void* out, const void* q, int q_dtype,
  * max_blocks_per_seq <= 0, num_heads not a multiple of num_kv_heads, a null
  * pointer, a pointer not 16-byte (out, q, pools) or 4-byte (int32 arrays)
  * aligned, or a non-finite k_scale / v_scale with an FP8 cache;
- * PKV_EUNSUPPORTED for another dtype, head_dim or block_size, or more than
- * 65,535 sequences or heads.  No sequences or no queries: PKV_OK, nothing runs.
+ * PKV_EUNSUPPORTED for another dtype, head_dim or block_size, more than
+ * 65,535 sequences or heads, or a max_query_len above 65,535 x 256 tokens.
+ * No sequences or no queries: PKV_OK, nothing runs.
  * Device-data errors (a table entry out of range among the blocks a sequence
  * reads: its tokens are left out; nq_s > context_lens[s] or a context longer
  * than the table: the sequence's rows are zeroed) are counted into err_count.
