@@ -396,7 +396,7 @@ int pkv_paged_attention_prefill(void* out, const void* q, int q_dtype, const voi
     if (q_dtype != PKV_BF16 || (cache_dtype != PKV_BF16 && !fp8) || head_dim != 128) return PKV_EUNSUPPORTED;
     if (fp8 && !(std::isfinite(k_scale) && std::isfinite(v_scale))) return PKV_EINVAL;
     if (num_seqs == 0 || max_query_len == 0 || total_query_tokens == 0) return PKV_OK;
-    // grid (heads, sequences, 256-row query tiles): y and z are limited to 65535
+    // grid (heads, 256-row query tiles, sequences): y and z are limited to 65535
     if (num_seqs > 65535 || num_heads > 65535 || (max_query_len + 255) / 256 > 65535) return PKV_EUNSUPPORTED;
     if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens || !query_start) return PKV_EINVAL;
     if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) ||

@@ -289,11 +289,11 @@ __global__ void __launch_bounds__(448, 1)
     constexpr int kConvWarps = kTcBlocks;
     constexpr uint32_t kFull = 0xffffffffu;
 
-    // grid (head, sequence, 256-row tile): tiles are the slowest dimension, the last
-    // rows of the prompts (the most KV tiles) first, so that the CTAs are handed to
-    // the SMs roughly longest first and the launch ends with short ones
-    const int h = blockIdx.x, s = blockIdx.y, kvh = h / p.group;
-    const int tile = gridDim.z - 1 - blockIdx.z;
+    // grid (head, 256-row tile, sequence): a sequence's CTAs run together (its K/V
+    // stays in L2 for all its tiles and heads), its last rows (the most KV tiles)
+    // first, so that each sequence's CTAs reach the SMs longest first and end short
+    const int h = blockIdx.x, s = blockIdx.z, kvh = h / p.group;
+    const int tile = gridDim.y - 1 - blockIdx.y;
     if (threadIdx.x == 0) {
         for (int i = 0; i < kTcStages; ++i) {
             mbar_init(kv_full + 8 * i, kConvWarps);
@@ -814,11 +814,11 @@ __global__ void __launch_bounds__(320, 1)
     constexpr int kProducer = 8, kMma = 9;
     constexpr uint32_t kFull = 0xffffffffu;
 
-    // grid (head, sequence, 256-row tile): tiles are the slowest dimension, the last
-    // rows of the prompts (the most KV tiles) first, so that the CTAs are handed to
-    // the SMs roughly longest first and the launch ends with short ones
-    const int h = blockIdx.x, s = blockIdx.y, kvh = h / p.group;
-    const int tile = gridDim.z - 1 - blockIdx.z;
+    // grid (head, 256-row tile, sequence): a sequence's CTAs run together (its K/V
+    // stays in L2 for all its tiles and heads), its last rows (the most KV tiles)
+    // first, so that each sequence's CTAs reach the SMs longest first and end short
+    const int h = blockIdx.x, s = blockIdx.z, kvh = h / p.group;
+    const int tile = gridDim.y - 1 - blockIdx.y;
     if (threadIdx.x == 0) {
         for (int i = 0; i < kWKStages; ++i) {
             mbar_init(k_full + 8 * i, 1);
@@ -1188,7 +1188,7 @@ __global__ void __launch_bounds__(320, 1)
 cudaError_t launch_prefill_tc(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                               const PrefillParams& p, bool fp8, int max_query_len, cudaStream_t stream) {
     const int tiles = (max_query_len + kTcQT * kTcRows - 1) / (kTcQT * kTcRows);
-    const dim3 grid(p.num_heads, p.num_seqs, tiles);
+    const dim3 grid(p.num_heads, tiles, p.num_seqs);
     if (fp8) {
         const int smem = kTcSmemFp8 + 1024;
         cudaError_t e = cudaFuncSetAttribute(prefill_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

@@ -188,8 +188,8 @@ def test_prefill_validation(L):
     assert _prefill(L, d=64) == L.PKV_EUNSUPPORTED
     assert _prefill(L, cdt=L.PKV_FP8_E4M3, ks=float("nan")) == L.PKV_EINVAL
     assert _prefill(L, cdt=L.PKV_FP8_E4M3, vs=float("inf")) == L.PKV_EINVAL
-    assert _prefill(L, S=70000) == L.PKV_EUNSUPPORTED       # grid y limit
-    assert _prefill(L, mq=65535 * 256 + 1, T=65535 * 256 + 1) == L.PKV_EUNSUPPORTED   # grid z: 256-row tiles
+    assert _prefill(L, S=70000) == L.PKV_EUNSUPPORTED       # grid z limit
+    assert _prefill(L, mq=65535 * 256 + 1, T=65535 * 256 + 1) == L.PKV_EUNSUPPORTED   # grid y: 256-row tiles
     assert _prefill(L, hq=70000, hkv=70000) == L.PKV_EUNSUPPORTED
     assert _prefill(L, out=None) == L.PKV_EINVAL
     assert _prefill(L, qs=None) == L.PKV_EINVAL
