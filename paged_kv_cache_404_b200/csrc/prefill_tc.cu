@@ -24,8 +24,9 @@
 //
 // bf16 cache (prefill_bf16_kernel, ten warps): 128-key tiles, so that the score
 // products are M = N = 128, K = 128 (full tensor-core rate; N = 64 products read
-// their operands from shared memory faster than it delivers them), K in a 3-stage
-// and V in a 2-stage ring (224 KB with the Q tiles), one score buffer per Q tile.
+// their operands from shared memory faster than it delivers them), K and V in 2-stage
+// rings apart (192 KB with the Q tiles; 3 stages of either measured slower), one score
+// buffer per Q tile.
 // Per KV tile j the issuer runs PV_0(j), S_0(j+1), PV_1(j), S_1(j+1): while one Q
 // tile's softmax runs, the tensor core does the other Q tile's products.
 //
@@ -162,11 +163,11 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 constexpr int kWKeys = 128;                        // keys per KV tile (MMA N of S, K of PV)
 constexpr int kWChunk = kWKeys * 128;              // one 64-column chunk of a 128-row operand: 16 KB
 constexpr int kWTile = 2 * kWChunk;                // K (or V) tile: 128 keys x 128 bf16
-constexpr int kWKStages = 3, kWVStages = 2;        // K ring, V ring
+constexpr int kWKStages = 2, kWVStages = 2;        // K ring, V ring
 constexpr int kWBlocks = kWKeys / kBlockSize;      // table blocks per KV tile
 constexpr int kWK = kTcQT * kTcQBytes;             // shared memory: Q tiles, then the K ring, then the V ring
 constexpr int kWV = kWK + kWKStages * kWTile;
-constexpr int kWSmem = kWV + kWVStages * kWTile;   // 224 KB
+constexpr int kWSmem = kWV + kWVStages * kWTile;   // 192 KB
 constexpr int kWSCol = 256;                        // TMEM: O_t at 128 t, S_t at 256 + 128 t (P_t over its first 64)
 static_assert(kWSmem + 1024 <= 227 * 1024, "shared memory");
 
@@ -779,7 +780,7 @@ __global__ void __launch_bounds__(448, 1)
 // Causal prompt pass over a bf16 cache with 128-key tiles.  One CTA per (sequence,
 // 256 query rows = two Q tiles of 128, query head); ten warps:
 //  - warp 8 (producer): TMA-loads the two Q tiles once, then per 128-key tile the K
-//    of 8 table blocks into a 3-stage ring and their V into a 2-stage ring (16-slot x
+//    of 8 table blocks into a 2-stage ring and their V into another (16-slot x
 //    1-head x 128-byte boxes, 128-byte swizzle), zeroing the V rows that hold no
 //    token of the context;
 //  - warp 9 (MMA): runs warp-uniformly, one elected lane issuing.  Per KV tile j and
@@ -800,7 +801,7 @@ __global__ void __launch_bounds__(320, 1)
     prefill_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
-    // k_full[3], k_empty[3], v_full[2], v_ready[2], v_empty[2], q_full, s_full[2], p_full[2], o_done[2]
+    // k_full[2], k_empty[2], v_full[2], v_ready[2], v_empty[2], q_full, s_full[2], p_full[2], o_done[2]
     __shared__ __align__(8) uint64_t bars[2 * kWKStages + 3 * kWVStages + 1 + 3 * kTcQT];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
