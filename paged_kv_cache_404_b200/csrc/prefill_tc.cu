@@ -8,7 +8,9 @@
 // holds).
 //
 // Two kernels, one per cache type; both take one CTA per (sequence, 256 query rows
-// = two Q tiles of 128, query head), hold O and the scores of both Q tiles in the
+// = two Q tiles of 128, query head), on a grid ordered (head, tile, sequence) so that
+// a sequence's CTAs run together and its last rows come first, hold O and the scores
+// of both Q tiles in the
 // 512 TMEM columns, and split the work between warps: a producer (TMA loads of Q
 // once and of K/V tiles through the block table, with the V rows that hold no token
 // zeroed in shared memory, so that a zero probability never meets a NaN there), an
@@ -23,7 +25,7 @@
 // overwrite the P it reads, and the commit that follows it also covers PV_t(j).
 //
 // bf16 cache (prefill_bf16_kernel, ten warps): 128-key tiles, so that the score
-// products are M = N = 128, K = 128 (full tensor-core rate; N = 64 products read
+// products are M = N = 128, K = 128 (full tensor-core rate; N = 64 products need
 // their operands from shared memory faster than it delivers them), K and V in 2-stage
 // rings apart (192 KB with the Q tiles; 3 stages of either measured slower), one score
 // buffer per Q tile.
