@@ -125,11 +125,41 @@ DECODE_SOURCES = ("decode_tc.cu", "pkv_common.cuh", "decode_plan.cu", "api.cu")
 PREFILL_SOURCES = ("prefill_tc.cu", "pkv_common.cuh", "api.cu")
 
 
-def kernel_source_hash(files=DECODE_SOURCES):
+def code_of(text: str) -> str:
+    """C/C++/CUDA source without its comments, trailing spaces and blank lines: what a
+    change of comments leaves the same (the kernels compile to the same code)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        if text.startswith("//", i):
+            i = text.find("\n", i)
+            i = n if i < 0 else i
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        elif text[i] == '"':                                  # a string literal (inline PTX)
+            j = i + 1
+            while j < n and text[j] != '"':
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        else:
+            out.append(text[i])
+            i += 1
+    lines = (line.rstrip() for line in "".join(out).splitlines())
+    return "\n".join(line for line in lines if line)
+
+
+def kernel_source_hash(files=DECODE_SOURCES, read=None):
+    """Hash of the kernel sources' code (comments left out), keying the committed ncu
+    traffic of a workload to the code it was captured from."""
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "paged_kv_cache_404_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        if read is None:
+            with open(os.path.join(ROOT, "paged_kv_cache_404_b200", "csrc", f), encoding="utf-8") as fh:
+                text = fh.read()
+        else:
+            text = read(f)
+        h.update(code_of(text).encode("utf-8"))
     return h.hexdigest()[:16]
 
 

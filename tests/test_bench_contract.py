@@ -86,3 +86,16 @@ def test_unique_kv_bytes_counts_a_shared_block_once():
     assert bench.unique_kv_bytes(tables, np.array([40, 35]), 10) == (16 + 16 + 8 + 3) * 10
     assert bench.unique_kv_bytes(tables, np.array([20, 40]), 1) == 16 + 16 + 8      # block 6: 4 vs 16 tokens
     assert bench.unique_kv_bytes(tables, np.array([0, 0]), 1) == 0
+
+
+def test_source_hash_ignores_comments_only():
+    """The committed ncu traffic is keyed to the kernels' code: comments and blank
+    lines may change, code (inline PTX strings included) may not."""
+    import bench
+    base = 'int f(int a) {  // twice\n    return 2 * a;\n}\nasm("add.u32 %0; // in the string");\n'
+    same = '/* doubles */\nint f(int a) {\n\n    return 2 * a;   // comment\n}\nasm("add.u32 %0; // in the string");\n'
+    other = 'int f(int a) {\n    return 3 * a;\n}\nasm("add.u32 %0; // in the string");\n'
+    ptx = 'int f(int a) {\n    return 2 * a;\n}\nasm("add.u32 %0; // changed");\n'
+    h = lambda text: bench.kernel_source_hash(("x.cu",), read=lambda f: text)
+    assert h(base) == h(same)
+    assert h(base) != h(other) and h(base) != h(ptx)
