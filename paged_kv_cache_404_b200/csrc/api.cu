@@ -22,7 +22,7 @@ cudaError_t launch_decode_tc(const CUtensorMap& tmK, const CUtensorMap& tmV, con
 cudaError_t launch_decode_f32(const DecodeParams& p, int num_sms, cudaStream_t stream);
 int decode_tc_warps(bool fp8, int head_dim, bool grouped);
 bool decode_tc_groupable(bool fp8, int head_dim, int group);
-cudaError_t launch_decode_merge(const DecodeParams& p, int out_dtype, cudaStream_t stream);
+cudaError_t launch_decode_merge(const DecodeParams& p, int out_dtype, int num_sms, cudaStream_t stream);
 cudaError_t launch_prefill_tc(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                               const PrefillParams& p, bool fp8, int max_query_len, cudaStream_t stream);
 }  // namespace pkv
@@ -371,7 +371,7 @@ int decode_impl(void* out, const void* q, int q_dtype, const void* k_pool, const
     // shorter than the longest context, or if a sequence's shared and own
     // blocks are cut apart
     if (grouped || min_p < max_context_len) {
-        e = launch_decode_merge(p, out_dtype, st);
+        e = launch_decode_merge(p, out_dtype, num_sms, st);
         if (e != cudaSuccess) return PKV_ECUDA;
     }
     return PKV_OK;

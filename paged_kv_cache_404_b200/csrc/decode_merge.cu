@@ -10,20 +10,23 @@
 //
 // One warp per (sequence, query head).  Lanes are 4 partition groups x 8
 // head_dim slices (16 elements each): group r takes partitions r, r+4, ...;
-// the first four partitions are loaded in one round (weights and outputs
-// together, before the max is known), so up to four partitions cost two
+// the first 4 x KR partitions are loaded in one round (weights and outputs
+// together, before the max is known), so up to 4 x KR partitions cost two
 // dependent rounds of loads (the partition count, then the partials); the four
-// groups are combined with shuffles at the end.  Deterministic: the order of additions
-// depends only on the partition count.
+// groups are combined with shuffles at the end.  KR = 4 for a merge of up to 32
+// warps per SM, KR = 2 above (measured on B200, 148 SMs: KR = 4 took 3-6 us off the
+// calls with 2,048 and 4,096 merge warps; at 6,144 and 16,384 warps KR = 2 was as
+// fast or faster, where more resident warps hide the latency better than more
+// loads per warp).  Deterministic: the order of additions depends only on the
+// partition count.
 #include "pkv_common.cuh"
 
 namespace pkv {
 
-template <int D, typename OutT>
+template <int D, int KR, typename OutT>
 __global__ void __launch_bounds__(256) decode_merge_kernel(DecodeParams p) {
     pdl_wait();
     constexpr int SL = D / 8;   // head_dim elements per lane
-    constexpr int KR = 1;       // partitions per lane group loaded in the first round (4 per warp)
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (warp >= p.num_seqs * p.num_heads) return;
@@ -116,14 +119,23 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(DecodeParams p) {
     }
 }
 
-cudaError_t launch_decode_merge(const DecodeParams& p, int out_dtype, cudaStream_t stream) {
-    const int warps = p.num_seqs * p.num_heads;
+template <int D, int KR>
+cudaError_t launch_merge_kr(const DecodeParams& p, int out_dtype, unsigned grid, cudaStream_t stream) {
+    return out_dtype == 0 ? launch_pdl(decode_merge_kernel<D, KR, float>, dim3(grid), dim3(256), 0, stream, p)
+                          : launch_pdl(decode_merge_kernel<D, KR, __nv_bfloat16>, dim3(grid), dim3(256), 0, stream, p);
+}
+
+// Largest merge, in warps per SM, that takes the KR = 4 form.
+constexpr int kMergeWarpsPerSmKr4 = 32;
+
+cudaError_t launch_decode_merge(const DecodeParams& p, int out_dtype, int num_sms, cudaStream_t stream) {
+    const long long warps = (long long)p.num_seqs * p.num_heads;
     const unsigned grid = (unsigned)((warps * 32 + 255) / 256);
+    const bool kr4 = warps <= (long long)num_sms * kMergeWarpsPerSmKr4;
     if (p.head_dim == 128)
-        return out_dtype == 0 ? launch_pdl(decode_merge_kernel<128, float>, dim3(grid), dim3(256), 0, stream, p)
-                              : launch_pdl(decode_merge_kernel<128, __nv_bfloat16>, dim3(grid), dim3(256), 0, stream, p);
-    return out_dtype == 0 ? launch_pdl(decode_merge_kernel<64, float>, dim3(grid), dim3(256), 0, stream, p)
-                          : launch_pdl(decode_merge_kernel<64, __nv_bfloat16>, dim3(grid), dim3(256), 0, stream, p);
+        return kr4 ? launch_merge_kr<128, 4>(p, out_dtype, grid, stream)
+                   : launch_merge_kr<128, 2>(p, out_dtype, grid, stream);
+    return kr4 ? launch_merge_kr<64, 4>(p, out_dtype, grid, stream) : launch_merge_kr<64, 2>(p, out_dtype, grid, stream);
 }
 
 }  // namespace pkv

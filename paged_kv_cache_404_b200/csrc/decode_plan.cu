@@ -26,39 +26,22 @@ constexpr int kMaxCandidates = 12;
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 __device__ __forceinline__ int bucket_of(int nblk, int nb_top, int nbuckets) {
-    // bucket 0 = one block ... nbuckets-1 = a largest partition
+    // bucket 0 = one block ... nbuckets-1 = a largest partition: (nblk - 1) * nbuckets
+    // / nb_top, in 32 bits while the product fits (nbuckets <= 1024, nblk <= nb_top)
+    if (nbuckets == nb_top) return nblk - 1;
+    if (nb_top < (1 << 21)) return (int)((unsigned)(nblk - 1) * (unsigned)nbuckets / (unsigned)nb_top);
     return (int)(((long long)(nblk - 1) * nbuckets) / nb_top);
 }
 
-// Partitions of one sequence of B blocks, in order along the context.
+// Partitions of one sequence of B blocks, in order along the context (the pieces):
 //  uniform (user-fixed size): pieces of nb blocks, the last one shorter;
 //  geometric (automatic): whole pieces of nb blocks, then the remaining chunk T
 //  (1..nb blocks) halved while it exceeds 2*mb: T/2, T/4, ..., then the rest.
 //  Each piece is >= mb blocks unless the sequence is shorter, so a sequence of
 //  B blocks has at most ceil(B / mb) pieces; under longest-first scheduling the
 //  last units handed out are the small ones, which evens out the finish times.
-// Calls emit(first_block, blocks) for each piece and returns the count.
-template <typename F>
-__device__ __forceinline__ int for_each_piece(int B, int nb, int mb, bool geometric, F&& emit) {
-    if (B <= 0) return 0;
-    int count = 0, at = 0;
-    if (!geometric) {
-        for (; at < B; at += nb, ++count) emit(at, min(nb, B - at));
-        return count;
-    }
-    const int body = (B - 1) / nb;  // whole pieces before the last chunk
-    for (int i = 0; i < body; ++i, at += nb, ++count) emit(at, nb);
-    int T = B - at;
-    while (T > 2 * mb) {
-        const int piece = T / 2;
-        emit(at, piece);
-        at += piece;
-        T -= piece;
-        ++count;
-    }
-    emit(at, T);
-    return count + 1;
-}
+// count_pieces, hist_pieces and scatter_pieces (below) count, histogram and write
+// these pieces.
 
 // Shared-prefix groups.  Sequences that start with the same physical blocks
 // (parallel samples of one prompt, requests with a common system prompt: the
@@ -154,30 +137,87 @@ __device__ void build_groups(const DecodeParams& p, int* n_subs, int* n_members)
     __syncthreads();
 }
 
-// Number of pieces for_each_piece cuts B blocks into (closed form of its loop).
+// Halvings of a last chunk of T blocks (T becomes ceil(T / 2) while T > 2 mb):
+// ceil(T / 2^k) <= 2 mb first holds at k = ceil(log2(ceil(T / 2 mb))).
+__device__ __forceinline__ int halvings(int T, int mb) {
+    if (T <= 2 * mb) return 0;
+    const unsigned q = ((unsigned)T + 2u * mb - 1u) / (2u * mb);  // >= 2
+    return 32 - __clz((int)(q - 1u));
+}
+
+// The three helpers below are out of line: each phase of the one-CTA plan runs its
+// code once per launch, so its time follows the instructions it fetches more than
+// their arithmetic, and one copy serves every call site.
+//
+// Number of pieces B blocks are cut into (closed form).
 __device__ __noinline__ int count_pieces(int B, int nb, int mb, bool geometric) {
     if (B <= 0) return 0;
-    if (!geometric) return (B + nb - 1) / nb;
+    if (!geometric) return (B - 1) / nb + 1;
     const int body = (B - 1) / nb;
-    int T = B - body * nb, n = body + 1;
-    while (T > 2 * mb) {
-        T -= T / 2;
-        ++n;
-    }
-    return n;
+    return body + 1 + halvings(B - body * nb, mb);
+}
+
+// Adds the sizes of the pieces of B blocks to the histogram, the whole pieces
+// (all in the top bucket) with one atomic.
+__device__ __noinline__ void hist_pieces(int* hist, int B, int nb, int mb, bool geometric, int nbuckets) {
+    if (B <= 0) return;
+    const int whole = geometric ? (B - 1) / nb : B / nb;
+    if (whole > 0) atomicAdd(&hist[nbuckets - 1], whole);
+    int T = B - whole * nb;
+    if (geometric)
+        while (T > 2 * mb) {
+            const int piece = T / 2;
+            atomicAdd(&hist[bucket_of(piece, nb, nbuckets)], 1);
+            T -= piece;
+        }
+    if (T > 0) atomicAdd(&hist[bucket_of(T, nb, nbuckets)], 1);
+}
+
+// Writes the work items of the pieces of B blocks (item.x = code, item.y =
+// partition part0, part0 + 1, ... along the context, item.z = first block + k0,
+// item.w = blocks), each at the place its bucket's counter in the exclusive-scanned
+// histogram gives.  (One atomic per piece measured faster here than one per
+// sequence for its whole pieces followed by their stores.)
+__device__ __noinline__ void scatter_pieces(int4* items, int* hist, int code, int part0, int k0, int B, int nb,
+                                               int mb, bool geometric, int nbuckets) {
+    if (B <= 0) return;
+    const int whole = geometric ? (B - 1) / nb : B / nb;
+    int part = part0, at = 0;
+    for (int i = 0; i < whole; ++i, at += nb)
+        items[atomicAdd(&hist[nbuckets - 1], 1)] = make_int4(code, part++, k0 + at, nb);
+    int T = B - at;
+    if (geometric)
+        while (T > 2 * mb) {
+            const int piece = T / 2;
+            items[atomicAdd(&hist[bucket_of(piece, nb, nbuckets)], 1)] = make_int4(code, part++, k0 + at, piece);
+            at += piece;
+            T -= piece;
+        }
+    if (T > 0) items[atomicAdd(&hist[bucket_of(T, nb, nbuckets)], 1)] = make_int4(code, part, k0 + at, T);
 }
 
 constexpr int kSmemSeqs = 4096;  // per-sequence block counts kept in shared memory up to this many
+
+// Block counts of sequences and subgroups past the shared-memory copies, read from
+// global memory.  Out of line: the loads of the same addresses in the phase that
+// fills the copies would otherwise let the compiler evaluate these global reads
+// in place of every shared-memory read as well (an L2 round trip per use).
+__device__ __noinline__ int own_blocks_global(const int32_t* lens, const int* seq_k, int cap, int s) {
+    const int L = min(max(lens[s], 0), cap);
+    return (L + kBlockSize - 1) / kBlockSize - (seq_k != nullptr ? seq_k[s] : 0);
+}
+__device__ __noinline__ int sub_blocks_global(const int4* sub_info, int q) { return sub_info[q].z; }
 
 __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams p, int fixed_partition, int min_partition,
                                                                    int num_candidates, int target_units,
                                                                    int zero_out_dtype) {
     __shared__ int hist[kMaxBuckets];
     __shared__ int own_blocks[kSmemSeqs];  // blocks of sequence s outside its shared prefix
-    __shared__ unsigned long long units_of[kMaxCandidates];
+    __shared__ int sub_blocks[kSmemSeqs];  // blocks subgroup q computes for its members
+    __shared__ unsigned long long units_of[kMaxCandidates][32];  // per candidate and warp
     __shared__ int chosen, total_items;
     __shared__ int n_subs, n_members;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // automatic partitioning ends each context with geometrically shrinking pieces
     const bool geometric = fixed_partition == 0;
     const int mb = min_partition / kBlockSize;
@@ -202,7 +242,6 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
     // 0. shared-prefix subgroups: sequence s then owns blocks [seq_k[s], B) and
     //    its subgroup computes blocks [0, seq_k[s]) once for all its members
     if (tid == 0) n_subs = n_members = 0;
-    if (tid < kMaxCandidates) units_of[tid] = 0;
     for (int b = tid; b < kMaxBuckets; b += kPlanThreads) hist[b] = 0;
     __syncthreads();
     if (grouped) build_groups(p, &n_subs, &n_members);
@@ -213,33 +252,43 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
     };
     for (int s = tid; s < p.num_seqs && s < kSmemSeqs; s += kPlanThreads) own_blocks[s] = own_of(s, true);
     for (int s = kSmemSeqs + tid; s < p.num_seqs; s += kPlanThreads) own_of(s, true);
+    for (int q = tid; q < num_subs && q < kSmemSeqs; q += kPlanThreads) sub_blocks[q] = p.sub_info[q].z;
     __syncthreads();
-    auto own = [&](int s) { return s < kSmemSeqs ? own_blocks[s] : own_of(s, false); };
+    const int len_cap = min(p.max_blocks_per_seq * kBlockSize, p.max_context_len);
+    auto own = [&](int s) {
+        return s < kSmemSeqs ? own_blocks[s] : own_blocks_global(p.context_lens, grouped ? p.seq_k : nullptr, len_cap, s);
+    };
+    auto sub = [&](int q) { return q < kSmemSeqs ? sub_blocks[q] : sub_blocks_global(p.sub_info, q); };
 
     // 1. largest partition: the largest candidate min_partition << c whose work
     //    list still has target_units units
     if (fixed_partition > 0) {
         if (tid == 0) chosen = fixed_partition;
     } else {
+        // per candidate, each warp's count in its own slot (no atomics), summed by one warp
 #pragma unroll 1
         for (int c = 0; c < num_candidates; ++c) {
             const int nb = (min_partition << c) / kBlockSize;
             unsigned long long v = 0;
             for (int s = tid; s < p.num_seqs; s += kPlanThreads) v += count_pieces(own(s), nb, mb, geometric);
-            for (int q = tid; q < num_subs; q += kPlanThreads) v += count_pieces(p.sub_info[q].z, nb, mb, geometric);
+            for (int q = tid; q < num_subs; q += kPlanThreads) v += count_pieces(sub(q), nb, mb, geometric);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if ((tid & 31) == 0 && v) atomicAdd(&units_of[c], v);
+            if (lane == 0) units_of[c][warp] = v;
         }
         __syncthreads();
-        if (tid == 0) {
+        if (warp == 0) {
             int P = min_partition;
-            for (int c = num_candidates - 1; c >= 0; --c)
-                if (units_of[c] * (unsigned long long)p.num_kv_heads >= (unsigned long long)target_units) {
+            for (int c = num_candidates - 1; c >= 0; --c) {
+                unsigned long long v = lane < kPlanThreads / 32 ? units_of[c][lane] : 0ull;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                if (v * (unsigned long long)p.num_kv_heads >= (unsigned long long)target_units) {
                     P = min_partition << c;
                     break;
                 }
-            chosen = P;
+            }
+            if (lane == 0) chosen = P;
         }
     }
     __syncthreads();
@@ -248,12 +297,8 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
     const int nbuckets = nb_top < kMaxBuckets ? nb_top : kMaxBuckets;
 
     // 2. histogram of item sizes
-    for (int s = tid; s < p.num_seqs; s += kPlanThreads)
-        for_each_piece(own(s), nb_top, mb, geometric,
-                       [&](int, int n) { atomicAdd(&hist[bucket_of(n, nb_top, nbuckets)], 1); });
-    for (int q = tid; q < num_subs; q += kPlanThreads)
-        for_each_piece(p.sub_info[q].z, nb_top, mb, geometric,
-                       [&](int, int n) { atomicAdd(&hist[bucket_of(n, nb_top, nbuckets)], 1); });
+    for (int s = tid; s < p.num_seqs; s += kPlanThreads) hist_pieces(hist, own(s), nb_top, mb, geometric, nbuckets);
+    for (int q = tid; q < num_subs; q += kPlanThreads) hist_pieces(hist, sub(q), nb_top, mb, geometric, nbuckets);
     __syncthreads();
 
     // 3. exclusive scan, largest bucket first (serial over <= 1024 buckets by one warp)
@@ -292,7 +337,7 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
     for (int s = tid; s < p.num_seqs; s += kPlanThreads) {
         const int k = grouped ? p.seq_k[s] : 0;
         const int B = own(s);
-        int part = count_pieces(k, nb_top, mb, geometric);
+        const int part = count_pieces(k, nb_top, mb, geometric);
         p.nparts[s] = part + count_pieces(B, nb_top, mb, geometric);
         if (B + k == 0) {
             // an empty context produces a zero output row (nothing else writes it)
@@ -305,19 +350,11 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
                     static_cast<__nv_bfloat16*>(p.out)[row + e] = __float2bfloat16(0.f);
             }
         }
-        for_each_piece(B, nb_top, mb, geometric, [&](int first, int n) {
-            const int pos = atomicAdd(&hist[bucket_of(n, nb_top, nbuckets)], 1);
-            p.items[pos] = make_int4(s, part++, k + first, n);
-        });
+        scatter_pieces(p.items, hist, s, part, k, B, nb_top, mb, geometric, nbuckets);
     }
     // subgroup items carry -(subgroup + 1) in place of the sequence
-    for (int q = tid; q < num_subs; q += kPlanThreads) {
-        int part = 0;
-        for_each_piece(p.sub_info[q].z, nb_top, mb, geometric, [&](int first, int n) {
-            const int pos = atomicAdd(&hist[bucket_of(n, nb_top, nbuckets)], 1);
-            p.items[pos] = make_int4(-(q + 1), part++, first, n);
-        });
-    }
+    for (int q = tid; q < num_subs; q += kPlanThreads)
+        scatter_pieces(p.items, hist, -(q + 1), 0, 0, sub(q), nb_top, mb, geometric, nbuckets);
 }
 
 cudaError_t launch_decode_plan(const DecodeParams& p, int fixed_partition, int min_partition, int num_candidates,

@@ -106,6 +106,22 @@ def test_small_cases_every_element(name, P):
     _run(DecodeCase(w, lens=lens), P)
 
 
+@pytest.mark.parametrize("P", [16, 48])
+def test_merge_of_few_and_many_rows_past_its_first_round(P):
+    """The merge loads 16 partitions per warp in its first round when it has at most
+    32 (sequence, query head) rows per SM, 8 when it has more; both forms here, with
+    more partitions than that first round (16- and 48-token pieces of ragged contexts
+    up to 700 tokens), every element against the oracle."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    for rows in (sms * 8, sms * 40):
+        S = -(-rows // 64)
+        w = W.scaled(W.WORKLOADS["gqa70b"], num_seqs=S)
+        rng = np.random.default_rng(S * 1000 + P)
+        lens = rng.choice(RAGGED, size=S).astype(np.int32)
+        lens[0] = 700
+        _run(DecodeCase(w, lens=lens), P)
+
+
 @pytest.mark.parametrize("G,D", [(1, 64), (2, 128), (4, 128), (8, 64), (8, 128), (16, 128), (12, 128), (3, 64)])
 def test_group_sizes_and_head_dims(G, D):
     w = W.scaled(W.WORKLOADS["gqa70b"], num_heads=2 * G, num_kv_heads=2, head_dim=D, num_seqs=4)
