@@ -122,6 +122,18 @@ def test_merge_of_few_and_many_rows_past_its_first_round(P):
         _run(DecodeCase(w, lens=lens), P)
 
 
+@pytest.mark.parametrize("P", [0, 16])
+def test_batch_past_the_plans_shared_memory_copies(P):
+    """4,500 sequences: the plan keeps the block counts of the first 4,096 in shared
+    memory and reads the others' from global memory; every element against the
+    oracle (contexts of 1-200 tokens, one KV head for eight query heads)."""
+    w = W.scaled(W.WORKLOADS["gqa70b"], num_seqs=4500, num_heads=8, num_kv_heads=1)
+    rng = np.random.default_rng(4500 + P)
+    lens = rng.integers(1, 201, size=4500).astype(np.int32)
+    lens[-1] = 200
+    _run(DecodeCase(w, lens=lens), P)
+
+
 @pytest.mark.parametrize("G,D", [(1, 64), (2, 128), (4, 128), (8, 64), (8, 128), (16, 128), (12, 128), (3, 64)])
 def test_group_sizes_and_head_dims(G, D):
     w = W.scaled(W.WORKLOADS["gqa70b"], num_heads=2 * G, num_kv_heads=2, head_dim=D, num_seqs=4)

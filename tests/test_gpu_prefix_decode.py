@@ -146,6 +146,38 @@ def test_gqa8_group_of_three_splits_into_subgroups(extra):
     assert_close(out_to_f64(out), ref, "bf16", "gqa8 subgroups %s" % extra)
 
 
+def test_more_subgroups_than_the_plans_shared_memory_copies():
+    """4,200 prompts of 17-40 tokens, each forked once: 4,200 two-member groups
+    sharing their full blocks (one or two; G = 8: two members per subgroup), more
+    subgroups than the plan keeps in shared memory (4,096); every element against
+    the oracle."""
+    import paged_kv_cache_404_b200 as pkv
+    R = 4200
+    w = W.scaled(W.WORKLOADS["gqa70b"], num_seqs=2 * R, num_heads=16, num_kv_heads=2)
+    NB = 3 * R + 16
+    rng = np.random.default_rng(4200)
+    bm = pkv.BlockManager(NB, 16, free_order=rng.permutation(NB))
+    ids = []
+    for r in range(R):
+        parent = bm.alloc_seq(int(rng.integers(17, 41)))
+        ids += [parent, bm.fork(parent)]
+    lens = np.array([bm.seq_len(s) for s in ids], dtype=np.int32)
+    tabs, _ = bm.tables(ids, 3, pad=-1)
+    offs, mem, sh = bm.prefix_groups(ids)
+    assert len(offs) == R + 1 and all(int(x) in (1, 2) for x in sh)
+    kp, vp, _, _ = W.random_pools(w, NB, "cuda")
+    q = W.queries(w, 2 * R, "cuda")
+    g_t, g_l = torch.from_numpy(tabs).cuda(), torch.from_numpy(lens).cuda()
+    out, err, ws = _grouped(q, kp, vp, g_t, g_l, w.scale, int(lens.max()), offs, mem, sh)
+    assert err == 0
+    _, nsubs, nmem = _hdr(ws)
+    assert (nsubs, nmem) == (R, 2 * R)
+    ref, bad = oracle.paged_attention_decode(to_np_bits(q), oracle.BF16, to_np_bits(kp), to_np_bits(vp),
+                                             oracle.BF16, tabs, lens, w.scale)
+    assert bad == 0
+    assert_close(out_to_f64(out), ref, "bf16", "4,200 subgroups")
+
+
 def test_fp8_cache_ignores_hints_and_equals_plain_decode():
     import paged_kv_cache_404_b200 as pkv
     w = W.scaled(W.WORKLOADS["fp8_long"], num_seqs=3)
