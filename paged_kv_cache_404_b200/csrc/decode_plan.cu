@@ -19,6 +19,7 @@
 namespace pkv {
 
 constexpr int kPlanThreads = 1024;
+static_assert(kPlanThreads % 32 == 0 && kPlanThreads <= 1024, "one slot per warp in the candidate counts");
 constexpr int kMaxBuckets = 1024;
 constexpr int kMaxCandidates = 12;
 
@@ -199,9 +200,10 @@ __device__ __noinline__ void scatter_pieces(int4* items, int* hist, int code, in
 constexpr int kSmemSeqs = 4096;  // per-sequence block counts kept in shared memory up to this many
 
 // Block counts of sequences and subgroups past the shared-memory copies, read from
-// global memory.  Out of line: the loads of the same addresses in the phase that
-// fills the copies would otherwise let the compiler evaluate these global reads
-// in place of every shared-memory read as well (an L2 round trip per use).
+// global memory.  Out of line: inlined, the compiler (which has seen the same
+// addresses loaded in the phase that fills the copies) issues these global reads
+// unconditionally beside every shared-memory read and selects afterwards, an L2
+// round trip per use.
 __device__ __noinline__ int own_blocks_global(const int32_t* lens, const int* seq_k, int cap, int s) {
     const int L = min(max(lens[s], 0), cap);
     return (L + kBlockSize - 1) / kBlockSize - (seq_k != nullptr ? seq_k[s] : 0);
