@@ -18,8 +18,7 @@
 
 namespace pkv {
 
-constexpr int kPlanThreads = 1024;
-static_assert(kPlanThreads % 32 == 0 && kPlanThreads <= 1024, "one slot per warp in the candidate counts");
+constexpr int kPlanThreads = 1024;  // at most 32 warps: one slot per warp in the candidate counts
 constexpr int kMaxBuckets = 1024;
 constexpr int kMaxCandidates = 12;
 
