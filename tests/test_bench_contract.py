@@ -99,3 +99,13 @@ def test_source_hash_ignores_comments_only():
     h = lambda text: bench.kernel_source_hash(("x.cu",), read=lambda f: text)
     assert h(base) == h(same)
     assert h(base) != h(other) and h(base) != h(ptx)
+
+
+def test_every_traffic_entry_matches_the_current_kernels():
+    """Each workload's committed DRAM traffic was captured from the code that is in
+    the tree now (otherwise the bench line reports null traffic for it)."""
+    import bench
+    data = json.load(open(os.path.join(ROOT, "profiles", "ncu_traffic.json")))
+    for w in ("gqa70b", "mha13b", "fp8_long", "shared_prefix", "beam", "prefill70b", "prefill70b_fp8"):
+        assert w in data, w
+        assert bench.ncu_traffic(w) == data[w]["dram_bytes_per_launch"], "stale traffic entry: %s" % w
