@@ -24,7 +24,7 @@
 // thread's products in issue order, so a score product issued after PV_t(j) may
 // overwrite the P it reads, and the commit that follows it also covers PV_t(j).
 //
-// bf16 cache (prefill_bf16_kernel, ten warps): 128-key tiles, so that the score
+// bf16 cache (prefill_bf16_kernel, twelve warps): 128-key tiles, so that the score
 // products are M = N = 128, K = 128 (full tensor-core rate; N = 64 products need
 // their operands from shared memory faster than it delivers them), K and V in 2-stage
 // rings apart (192 KB with the Q tiles; 3 stages of either measured slower), one score
@@ -780,7 +780,11 @@ __global__ void __launch_bounds__(448, 1)
 }
 
 // Causal prompt pass over a bf16 cache with 128-key tiles.  One CTA per (sequence,
-// 256 query rows = two Q tiles of 128, query head); ten warps:
+// 256 query rows = two Q tiles of 128, query head); twelve warps, of which warps 10
+// and 11 only complete warpgroup 2 (warps 8-11), so that registers can move between
+// warpgroups: launched at 168 per thread (65,536 / 384), warpgroup 2 gives up to 80
+// and the softmax warpgroups take 200 (2 x 128 x 200 + 128 x 80 = 61,440 <= 384 x 168;
+// 200 registers hold a row's 128 scores and its P without spills, where 168 spilled):
 //  - warp 8 (producer): TMA-loads the two Q tiles once, then per 128-key tile the K
 //    of 8 table blocks into a 2-stage ring and their V into another (16-slot x
 //    1-head x 128-byte boxes, 128-byte swizzle), zeroing the V rows that hold no
@@ -799,7 +803,7 @@ __global__ void __launch_bounds__(448, 1)
 //    previous tile when the scores land, is then rescaled in TMEM), writes P as bf16
 //    pairs over the first 64 score columns, and finally normalises O and stores the
 //    row.
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     prefill_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -886,153 +890,158 @@ __global__ void __launch_bounds__(320, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
-
-    if (warp == kProducer) {
-        // ================= producer =================
-        if (lane == 0) {
-            mbar_arrive_expect_tx(q_full, kTcQT * kTcQBytes);
-            for (int t = 0; t < kTcQT; ++t) {
-                tma_load_3d(base + t * kTcQBytes, &tmQ, 0, h, qs0 + row0 + t * kTcRows, q_full);
-                tma_load_3d(base + t * kTcQBytes + kTcQChunk, &tmQ, 64, h, qs0 + row0 + t * kTcRows, q_full);
+    // registers move from warpgroup 2 (producer, issuer, two idle warps) to the two
+    // softmax warpgroups; each warpgroup's four warps run its setmaxnreg together
+    if (warp >= 8) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 80;");
+        if (warp == kProducer) {
+            // ================= producer =================
+            if (lane == 0) {
+                mbar_arrive_expect_tx(q_full, kTcQT * kTcQBytes);
+                for (int t = 0; t < kTcQT; ++t) {
+                    tma_load_3d(base + t * kTcQBytes, &tmQ, 0, h, qs0 + row0 + t * kTcRows, q_full);
+                    tma_load_3d(base + t * kTcQBytes + kTcQChunk, &tmQ, 64, h, qs0 + row0 + t * kTcRows, q_full);
+                }
             }
-        }
-        bool ok = true;
-        for (int j = 0; j < ntiles && !*abort_flag; ++j) {
-            // block ids of this tile: lanes 0..7; a block is loaded if it is in the table
-            // and its id is in range
-            const int jb = j * kWBlocks + (lane & (kWBlocks - 1));
-            int id = -1;
-            if (lane < kWBlocks && jb < nblk_seq) id = __ldg(tab + jb);
-            const bool load = lane < kWBlocks && jb < nblk_seq && id >= 0 && id < p.num_blocks;
-            if (lane < kWBlocks && jb < nblk_seq && !load && h == 0 && jb >= count_from && jb <= last_pos / kBlockSize)
+            bool ok = true;
+            for (int j = 0; j < ntiles && !*abort_flag; ++j) {
+                // block ids of this tile: lanes 0..7; a block is loaded if it is in the table
+                // and its id is in range
+                const int jb = j * kWBlocks + (lane & (kWBlocks - 1));
+                int id = -1;
+                if (lane < kWBlocks && jb < nblk_seq) id = __ldg(tab + jb);
+                const bool load = lane < kWBlocks && jb < nblk_seq && id >= 0 && id < p.num_blocks;
+                if (lane < kWBlocks && jb < nblk_seq && !load && h == 0 && jb >= count_from && jb <= last_pos / kBlockSize)
+                    count_error(p.err);
+                const unsigned loaded = __ballot_sync(kFull, load);
+                const int row = id * kBlockSize;
+                const uint32_t off = lane * kBlockSize * 128;
+                const uint32_t tx = __popc(loaded) * 2 * (kBlockSize * 128);
+                // K of this tile into its ring slot, once the products that read the slot's
+                // previous tile are done
+                const int ks = j % kWKStages, kr = j / kWKStages;
+                bool go = true;
+                if (lane == 0 && kr > 0) go = mbar_wait_bounded(k_empty + 8 * ks, (kr - 1) & 1);
+                if (!(ok = __shfl_sync(kFull, go, 0))) break;
+                const uint32_t kdst = base + kWK + ks * kWTile;
+                if (lane == 0) mbar_arrive_expect_tx(k_full + 8 * ks, tx);
+                __syncwarp();
+                if (load) {
+                    tma_load_3d(kdst + off, &tmK, 0, kvh, row, k_full + 8 * ks);
+                    tma_load_3d(kdst + kWChunk + off, &tmK, 64, kvh, row, k_full + 8 * ks);
+                }
+                // V likewise
+                const int vs = j % kWVStages, vr = j / kWVStages;
+                if (lane == 0 && vr > 0) go = mbar_wait_bounded(v_empty + 8 * vs, (vr - 1) & 1);
+                if (!(ok = __shfl_sync(kFull, go, 0))) break;
+                const uint32_t vdst = base + kWV + vs * kWTile;
+                if (lane == 0) mbar_arrive_expect_tx(v_full + 8 * vs, tx);
+                __syncwarp();
+                if (load) {
+                    tma_load_3d(vdst + off, &tmV, 0, kvh, row, v_full + 8 * vs);
+                    tma_load_3d(vdst + kWChunk + off, &tmV, 64, kvh, row, v_full + 8 * vs);
+                }
+                // V rows with no token: whole blocks not loaded, and the slots past the context
+                // in the sequence's last block (once it has landed)
+                for (int b = 0; b < kWBlocks; ++b) {
+                    if ((loaded >> b) & 1u) continue;
+                    for (int i = lane; i < kBlockSize * 16; i += 32) {
+                        const int r = b * kBlockSize + (i >> 4), c = i & 15;
+                        const uint32_t a = vdst + (c >> 3) * kWChunk + r * 128 + ((c & 7) << 4);
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0) : "memory");
+                    }
+                }
+                const int jt = (ctx % kBlockSize) ? nblk_seq - 1 : -1;
+                const int bt = jt - j * kWBlocks;
+                if (bt >= 0 && bt < kWBlocks && ((loaded >> bt) & 1u)) {
+                    bool landed = true;
+                    if (lane == 0) landed = mbar_wait_bounded(v_full + 8 * vs, vr & 1);
+                    if (!(ok = __shfl_sync(kFull, landed, 0))) break;
+                    const int r0 = ctx % kBlockSize;
+                    for (int i = lane; i < (kBlockSize - r0) * 16; i += 32) {
+                        const int r = bt * kBlockSize + r0 + (i >> 4), c = i & 15;
+                        const uint32_t a = vdst + (c >> 3) * kWChunk + r * 128 + ((c & 7) << 4);
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0) : "memory");
+                    }
+                }
+                fence_proxy_async_smem();  // these generic stores are read by the tensor core
+                __syncwarp();
+                if (lane == 0) mbar_arrive(v_ready + 8 * vs);
+            }
+            if (!ok && lane == 0) {
                 count_error(p.err);
-            const unsigned loaded = __ballot_sync(kFull, load);
-            const int row = id * kBlockSize;
-            const uint32_t off = lane * kBlockSize * 128;
-            const uint32_t tx = __popc(loaded) * 2 * (kBlockSize * 128);
-            // K of this tile into its ring slot, once the products that read the slot's
-            // previous tile are done
-            const int ks = j % kWKStages, kr = j / kWKStages;
-            bool go = true;
-            if (lane == 0 && kr > 0) go = mbar_wait_bounded(k_empty + 8 * ks, (kr - 1) & 1);
-            if (!(ok = __shfl_sync(kFull, go, 0))) break;
-            const uint32_t kdst = base + kWK + ks * kWTile;
-            if (lane == 0) mbar_arrive_expect_tx(k_full + 8 * ks, tx);
-            __syncwarp();
-            if (load) {
-                tma_load_3d(kdst + off, &tmK, 0, kvh, row, k_full + 8 * ks);
-                tma_load_3d(kdst + kWChunk + off, &tmK, 64, kvh, row, k_full + 8 * ks);
+                atomicExch(&abort_sh, 1);
             }
-            // V likewise
-            const int vs = j % kWVStages, vr = j / kWVStages;
-            if (lane == 0 && vr > 0) go = mbar_wait_bounded(v_empty + 8 * vs, (vr - 1) & 1);
-            if (!(ok = __shfl_sync(kFull, go, 0))) break;
-            const uint32_t vdst = base + kWV + vs * kWTile;
-            if (lane == 0) mbar_arrive_expect_tx(v_full + 8 * vs, tx);
-            __syncwarp();
-            if (load) {
-                tma_load_3d(vdst + off, &tmV, 0, kvh, row, v_full + 8 * vs);
-                tma_load_3d(vdst + kWChunk + off, &tmV, 64, kvh, row, v_full + 8 * vs);
+        } else if (warp == kMma) {
+            // ================= MMA issuer (warp-uniform) =================
+            const uint32_t idesc_s = instr_desc_16(kTcRows, kWKeys, false, false);
+            const uint32_t idesc_o = instr_desc_16(kTcRows, kTcD, true, false);
+            // descriptors of an operand's first k-step; a k-step adds its byte offset >> 4 to
+            // the start-address field (all of shared memory is below 2^18 bytes: no carry)
+            const uint64_t dq0 = smem_desc(base, 16, 1024);
+            const uint64_t dk0 = smem_desc(base + kWK, 16, 1024);
+            const uint64_t dv0 = smem_desc(base + kWV, kWChunk, 1024);
+            auto wait_all = [&](uint32_t bar, uint32_t parity) {
+                return __all_sync(kFull, mbar_wait_bounded(bar, parity));
+            };
+            auto issue_s = [&](int t, int j) {
+                tc_fence_after();
+                const uint64_t dk = dk0 + (uint64_t)(((j % kWKStages) * kWTile) >> 4);
+                const uint64_t dq = dq0 + (uint64_t)((t * kTcQBytes) >> 4);
+    #pragma unroll
+                for (int k = 0; k < kTcD / 16; ++k)
+                    umma_ss_e(tmem + kWSCol + t * kWKeys, dq + (uint64_t)((((k >> 2) * kTcQChunk) + (k & 3) * 32) >> 4),
+                              dk + (uint64_t)((((k >> 2) * kWChunk) + (k & 3) * 32) >> 4), idesc_s, k > 0 ? 1u : 0u);
+                umma_commit_e(s_full + 8 * t);
+            };
+            auto issue_pv = [&](int t, int j) {
+                tc_fence_after();
+                const uint64_t dv = dv0 + (uint64_t)(((j % kWVStages) * kWTile) >> 4);
+                // P_t(j) from TMEM over the Q tile's score buffer: 16 keys = 8 columns per k-step
+    #pragma unroll
+                for (int k = 0; k < kWKeys / 16; ++k)
+                    umma_ts_e(tmem + t * kTcD, tmem + kWSCol + t * kWKeys + k * 8, dv + (uint64_t)((k * 16 * 128) >> 4),
+                              idesc_o, (j > 0 || k > 0) ? 1u : 0u);
+            };
+            bool alive = wait_all(q_full, 0) && wait_all(k_full, 0);
+            if (alive) {
+                for (int t = 0; t < kTcQT; ++t)
+                    if (ntq[t] > 0) issue_s(t, 0);
+                umma_commit_e(k_empty);
             }
-            // V rows with no token: whole blocks not loaded, and the slots past the context
-            // in the sequence's last block (once it has landed)
-            for (int b = 0; b < kWBlocks; ++b) {
-                if ((loaded >> b) & 1u) continue;
-                for (int i = lane; i < kBlockSize * 16; i += 32) {
-                    const int r = b * kBlockSize + (i >> 4), c = i & 15;
-                    const uint32_t a = vdst + (c >> 3) * kWChunk + r * 128 + ((c & 7) << 4);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0) : "memory");
+            for (int j = 0; j < ntiles && alive; ++j) {
+                if (__any_sync(kFull, *abort_flag != 0)) break;
+                bool v_in = false, k_in = false;
+                for (int t = 0; t < kTcQT && alive; ++t) {
+                    if (j < ntq[t]) {
+                        alive = wait_all(p_full + 8 * t, j & 1);
+                        // V landed (its own copy barrier) and its empty rows zeroed (producer)
+                        if (alive && !v_in)
+                            alive = wait_all(v_full + 8 * (j % kWVStages), (j / kWVStages) & 1) &&
+                                    wait_all(v_ready + 8 * (j % kWVStages), (j / kWVStages) & 1);
+                        v_in = true;
+                        if (!alive) break;
+                        issue_pv(t, j);
+                        if (j == ntq[t] - 1) umma_commit_e(o_done + 8 * t);
+                    }
+                    if (j + 1 < ntq[t]) {
+                        if (!k_in) alive = wait_all(k_full + 8 * ((j + 1) % kWKStages), ((j + 1) / kWKStages) & 1);
+                        k_in = true;
+                        if (!alive) break;
+                        issue_s(t, j + 1);
+                    }
                 }
+                if (!alive) break;
+                if (j + 1 < ntiles) umma_commit_e(k_empty + 8 * ((j + 1) % kWKStages));
+                umma_commit_e(v_empty + 8 * (j % kWVStages));
             }
-            const int jt = (ctx % kBlockSize) ? nblk_seq - 1 : -1;
-            const int bt = jt - j * kWBlocks;
-            if (bt >= 0 && bt < kWBlocks && ((loaded >> bt) & 1u)) {
-                bool landed = true;
-                if (lane == 0) landed = mbar_wait_bounded(v_full + 8 * vs, vr & 1);
-                if (!(ok = __shfl_sync(kFull, landed, 0))) break;
-                const int r0 = ctx % kBlockSize;
-                for (int i = lane; i < (kBlockSize - r0) * 16; i += 32) {
-                    const int r = bt * kBlockSize + r0 + (i >> 4), c = i & 15;
-                    const uint32_t a = vdst + (c >> 3) * kWChunk + r * 128 + ((c & 7) << 4);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0) : "memory");
-                }
+            if (!alive && lane == 0) {
+                count_error(p.err);
+                atomicExch(&abort_sh, 1);
             }
-            fence_proxy_async_smem();  // these generic stores are read by the tensor core
-            __syncwarp();
-            if (lane == 0) mbar_arrive(v_ready + 8 * vs);
-        }
-        if (!ok && lane == 0) {
-            count_error(p.err);
-            atomicExch(&abort_sh, 1);
-        }
-    } else if (warp == kMma) {
-        // ================= MMA issuer (warp-uniform) =================
-        const uint32_t idesc_s = instr_desc_16(kTcRows, kWKeys, false, false);
-        const uint32_t idesc_o = instr_desc_16(kTcRows, kTcD, true, false);
-        // descriptors of an operand's first k-step; a k-step adds its byte offset >> 4 to
-        // the start-address field (all of shared memory is below 2^18 bytes: no carry)
-        const uint64_t dq0 = smem_desc(base, 16, 1024);
-        const uint64_t dk0 = smem_desc(base + kWK, 16, 1024);
-        const uint64_t dv0 = smem_desc(base + kWV, kWChunk, 1024);
-        auto wait_all = [&](uint32_t bar, uint32_t parity) {
-            return __all_sync(kFull, mbar_wait_bounded(bar, parity));
-        };
-        auto issue_s = [&](int t, int j) {
-            tc_fence_after();
-            const uint64_t dk = dk0 + (uint64_t)(((j % kWKStages) * kWTile) >> 4);
-            const uint64_t dq = dq0 + (uint64_t)((t * kTcQBytes) >> 4);
-#pragma unroll
-            for (int k = 0; k < kTcD / 16; ++k)
-                umma_ss_e(tmem + kWSCol + t * kWKeys, dq + (uint64_t)((((k >> 2) * kTcQChunk) + (k & 3) * 32) >> 4),
-                          dk + (uint64_t)((((k >> 2) * kWChunk) + (k & 3) * 32) >> 4), idesc_s, k > 0 ? 1u : 0u);
-            umma_commit_e(s_full + 8 * t);
-        };
-        auto issue_pv = [&](int t, int j) {
-            tc_fence_after();
-            const uint64_t dv = dv0 + (uint64_t)(((j % kWVStages) * kWTile) >> 4);
-            // P_t(j) from TMEM over the Q tile's score buffer: 16 keys = 8 columns per k-step
-#pragma unroll
-            for (int k = 0; k < kWKeys / 16; ++k)
-                umma_ts_e(tmem + t * kTcD, tmem + kWSCol + t * kWKeys + k * 8, dv + (uint64_t)((k * 16 * 128) >> 4),
-                          idesc_o, (j > 0 || k > 0) ? 1u : 0u);
-        };
-        bool alive = wait_all(q_full, 0) && wait_all(k_full, 0);
-        if (alive) {
-            for (int t = 0; t < kTcQT; ++t)
-                if (ntq[t] > 0) issue_s(t, 0);
-            umma_commit_e(k_empty);
-        }
-        for (int j = 0; j < ntiles && alive; ++j) {
-            if (__any_sync(kFull, *abort_flag != 0)) break;
-            bool v_in = false, k_in = false;
-            for (int t = 0; t < kTcQT && alive; ++t) {
-                if (j < ntq[t]) {
-                    alive = wait_all(p_full + 8 * t, j & 1);
-                    // V landed (its own copy barrier) and its empty rows zeroed (producer)
-                    if (alive && !v_in)
-                        alive = wait_all(v_full + 8 * (j % kWVStages), (j / kWVStages) & 1) &&
-                                wait_all(v_ready + 8 * (j % kWVStages), (j / kWVStages) & 1);
-                    v_in = true;
-                    if (!alive) break;
-                    issue_pv(t, j);
-                    if (j == ntq[t] - 1) umma_commit_e(o_done + 8 * t);
-                }
-                if (j + 1 < ntq[t]) {
-                    if (!k_in) alive = wait_all(k_full + 8 * ((j + 1) % kWKStages), ((j + 1) / kWKStages) & 1);
-                    k_in = true;
-                    if (!alive) break;
-                    issue_s(t, j + 1);
-                }
-            }
-            if (!alive) break;
-            if (j + 1 < ntiles) umma_commit_e(k_empty + 8 * ((j + 1) % kWKStages));
-            umma_commit_e(v_empty + 8 * (j % kWVStages));
-        }
-        if (!alive && lane == 0) {
-            count_error(p.err);
-            atomicExch(&abort_sh, 1);
         }
     } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 200;");
         // ================= softmax: warpgroup t = Q tile t, thread = query row =================
         const int t = warp >> 2;
         const int r = threadIdx.x & 127;
@@ -1201,7 +1210,7 @@ cudaError_t launch_prefill_tc(const CUtensorMap& tmQ, const CUtensorMap& tmK, co
     const int smem = kWSmem + 1024;
     cudaError_t e = cudaFuncSetAttribute(prefill_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(prefill_bf16_kernel, grid, dim3(320), smem, stream, tmQ, tmK, tmV, p);
+    return launch_pdl(prefill_bf16_kernel, grid, dim3(384), smem, stream, tmQ, tmK, tmV, p);
 }
 
 }  // namespace pkv
