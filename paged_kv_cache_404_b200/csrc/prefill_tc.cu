@@ -988,7 +988,7 @@ __global__ void __launch_bounds__(384, 1)
                 tc_fence_after();
                 const uint64_t dk = dk0 + (uint64_t)(((j % kWKStages) * kWTile) >> 4);
                 const uint64_t dq = dq0 + (uint64_t)((t * kTcQBytes) >> 4);
-#pragma unroll
+    #pragma unroll
                 for (int k = 0; k < kTcD / 16; ++k)
                     umma_ss_e(tmem + kWSCol + t * kWKeys, dq + (uint64_t)((((k >> 2) * kTcQChunk) + (k & 3) * 32) >> 4),
                               dk + (uint64_t)((((k >> 2) * kWChunk) + (k & 3) * 32) >> 4), idesc_s, k > 0 ? 1u : 0u);
@@ -998,7 +998,7 @@ __global__ void __launch_bounds__(384, 1)
                 tc_fence_after();
                 const uint64_t dv = dv0 + (uint64_t)(((j % kWVStages) * kWTile) >> 4);
                 // P_t(j) from TMEM over the Q tile's score buffer: 16 keys = 8 columns per k-step
-#pragma unroll
+    #pragma unroll
                 for (int k = 0; k < kWKeys / 16; ++k)
                     umma_ts_e(tmem + t * kTcD, tmem + kWSCol + t * kWKeys + k * 8, dv + (uint64_t)((k * 16 * 128) >> 4),
                               idesc_o, (j > 0 || k > 0) ? 1u : 0u);
