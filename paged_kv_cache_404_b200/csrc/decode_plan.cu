@@ -19,7 +19,7 @@
 namespace pkv {
 
 constexpr int kPlanThreads = 1024;  // at most 32 warps: one slot per warp in the candidate counts
-constexpr int kMaxBuckets = 1024;
+constexpr int kMaxBuckets = 128;  // size classes of the longest-first order (a 4-step scan)
 constexpr int kMaxCandidates = 12;
 
 
@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
     __shared__ int hist[kMaxBuckets];
     __shared__ int own_blocks[kSmemSeqs];  // blocks of sequence s outside its shared prefix
     __shared__ int sub_blocks[kSmemSeqs];  // blocks subgroup q computes for its members
-    __shared__ unsigned long long units_of[kMaxCandidates][32];  // per candidate and warp
+    __shared__ unsigned units_of[kMaxCandidates][32];  // per candidate and warp
     __shared__ int chosen, total_items;
     __shared__ int n_subs, n_members;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -266,22 +266,28 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
     if (fixed_partition > 0) {
         if (tid == 0) chosen = fixed_partition;
     } else {
-        // per candidate, each warp's count in its own slot (no atomics), summed by one warp
+        // per candidate, each warp's count in its own slot (no atomics), summed by one
+        // warp; a warp with no sequence and no subgroup writes zeros.  A thread's count is
+        // capped at 2^26 so that a warp's sum fits 32 bits (one redux instruction): a cap
+        // this far above any target cannot change which candidates reach it.
+        const bool busy = tid - lane < p.num_seqs || tid - lane < num_subs;
 #pragma unroll 1
         for (int c = 0; c < num_candidates; ++c) {
-            const int nb = (min_partition << c) / kBlockSize;
-            unsigned long long v = 0;
-            for (int s = tid; s < p.num_seqs; s += kPlanThreads) v += count_pieces(own(s), nb, mb, geometric);
-            for (int q = tid; q < num_subs; q += kPlanThreads) v += count_pieces(sub(q), nb, mb, geometric);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            unsigned v = 0;
+            if (busy) {
+                const int nb = (min_partition << c) / kBlockSize;
+                unsigned long long n = 0;
+                for (int s = tid; s < p.num_seqs; s += kPlanThreads) n += count_pieces(own(s), nb, mb, geometric);
+                for (int q = tid; q < num_subs; q += kPlanThreads) n += count_pieces(sub(q), nb, mb, geometric);
+                v = __reduce_add_sync(0xffffffffu, (unsigned)min(n, 1ull << 26));
+            }
             if (lane == 0) units_of[c][warp] = v;
         }
         __syncthreads();
         if (warp == 0) {
             int P = min_partition;
             for (int c = num_candidates - 1; c >= 0; --c) {
-                unsigned long long v = lane < kPlanThreads / 32 ? units_of[c][lane] : 0ull;
+                unsigned long long v = lane < kPlanThreads / 32 ? units_of[c][lane] : 0u;
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
                 if (v * (unsigned long long)p.num_kv_heads >= (unsigned long long)target_units) {
