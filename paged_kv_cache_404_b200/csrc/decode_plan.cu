@@ -285,12 +285,18 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
         }
         __syncthreads();
         if (warp == 0) {
+            // with prefix groups, 0.45 of the target: a subgroup's unit carries up to 16
+            // score columns, and each further piece costs the plan and the merge
+            // (measured on a shared-prefix batch: 101 us with 512-token pieces, 109 with
+            // the 256 that the full target leaves)
+            const unsigned long long target =
+                grouped ? (unsigned long long)target_units * 9 / 20 : (unsigned long long)target_units;
             int P = min_partition;
             for (int c = num_candidates - 1; c >= 0; --c) {
                 unsigned long long v = lane < kPlanThreads / 32 ? units_of[c][lane] : 0u;
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                if (v * (unsigned long long)p.num_kv_heads >= (unsigned long long)target_units) {
+                if (v * (unsigned long long)p.num_kv_heads >= target) {
                     P = min_partition << c;
                     break;
                 }
